@@ -1,0 +1,164 @@
+"""fp64 CPU oracle for zero-centred and gated RMSNorm, forward and backward.
+
+TEST INFRASTRUCTURE ONLY.  The parity tests under ``tests/``,
+``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline / reference leg are
+the only callers.  The library (``rollout_parity_b200``) never imports, links or
+runs anything here, and nothing here imports the library: the two share no
+code.  The only module both sides use is the seeded input generator
+(``rollout_parity_b200.workloads``), which holds none of this arithmetic.
+
+What is computed, and where it is defined
+-----------------------------------------
+[PR468] RL-Kernel PR #468, "[WS1][CUDA][Qwen3-Next] Gated RMSNorm CUDA kernel for
+        the GDN block", section "Summary" (the displayed formula for y, and the
+        kernel, activation, rstd and backward bullets).
+[RFC415] RL-Kernel RFC #415 (Gemma-4-31B consistency roadmap), section 4
+        "Numerical contract" (declared accumulator, casts only at epilogues).
+
+For one row x of width H (all values are the stored inputs widened exactly to
+fp64; nothing here rounds to a narrower type):
+
+    ms   = (1/H) * sum_j x_j^2                    mean square over the width
+    rho  = 1 / sqrt(ms + eps)                     the row's rstd
+    xh_j = x_j * rho
+    zero-centred:  y_j = xh_j * (1 + w_j)         weight offset 1
+    gated:         y_j = xh_j * w_j * silu(z_j)   weight offset 0, act = silu
+                   silu(z) = z * s(z),  s(z) = 1 / (1 + exp(-z))
+
+The backward is the exact gradient of L = sum_rj y_rj * dy_rj (plain calculus of
+the forward; [PR468] Summary, "Backward" bullet, states that the gated dx is the
+ungated dx with the gain (w + offset) replaced by (w + offset) * act(z)):
+
+    g_j  = 1 + w_j            (zero-centred)   or   w_j * silu(z_j)   (gated)
+    m    = (1/H) * sum_j g_j * dy_j * xh_j
+    dx_j = rho * (g_j * dy_j - xh_j * m)
+    dz_j = dy_j * xh_j * w_j * s_j * (1 + z_j * (1 - s_j))            (gated)
+    dw_j = sum_r dy_rj * xh_rj                     (zero-centred)
+         = sum_r dy_rj * xh_rj * silu(z_rj)        (gated)
+
+Parity pins (``tests/oracle_pins.py``, run by ``tests/test_oracle_pins.py``,
+with planted mistakes in ``tests/test_oracle_mutations.py``):
+  rstd/forward : constant-row closed form, RMS(xh) == 1 at eps = 0, scale
+                 invariance at eps = 0, w = 0 reduces y to xh, an exact rational
+                 worked example (tests/golden/), sigmoid at ln(k) points.
+  backward     : central finite differences of L (dx, dz, dw), the scale
+                 identity sum_j x_j dx_j = rho * S * eps / (ms + eps), and a
+                 brute-force double loop for dw.
+Every public function below is pinned; none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def _rows(a) -> np.ndarray:
+    a = np.asarray(a, dtype=np.float64)
+    if a.ndim != 2:
+        raise ValueError("expected a [rows, width] array")
+    return a
+
+
+def sigmoid(z):
+    """s(z) = 1 / (1 + exp(-z)) in fp64 ([PR468] Summary, activation bullet)."""
+    z = np.asarray(z, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-z))
+
+
+def silu(z):
+    """silu(z) = z * s(z); "swish" is the same function ([PR468] Summary)."""
+    z = np.asarray(z, dtype=np.float64)
+    return z * sigmoid(z)
+
+
+def rstd(x, eps: float) -> np.ndarray:
+    """rho_r = 1 / sqrt(mean_j x_rj^2 + eps), one value per row ([PR468]
+    Summary, rstd bullet: a sum of squares over the row, then the reciprocal
+    square root of its mean plus eps)."""
+    x = _rows(x)
+    width = x.shape[1]
+    ms = np.sum(x * x, axis=1) / width
+    return 1.0 / np.sqrt(ms + eps)
+
+
+def norm_fwd(x, w, eps: float):
+    """Zero-centred RMSNorm forward: y = x * rho * (1 + w).  Returns (y, rho)."""
+    x = _rows(x)
+    w = np.asarray(w, dtype=np.float64)
+    rho = rstd(x, eps)
+    xh = x * rho[:, None]
+    return xh * (1.0 + w)[None, :], rho
+
+
+def gated_norm_fwd(x, z, w, eps: float):
+    """Gated RMSNorm forward: y = x * rho * w * silu(z), the norm applied before
+    the gate and one group per row.  Returns (y, rho)."""
+    x, z = _rows(x), _rows(z)
+    w = np.asarray(w, dtype=np.float64)
+    rho = rstd(x, eps)
+    xh = x * rho[:, None]
+    return xh * w[None, :] * silu(z), rho
+
+
+def _dx(x, g, dy, rho):
+    width = x.shape[1]
+    xh = x * rho[:, None]
+    m = np.sum(g * dy * xh, axis=1) / width
+    return rho[:, None] * (g * dy - xh * m[:, None])
+
+
+def norm_bwd(x, w, dy, eps: float):
+    """Zero-centred RMSNorm backward.  Returns (dx [rows, width], dw [width])."""
+    x, dy = _rows(x), _rows(dy)
+    w = np.asarray(w, dtype=np.float64)
+    rho = rstd(x, eps)
+    g = np.broadcast_to((1.0 + w)[None, :], x.shape)
+    dx = _dx(x, g, dy, rho)
+    dw = np.sum(dy * (x * rho[:, None]), axis=0)
+    return dx, dw
+
+
+def gated_norm_bwd(x, z, w, dy, eps: float):
+    """Gated RMSNorm backward.  Returns (dx, dz, dw)."""
+    x, z, dy = _rows(x), _rows(z), _rows(dy)
+    w = np.asarray(w, dtype=np.float64)
+    rho = rstd(x, eps)
+    xh = x * rho[:, None]
+    s = sigmoid(z)
+    g = w[None, :] * (z * s)
+    dx = _dx(x, g, dy, rho)
+    dz = dy * xh * w[None, :] * s * (1.0 + z * (1.0 - s))
+    dw = np.sum(dy * xh * (z * s), axis=0)
+    return dx, dz, dw
+
+
+# ---------------------------------------------------------------------------
+# Cancellation scales used by the parity tolerance.  They are not outputs of
+# the method: they give, per element, the size of the largest term that
+# cancels in an fp32 evaluation of dx or dz, so a test can allow for the
+# rounding that cancellation amplifies.
+# ---------------------------------------------------------------------------
+def dx_cancellation_scale(x, w, dy, eps: float, z=None) -> np.ndarray:
+    """max(|rho * g * dy|, |rho * xh * m|) per element (the two terms of dx)."""
+    x, dy = _rows(x), _rows(dy)
+    w = np.asarray(w, dtype=np.float64)
+    rho = rstd(x, eps)
+    xh = x * rho[:, None]
+    if z is None:
+        g = np.broadcast_to((1.0 + w)[None, :], x.shape)
+    else:
+        g = w[None, :] * silu(_rows(z))
+    m = np.sum(g * dy * xh, axis=1) / x.shape[1]
+    a = np.abs(rho[:, None] * g * dy)
+    b = np.abs(rho[:, None] * xh * m[:, None])
+    return np.maximum(a, b)
+
+
+def dz_cancellation_scale(x, z, w, dy, eps: float) -> np.ndarray:
+    """|dy * xh * w * s| * max(1, |z * (1 - s)|) per element."""
+    x, z, dy = _rows(x), _rows(z), _rows(dy)
+    w = np.asarray(w, dtype=np.float64)
+    rho = rstd(x, eps)
+    s = sigmoid(z)
+    lead = np.abs(dy * x * rho[:, None] * w[None, :] * s)
+    return lead * np.maximum(1.0, np.abs(z * (1.0 - s)))

@@ -1,0 +1,296 @@
+"""Pins that tie the fp64 oracle to facts other than itself.
+
+Each ``pin_*`` takes an oracle-like module and raises AssertionError when the
+module disagrees with a closed form, an exact hand-derived worked example, a
+finite-difference derivative, an identity or a brute-force loop.
+``test_oracle_pins.py`` runs them on the real oracle; ``test_oracle_mutations.py``
+plants plausible mistakes in copies of the oracle and checks that at least one
+pin fails for each.
+
+The operators are those of RL-Kernel PR #468 ("[WS1][CUDA][Qwen3-Next] Gated
+RMSNorm CUDA kernel for the GDN block", Summary): zero-centred RMSNorm
+y = x*rstd*(1+w) and gated RMSNorm y = x*rstd*w*silu(z), and their gradients.
+The pages print no worked numeric example, so the worked examples here are
+derived by hand with exact rational arithmetic; the derivations are written out
+next to each one.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+L3 = math.log(3.0)
+
+
+def _close(got, want, rtol=1e-13, atol=1e-15, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    assert got.shape == want.shape, f"{what}: shape {got.shape} != {want.shape}"
+    err = np.abs(got - want)
+    lim = atol + rtol * np.abs(want)
+    assert np.all(err <= lim), f"{what}: max err {err.max():.3e}\n got={got}\nwant={want}"
+
+
+# --------------------------------------------------------------------------
+# worked examples (exact)
+# --------------------------------------------------------------------------
+def pin_worked_example_norm(orc):
+    """H=4, x=[1,2,2,4], eps=0: sum x^2 = 25, ms = 25/4, rho = 2/5,
+    xh = [2/5, 4/5, 4/5, 8/5].  w = [0, 1/2, -1, 1] -> g = 1+w = [1, 3/2, 0, 2],
+    y = xh*g = [2/5, 6/5, 0, 16/5].
+    dy = [1, -1, 2, 1/2]: g*dy = [1, -3/2, 0, 1]; g*dy*xh = [2/5, -6/5, 0, 8/5],
+    sum = 4/5, m = 1/5; xh*m = [2, 4, 4, 8]/25;
+    g*dy - xh*m = [23/25, -83/50, -4/25, 17/25];
+    dx = rho*(...) = [46, -83, -8, 34]/125;  dw = dy*xh = [2/5, -4/5, 8/5, 4/5]."""
+    x = [[1.0, 2.0, 2.0, 4.0]]
+    w = [0.0, 0.5, -1.0, 1.0]
+    dy = [[1.0, -1.0, 2.0, 0.5]]
+    y, rho = orc.norm_fwd(x, w, 0.0)
+    _close(rho, [0.4], what="rho")
+    _close(y, [[0.4, 1.2, 0.0, 3.2]], what="y")
+    _close(orc.rstd(x, 0.0), [0.4], what="rstd")
+    dx, dw = orc.norm_bwd(x, w, dy, 0.0)
+    _close(dx, [[46 / 125, -83 / 125, -8 / 125, 34 / 125]], what="dx")
+    _close(dw, [0.4, -0.8, 1.6, 0.8], what="dw")
+
+
+def pin_worked_example_eps(orc):
+    """eps sits inside the square root, added to the mean square.
+    H=2, x=[3,4]: ms = 25/2; eps = 7/2 -> ms+eps = 16, rho = 1/4, xh = [3/4, 1].
+    w = [1, -1/2] -> g = [2, 1/2], y = [3/2, 1/2].  dy = [1, 1]:
+    g*dy*xh = [3/2, 1/2], m = 2/2 = 1; g*dy - xh*m = [5/4, -1/2];
+    dx = [5/16, -1/8]; dw = dy*xh = [3/4, 1]."""
+    x = [[3.0, 4.0]]
+    w = [1.0, -0.5]
+    dy = [[1.0, 1.0]]
+    y, rho = orc.norm_fwd(x, w, 3.5)
+    _close(rho, [0.25], what="rho")
+    _close(y, [[1.5, 0.5]], what="y")
+    dx, dw = orc.norm_bwd(x, w, dy, 3.5)
+    _close(dx, [[5 / 16, -1 / 8]], what="dx")
+    _close(dw, [0.75, 1.0], what="dw")
+
+
+def pin_worked_example_gated(orc):
+    """Gated, H=4, x=[1,2,2,4], eps=0 (rho=2/5, xh=[2,4,4,8]/5), L = ln 3,
+    z = [L, -L, 0, L] so s(z) = [3/4, 1/4, 1/2, 3/4] and
+    silu(z) = [3L/4, -L/4, 0, 3L/4];  w = [1, 2, 5, -1].
+    y = xh*w*silu = [3L/10, -2L/5, 0, -6L/5].
+    dy = [1, -1, 2, 1/2]: g = w*silu = [3L/4, -L/2, 0, -3L/4];
+    g*dy*xh = [3L/10, 2L/5, 0, -3L/5], sum = L/10, m = L/40;
+    g*dy - xh*m = [37L/50, 12L/25, -L/50, -83L/200];
+    dx = [37L/125, 24L/125, -L/125, -83L/500];
+    dz = dy*xh*w*s*(1+z*(1-s)) = [(3/10)(1+L/4), -(2/5)(1-3L/4), 4, -(3/5)(1+L/4)];
+    dw = dy*xh*silu = [3L/10, L/5, 0, 3L/5]."""
+    L = L3
+    x = [[1.0, 2.0, 2.0, 4.0]]
+    z = [[L, -L, 0.0, L]]
+    w = [1.0, 2.0, 5.0, -1.0]
+    dy = [[1.0, -1.0, 2.0, 0.5]]
+    y, rho = orc.gated_norm_fwd(x, z, w, 0.0)
+    _close(rho, [0.4], what="rho")
+    _close(y, [[3 * L / 10, -2 * L / 5, 0.0, -6 * L / 5]], what="y")
+    dx, dz, dw = orc.gated_norm_bwd(x, z, w, dy, 0.0)
+    _close(dx, [[37 * L / 125, 24 * L / 125, -L / 125, -83 * L / 500]], what="dx")
+    _close(dz, [[0.3 * (1 + L / 4), -0.4 * (1 - 3 * L / 4), 4.0, -0.6 * (1 + L / 4)]],
+           what="dz")
+    _close(dw, [3 * L / 10, L / 5, 0.0, 3 * L / 5], what="dw")
+
+
+def pin_sigmoid_points(orc):
+    """s(ln k) = k/(k+1); s(0) = 1/2; saturates without NaN at +-800."""
+    ks = np.array([1.0, 3.0, 1 / 3, 7.0, 0.125])
+    _close(orc.sigmoid(np.log(ks)), ks / (ks + 1.0), what="sigmoid")
+    _close(orc.silu(np.log(ks)), np.log(ks) * ks / (ks + 1.0), what="silu")
+    s = orc.sigmoid(np.array([800.0, -800.0]))
+    assert s[0] == 1.0 and s[1] == 0.0, s
+    assert np.all(np.isfinite(orc.silu(np.array([800.0, -800.0]))))
+
+
+# --------------------------------------------------------------------------
+# closed forms and invariants on random data
+# --------------------------------------------------------------------------
+def pin_constant_row(orc):
+    """A constant row c gives ms = c^2, so y = c/sqrt(c^2+eps) * (1+w), and
+    gated y = c/sqrt(c^2+eps) * w * silu(z) with silu at exact ln(k) points."""
+    rng = np.random.default_rng(11)
+    H = 16
+    for c in (1e-3, -0.7, 2.5, 40.0):
+        for eps in (0.0, 1e-6, 0.3):
+            x = np.full((1, H), c)
+            w = rng.normal(0.0, 0.5, H)
+            base = c / math.sqrt(c * c + eps)
+            y, rho = orc.norm_fwd(x, w, eps)
+            _close(rho, [1.0 / math.sqrt(c * c + eps)], rtol=1e-14, what="rho")
+            _close(y, base * (1.0 + w)[None, :], rtol=1e-14, what="y")
+            ks = rng.choice([0.25, 1 / 3, 1.0, 3.0, 9.0], size=H)
+            z = np.log(ks)[None, :]
+            silu_exact = np.log(ks) * ks / (ks + 1.0)
+            yg, _ = orc.gated_norm_fwd(x, z, w, eps)
+            _close(yg, base * (w * silu_exact)[None, :], rtol=1e-13, atol=1e-15, what="yg")
+
+
+def pin_unit_rms(orc):
+    """At eps = 0 the normalised row has mean square exactly 1 (mean over H, not
+    H-1), and with w = 0 the zero-centred output is that normalised row."""
+    rng = np.random.default_rng(12)
+    for H in (3, 8, 128):
+        x = rng.normal(0.0, 2.0, (5, H))
+        y, rho = orc.norm_fwd(x, np.zeros(H), 0.0)
+        _close(np.mean(y * y, axis=1), np.ones(5), rtol=1e-14, what="ms(xh)")
+        _close(y, x * rho[:, None], rtol=1e-15, what="xh")
+        yg, rg = orc.gated_norm_fwd(x, np.zeros((5, H)), np.ones(H), 0.0)
+        _close(rg, rho, rtol=0, atol=0, what="gated rstd == plain rstd")
+
+
+def pin_eps_shrinks_rms(orc):
+    """With eps > 0 the normalised row's mean square is ms/(ms+eps)."""
+    rng = np.random.default_rng(13)
+    x = rng.normal(0.0, 0.01, (4, 32))
+    eps = 1e-4
+    ms = np.mean(x * x, axis=1)
+    y, _ = orc.norm_fwd(x, np.zeros(32), eps)
+    _close(np.mean(y * y, axis=1), ms / (ms + eps), rtol=1e-13, what="ms(xh)")
+
+
+def pin_scale_invariance(orc):
+    """At eps = 0 the outputs do not change when a row is scaled by a > 0."""
+    rng = np.random.default_rng(14)
+    x = rng.normal(size=(3, 24))
+    z = rng.normal(size=(3, 24))
+    w = rng.normal(size=24)
+    for a in (1e-3, 0.5, 7.0, 1e4):
+        _close(orc.norm_fwd(a * x, w, 0.0)[0], orc.norm_fwd(x, w, 0.0)[0], rtol=1e-13,
+               atol=1e-14, what="norm y(ax)")
+        _close(orc.gated_norm_fwd(a * x, z, w, 0.0)[0], orc.gated_norm_fwd(x, z, w, 0.0)[0],
+               rtol=1e-13, atol=1e-14, what="gated y(ax)")
+
+
+def pin_scale_identity(orc):
+    """sum_j x_j dx_j = rho * S * eps / (ms + eps), S = sum_j g_j dy_j x_j:
+    the derivative of L along x itself, from y(a x) at eps = 0 being flat.
+    Checked through the zero-centred op (g = 1+w) and the gated op."""
+    rng = np.random.default_rng(15)
+    R, H = 6, 40
+    x = rng.normal(size=(R, H))
+    z = rng.normal(size=(R, H))
+    w = rng.normal(size=H)
+    dy = rng.normal(size=(R, H))
+    for eps in (0.0, 1e-3, 0.5):
+        ms = np.mean(x * x, axis=1)
+        rho = 1.0 / np.sqrt(ms + eps)
+        dx, _ = orc.norm_bwd(x, w, dy, eps)
+        S = np.sum((1.0 + w)[None, :] * dy * x, axis=1)
+        _close(np.sum(x * dx, axis=1), rho * S * eps / (ms + eps), rtol=1e-10, atol=1e-12,
+               what="norm identity")
+        dxg, _, _ = orc.gated_norm_bwd(x, z, w, dy, eps)
+        zs = z / (1.0 + np.exp(-z))
+        Sg = np.sum(w[None, :] * zs * dy * x, axis=1)
+        _close(np.sum(x * dxg, axis=1), rho * Sg * eps / (ms + eps), rtol=1e-10, atol=1e-12,
+               what="gated identity")
+
+
+def _fd(f, a, h=1e-5):
+    """Central differences with one Richardson step, elementwise over ``a``."""
+    g = np.zeros_like(a)
+    it = np.nditer(a, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        def d(step):
+            ap = a.copy(); ap[i] += step
+            am = a.copy(); am[i] -= step
+            return (f(ap) - f(am)) / (2 * step)
+        g[i] = (4 * d(h / 2) - d(h)) / 3
+    return g
+
+
+def pin_finite_differences(orc):
+    """dx, dz, dw equal the numerical gradient of L = sum(y * dy)."""
+    rng = np.random.default_rng(16)
+    R, H, eps = 3, 8, 1e-2
+    x = rng.normal(size=(R, H))
+    z = rng.normal(size=(R, H)) * 2.0
+    w = rng.normal(size=H)
+    dy = rng.normal(size=(R, H))
+
+    def L_norm(x_, w_):
+        return float(np.sum(orc.norm_fwd(x_, w_, eps)[0] * dy))
+
+    def L_gated(x_, z_, w_):
+        return float(np.sum(orc.gated_norm_fwd(x_, z_, w_, eps)[0] * dy))
+
+    dx, dw = orc.norm_bwd(x, w, dy, eps)
+    _close(dx, _fd(lambda a: L_norm(a, w), x), rtol=1e-7, atol=1e-8, what="norm dx")
+    _close(dw, _fd(lambda a: L_norm(x, a), w), rtol=1e-7, atol=1e-8, what="norm dw")
+    dx, dz, dw = orc.gated_norm_bwd(x, z, w, dy, eps)
+    _close(dx, _fd(lambda a: L_gated(a, z, w), x), rtol=1e-7, atol=1e-8, what="gated dx")
+    _close(dz, _fd(lambda a: L_gated(x, a, w), z), rtol=1e-7, atol=1e-8, what="gated dz")
+    _close(dw, _fd(lambda a: L_gated(x, z, a), w), rtol=1e-7, atol=1e-8, what="gated dw")
+
+
+def pin_dw_brute_force(orc):
+    """dw recomputed by an explicit loop over rows and columns, using the
+    per-row forward outputs (dy * y / (1+w) is dy * xh for the zero-centred op;
+    gated: dy * y / w is dy * xh * silu(z))."""
+    rng = np.random.default_rng(17)
+    R, H, eps = 9, 5, 1e-6
+    x = rng.normal(size=(R, H))
+    z = rng.normal(size=(R, H))
+    w = rng.uniform(0.5, 1.5, size=H)          # nonzero so the ratios exist
+    dy = rng.normal(size=(R, H))
+    _, dw = orc.norm_bwd(x, w, dy, eps)
+    _, _, dwg = orc.gated_norm_bwd(x, z, w, dy, eps)
+    want = [0.0] * H
+    want_g = [0.0] * H
+    for r in range(R):
+        y, _ = orc.norm_fwd(x[r:r + 1], w, eps)
+        yg, _ = orc.gated_norm_fwd(x[r:r + 1], z[r:r + 1], w, eps)
+        for j in range(H):
+            want[j] += dy[r, j] * y[0, j] / (1.0 + w[j])
+            want_g[j] += dy[r, j] * yg[0, j] / w[j]
+    _close(dw, want, rtol=1e-12, atol=1e-14, what="norm dw")
+    _close(dwg, want_g, rtol=1e-12, atol=1e-14, what="gated dw")
+
+
+def pin_rows_independent(orc):
+    """Each row's outputs depend only on that row (computed alone == in batch)."""
+    rng = np.random.default_rng(18)
+    x = rng.normal(size=(5, 12)); z = rng.normal(size=(5, 12))
+    w = rng.normal(size=12); dy = rng.normal(size=(5, 12))
+    y, _ = orc.gated_norm_fwd(x, z, w, 1e-6)
+    dx, dz, _ = orc.gated_norm_bwd(x, z, w, dy, 1e-6)
+    for r in range(5):
+        s = slice(r, r + 1)
+        _close(orc.gated_norm_fwd(x[s], z[s], w, 1e-6)[0], y[s], rtol=0, atol=0, what="y row")
+        a, b, _ = orc.gated_norm_bwd(x[s], z[s], w, dy[s], 1e-6)
+        _close(a, dx[s], rtol=0, atol=0, what="dx row")
+        _close(b, dz[s], rtol=0, atol=0, what="dz row")
+
+
+ALL_PINS = [
+    pin_worked_example_norm,
+    pin_worked_example_eps,
+    pin_worked_example_gated,
+    pin_sigmoid_points,
+    pin_constant_row,
+    pin_unit_rms,
+    pin_eps_shrinks_rms,
+    pin_scale_invariance,
+    pin_scale_identity,
+    pin_finite_differences,
+    pin_dw_brute_force,
+    pin_rows_independent,
+]
+
+
+def failing_pins(orc):
+    """Names of the pins that ``orc`` fails (an exception counts as a failure)."""
+    bad = []
+    for p in ALL_PINS:
+        try:
+            with np.errstate(all="ignore"):
+                p(orc)
+        except Exception:  # noqa: BLE001 - any failure of a mutant counts
+            bad.append(p.__name__)
+    return bad

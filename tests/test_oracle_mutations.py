@@ -1,0 +1,177 @@
+"""Planted mistakes in copies of the oracle (CPU only).
+
+Each mutant replaces one function of a freshly loaded copy of
+``oracle/rmsnorm.py`` with a version carrying one plausible mistake -- a dropped
+term, a wrong sign, a wrong divisor, the offset added where it does not belong --
+and the test asserts that at least one pin in ``oracle_pins`` fails for it.
+The real oracle is never modified.
+"""
+import importlib.util
+import os
+
+import numpy as np
+import pytest
+
+import oracle_pins
+
+ORACLE_SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                          "oracle", "rmsnorm.py")
+
+
+def fresh():
+    spec = importlib.util.spec_from_file_location("oracle_mutant", ORACLE_SRC)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def m_eps_outside_sqrt(o):
+    def rstd(x, eps):
+        x = np.asarray(x, dtype=np.float64)
+        return 1.0 / (np.sqrt(np.sum(x * x, axis=1) / x.shape[1]) + eps)
+    o.rstd = rstd
+
+
+def m_mean_over_h_minus_1(o):
+    def rstd(x, eps):
+        x = np.asarray(x, dtype=np.float64)
+        return 1.0 / np.sqrt(np.sum(x * x, axis=1) / (x.shape[1] - 1) + eps)
+    o.rstd = rstd
+
+
+def m_eps_dropped(o):
+    def rstd(x, eps):
+        x = np.asarray(x, dtype=np.float64)
+        return 1.0 / np.sqrt(np.sum(x * x, axis=1) / x.shape[1])
+    o.rstd = rstd
+
+
+def m_no_offset(o):
+    def norm_fwd(x, w, eps):
+        x = np.asarray(x, dtype=np.float64); w = np.asarray(w, dtype=np.float64)
+        rho = o.rstd(x, eps)
+        return x * rho[:, None] * w[None, :], rho
+    o.norm_fwd = norm_fwd
+
+
+def m_gate_sigmoid_not_silu(o):
+    def gated_norm_fwd(x, z, w, eps):
+        x = np.asarray(x, dtype=np.float64); z = np.asarray(z, dtype=np.float64)
+        w = np.asarray(w, dtype=np.float64)
+        rho = o.rstd(x, eps)
+        return x * rho[:, None] * w[None, :] * o.sigmoid(z), rho
+    o.gated_norm_fwd = gated_norm_fwd
+
+
+def m_sigmoid_sign(o):
+    o.sigmoid = lambda z: 1.0 / (1.0 + np.exp(np.asarray(z, dtype=np.float64)))
+
+
+def m_dx_drops_mean_term(o):
+    def _dx(x, g, dy, rho):
+        return rho[:, None] * (g * dy)
+    o._dx = _dx
+
+
+def m_dx_mean_not_divided(o):
+    def _dx(x, g, dy, rho):
+        xh = x * rho[:, None]
+        m = np.sum(g * dy * xh, axis=1)
+        return rho[:, None] * (g * dy - xh * m[:, None])
+    o._dx = _dx
+
+
+def m_dx_drops_rho(o):
+    def _dx(x, g, dy, rho):
+        xh = x * rho[:, None]
+        m = np.sum(g * dy * xh, axis=1) / x.shape[1]
+        return g * dy - xh * m[:, None]
+    o._dx = _dx
+
+
+def m_dx_sign(o):
+    def _dx(x, g, dy, rho):
+        xh = x * rho[:, None]
+        m = np.sum(g * dy * xh, axis=1) / x.shape[1]
+        return rho[:, None] * (g * dy + xh * m[:, None])
+    o._dx = _dx
+
+
+def m_dz_drops_one_minus_s(o):
+    def gated_norm_bwd(x, z, w, dy, eps):
+        x = np.asarray(x, dtype=np.float64); z = np.asarray(z, dtype=np.float64)
+        w = np.asarray(w, dtype=np.float64); dy = np.asarray(dy, dtype=np.float64)
+        rho = o.rstd(x, eps); xh = x * rho[:, None]; s = o.sigmoid(z)
+        dx = o._dx(x, w[None, :] * z * s, dy, rho)
+        dz = dy * xh * w[None, :] * s * (1.0 + z)
+        return dx, dz, np.sum(dy * xh * z * s, axis=0)
+    o.gated_norm_bwd = gated_norm_bwd
+
+
+def m_dz_sigmoid_derivative_only(o):
+    def gated_norm_bwd(x, z, w, dy, eps):
+        x = np.asarray(x, dtype=np.float64); z = np.asarray(z, dtype=np.float64)
+        w = np.asarray(w, dtype=np.float64); dy = np.asarray(dy, dtype=np.float64)
+        rho = o.rstd(x, eps); xh = x * rho[:, None]; s = o.sigmoid(z)
+        dx = o._dx(x, w[None, :] * z * s, dy, rho)
+        dz = dy * xh * w[None, :] * s * (1.0 - s)
+        return dx, dz, np.sum(dy * xh * z * s, axis=0)
+    o.gated_norm_bwd = gated_norm_bwd
+
+
+def m_gated_dw_drops_gate(o):
+    def gated_norm_bwd(x, z, w, dy, eps):
+        x = np.asarray(x, dtype=np.float64); z = np.asarray(z, dtype=np.float64)
+        w = np.asarray(w, dtype=np.float64); dy = np.asarray(dy, dtype=np.float64)
+        rho = o.rstd(x, eps); xh = x * rho[:, None]; s = o.sigmoid(z)
+        dx = o._dx(x, w[None, :] * z * s, dy, rho)
+        dz = dy * xh * w[None, :] * s * (1.0 + z * (1.0 - s))
+        return dx, dz, np.sum(dy * xh, axis=0)
+    o.gated_norm_bwd = gated_norm_bwd
+
+
+def m_gated_gain_adds_offset(o):
+    def gated_norm_bwd(x, z, w, dy, eps):
+        x = np.asarray(x, dtype=np.float64); z = np.asarray(z, dtype=np.float64)
+        w = np.asarray(w, dtype=np.float64); dy = np.asarray(dy, dtype=np.float64)
+        rho = o.rstd(x, eps); xh = x * rho[:, None]; s = o.sigmoid(z)
+        dx = o._dx(x, (1.0 + w[None, :]) * z * s, dy, rho)
+        dz = dy * xh * w[None, :] * s * (1.0 + z * (1.0 - s))
+        return dx, dz, np.sum(dy * xh * z * s, axis=0)
+    o.gated_norm_bwd = gated_norm_bwd
+
+
+def m_norm_dw_uses_x(o):
+    def norm_bwd(x, w, dy, eps):
+        x = np.asarray(x, dtype=np.float64); w = np.asarray(w, dtype=np.float64)
+        dy = np.asarray(dy, dtype=np.float64)
+        rho = o.rstd(x, eps)
+        dx = o._dx(x, np.broadcast_to((1.0 + w)[None, :], x.shape), dy, rho)
+        return dx, np.sum(dy * x, axis=0)
+    o.norm_bwd = norm_bwd
+
+
+def m_norm_dw_wrong_axis(o):
+    def norm_bwd(x, w, dy, eps):
+        x = np.asarray(x, dtype=np.float64); w = np.asarray(w, dtype=np.float64)
+        dy = np.asarray(dy, dtype=np.float64)
+        rho = o.rstd(x, eps)
+        dx = o._dx(x, np.broadcast_to((1.0 + w)[None, :], x.shape), dy, rho)
+        c = dy * x * rho[:, None]
+        return dx, c[-1]          # last row only instead of the sum over rows
+    o.norm_bwd = norm_bwd
+
+
+MUTANTS = [m for name, m in sorted(globals().items()) if name.startswith("m_")]
+
+
+def test_real_oracle_passes_every_pin():
+    assert oracle_pins.failing_pins(fresh()) == []
+
+
+@pytest.mark.parametrize("mutate", MUTANTS, ids=lambda m: m.__name__)
+def test_mutant_is_caught(mutate):
+    o = fresh()
+    mutate(o)
+    bad = oracle_pins.failing_pins(o)
+    assert bad, f"no pin catches {mutate.__name__}"
