@@ -1,0 +1,456 @@
+#!/usr/bin/env python
+"""Benchmark: gated RMSNorm forward + backward on B200, through librn's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = gated_norm_fwd + gated_norm_bwd (the backward kernel and its dw
+fold) over one batch of 262144 rows (8192 tokens x 32 heads) x 128, bf16, with
+1% of channels scaled x50 in x, z and dy (seeded synthetic data).  Prints one
+JSON line on rank 0.
+
+value     = algorithmic HBM bytes of all steps on all ranks / max-over-ranks time
+            (GB/s); the byte model counts each tensor once: forward reads x, z
+            and writes y, rstd; backward reads x, z, dy, rstd and writes dx,
+            dz; w once per call, dw once.
+L2        = four buffer sets rotate (forward on set k%4, backward on set
+            (k+2)%4), so a buffer is touched again only after two steps over
+            other buffers (>= 512 MB, more than the 126 MB L2).
+roofline  = the backward call (k_bwd + its fold launches), the dominant one:
+            its algorithmic bytes / its mean CUDA-event duration, against the
+            measured HBM copy bandwidth.
+e2e       = the same metric through the public Python API with host buffers:
+            every step copies x, z, dy, w from pinned host memory and y, rstd,
+            dx, dz, dw back.
+--impl reference times the fp64 CPU oracle (the repository's checker) on
+the host cores, one bounded row sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from rollout_parity_b200 import workloads  # noqa: E402
+
+METRIC = "gated RMSNorm fwd+bwd HBM GB/s (% of B200 peak), rows/s; invariance pass"
+WORKLOAD = "gated_262144x128_bf16_outliers"
+FALLBACK_HBM_GBS = 6650.0
+SETS = 4
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=6000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def bytes_model(rows, width, esize=2, gated=True):
+    """Algorithmic bytes of one forward call and one backward call."""
+    t = 3 if gated else 2            # forward: x, (z), y
+    b = 5 if gated else 3            # backward: x, (z), dy, dx, (dz)
+    fwd = rows * (t * width * esize + 4) + width * 4
+    bwd = rows * (b * width * esize + 4) + 2 * width * 4
+    return fwd, bwd
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def src_sha():
+    h = hashlib.sha1()
+    for f in ("rollout_parity_b200/csrc/rn.cu", "include/rn.h"):
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:12]
+
+
+def profiled_traffic():
+    """DRAM bytes per backward call from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    want = src_sha()
+    for ln in open(p):
+        kv = dict(t.split("=", 1) for t in ln.split() if "=" in t)
+        if kv.get("unit") == "gated_norm_bwd" and kv.get("source_sha1") == want:
+            return int(kv["dram_bytes_per_call"])
+    return None
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons in the background."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.t0 = self.t1 = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            self.sel = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *self.sel, "--query-gpu=timestamp," + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = []
+        for ln in out.strip().splitlines():
+            f = [s.strip() for s in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                ts = time.mktime(time.strptime(f[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                ts += float("0." + f[0].split(".")[1]) if "." in f[0] else 0.0
+            except Exception:
+                ts = None
+            rows.append((ts, f))
+        inside = [f for ts, f in rows if ts is not None and self.t0 - 0.05 <= ts <= self.t1 + 0.05]
+        use = inside or [f for _, f in rows]
+        sm = [float(f[1]) for f in use if f[1].replace(".", "").isdigit()]
+        mx = [float(f[2]) for f in use if f[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for f in use for n, v in zip(names, f[5:9]) if v.strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(inside), "samples_outside_window": len(rows) - len(inside)}
+
+
+def dist_setup(n):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if n > 1 or world > 1:
+        import datetime
+        import torch.distributed as dist
+        rank = int(os.environ.get("RANK", "0"))
+        local = int(os.environ.get("LOCAL_RANK", str(rank)))
+        return rank, local, world, dist, datetime
+    return 0, 0, 1, None, None
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(a):
+    import rollout_parity_b200 as rn
+    from rollout_parity_b200._lib import DType, check
+
+    rank, local, world, dist, dt_mod = dist_setup(a.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if dist is not None:
+        dist.init_process_group("nccl", timeout=dt_mod.timedelta(seconds=120),
+                                device_id=dev)
+    lib = rn.load()
+
+    host = [workloads.cfg_gated_heads(seed=1000 * rank + s) for s in range(SETS)]
+    R, H, eps = host[0].rows, host[0].width, host[0].eps
+    fwd_b, bwd_b = bytes_model(R, H)
+    step_b = fwd_b + bwd_b
+    nws = lib.norm_bwd_workspace_bytes(R, H)
+    sets = []
+    for wl in host:
+        d = wl.to(dev)
+        sets.append(dict(x=d.x, z=d.z, w=d.w, dy=d.dy, y=torch.empty_like(d.x),
+                         rstd=torch.empty(R, dtype=torch.float32, device=dev),
+                         dx=torch.empty_like(d.x), dz=torch.empty_like(d.x),
+                         dw=torch.empty(H, dtype=torch.float32, device=dev),
+                         ws=torch.empty(nws, dtype=torch.uint8, device=dev)))
+    P = [{k: v.data_ptr() for k, v in s.items()} for s in sets]
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    bf16 = int(DType.BF16)
+
+    def fwd(p):
+        return lib.gated_norm_fwd(R, H, eps, bf16, p["x"], p["z"], p["w"], p["y"], p["rstd"], sp)
+
+    def bwd(p):
+        return lib.gated_norm_bwd(R, H, eps, bf16, p["x"], p["z"], p["w"], p["dy"], p["rstd"],
+                                  p["dx"], p["dz"], p["dw"], p["ws"], nws, sp)
+
+    for p in P:                       # every set gets its rstd before any backward
+        check("gated_norm_fwd", fwd(p))
+    for k in range(a.warmup):
+        check("gated_norm_fwd", fwd(P[k % SETS]))
+        check("gated_norm_bwd", bwd(P[(k + 2) % SETS]))
+    torch.cuda.synchronize()
+
+    K = a.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = Clocks(dev)
+    clocks.start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.mark("t0")
+    t_start.record(stream)
+    for k in range(K):
+        e = ev[k]
+        e[0].record(stream)
+        s1 = fwd(P[k % SETS])
+        e[1].record(stream)
+        s2 = bwd(P[(k + 2) % SETS])
+        e[2].record(stream)
+        if s1 or s2:
+            check("gated_norm_fwd", s1)
+            check("gated_norm_bwd", s2)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark("t1")
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    fwd_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
+    bwd_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
+    if dist is not None:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / K
+    value = world * step_b * K / (ms / 1e3) / 1e9
+    launches = K * (1 + lib.rn_bwd_launches(R, H, bf16))
+
+    inv = invariance_checks(rn, sets[0], R, H, eps) if rank == 0 else None
+    e2e = run_e2e(rn, host[0], dev, a.e2e_steps, step_b, world, dist)
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu = cpu_baseline(host[0], fwd_b, bwd_b)
+
+    if rank == 0:
+        peak, src = peaks()
+        bwd_mean = float(np.mean(bwd_ms))
+        fwd_mean = float(np.mean(fwd_ms))
+        achieved = bwd_b / (bwd_mean / 1e3) / 1e9
+        traffic = profiled_traffic()
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+            "steps": K, "warmup": a.warmup, "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; no dataset or checkpoint)",
+            "config": {"workload": WORKLOAD, "op": "gated RMSNorm fwd+bwd", "rows": R,
+                       "width": H, "layout": "8192 tokens x 32 heads, row = token*32 + head",
+                       "outliers": "1% of channels x50 in x, z, dy", "eps": eps,
+                       "io_dtype": "bf16 x/z/dy/y/dx/dz, fp32 w/rstd/dw", "accumulate": "fp32",
+                       "bytes_per_step": step_b, "parallelism": f"replicas x{world}",
+                       "l2": "4 rotating buffer sets (fwd on k%4, bwd on (k+2)%4): every "
+                             "buffer is re-touched only after >= 512 MB of other traffic "
+                             "(L2 is 126 MB); no flush kernel"},
+            "rows_per_s": round(world * R * K / (ms / 1e3), 1),
+            "pct_of_peak": round(100.0 * value / world / peak, 2),
+            "fwd_us": round(1e3 * fwd_mean, 2), "bwd_us": round(1e3 * bwd_mean, 2),
+            "fwd_gbs": round(fwd_b / (fwd_mean / 1e3) / 1e9, 1),
+            "bwd_gbs": round(achieved, 1),
+            "invariance": inv,
+            "roofline": {"bound": "hbm", "kernel": "gated_norm_bwd call (k_bwd + k_fold passes)",
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "peak_source": src,
+                         "traffic": traffic, "algorithmic_bytes": bwd_b},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+            "source_sha1": src_sha(),
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def invariance_checks(rn, s, R, H, eps):
+    """Bitwise: rows inside the full batch vs the same rows as their own batch,
+    and dw across repeats and launch geometries."""
+    y, rstd = rn.gated_norm_fwd(s["x"], s["z"], s["w"], eps)
+    dx, dz, dw = rn.gated_norm_bwd(s["x"], s["z"], s["w"], s["dy"], rstd, eps)
+    checks, bad = 0, 0
+    for st, n in ((12345, 1), (70001, 7), (R // 2 - 5, 4099), (R - 33, 33)):
+        sl = slice(st, st + n)
+        c = {k: s[k][sl].clone() for k in ("x", "z", "dy")}
+        y2, r2 = rn.gated_norm_fwd(c["x"], c["z"], s["w"], eps)
+        dx2, dz2, _ = rn.gated_norm_bwd(c["x"], c["z"], s["w"], c["dy"], r2, eps)
+        for a, b in ((y[sl], y2), (rstd[sl], r2), (dx[sl], dx2), (dz[sl], dz2)):
+            checks += 1
+            bad += int(not torch.equal(a.view(torch.int16 if a.dtype == torch.bfloat16
+                                              else torch.int32),
+                                       b.view(torch.int16 if b.dtype == torch.bfloat16
+                                              else torch.int32)))
+    for geo in ((0, 0, 0), (148, 1, 8), (7, 2, 64), (0, 0, 0)):
+        rn.rn_test_set_geometry(*geo)
+        _, _, dw2 = rn.gated_norm_bwd(s["x"], s["z"], s["w"], s["dy"], rstd, eps)
+        checks += 1
+        bad += int(not torch.equal(dw.view(torch.int32), dw2.view(torch.int32)))
+    rn.rn_test_set_geometry(0, 0, 0)
+    torch.cuda.synchronize()
+    return {"result": "pass" if bad == 0 else "fail", "bitwise_checks": checks, "failed": bad}
+
+
+def run_e2e(rn, wl, dev, steps, step_b, world, dist):
+    R, H, eps = wl.rows, wl.width, wl.eps
+    pin = lambda t: t.pin_memory()
+    hx, hz, hdy, hw = pin(wl.x), pin(wl.z), pin(wl.dy), pin(wl.w)
+    oy, ors = torch.empty_like(hx).pin_memory(), torch.empty(R, dtype=torch.float32).pin_memory()
+    odx, odz = torch.empty_like(hx).pin_memory(), torch.empty_like(hx).pin_memory()
+    odw = torch.empty(H, dtype=torch.float32).pin_memory()
+    x = torch.empty_like(hx, device=dev)
+    z = torch.empty_like(hx, device=dev)
+    dy = torch.empty_like(hx, device=dev)
+    w = torch.empty_like(hw, device=dev)
+    y = torch.empty_like(x)
+    rstd = torch.empty(R, dtype=torch.float32, device=dev)
+    dx, dz = torch.empty_like(x), torch.empty_like(x)
+    dw = torch.empty(H, dtype=torch.float32, device=dev)
+    ws = rn.workspace(R, H, dev)
+    h2d = sum(t.numel() * t.element_size() for t in (hx, hz, hdy, hw))
+    d2h = sum(t.numel() * t.element_size() for t in (oy, ors, odx, odz, odw))
+
+    def step():
+        x.copy_(hx, non_blocking=True)
+        z.copy_(hz, non_blocking=True)
+        dy.copy_(hdy, non_blocking=True)
+        w.copy_(hw, non_blocking=True)
+        rn.gated_norm_fwd(x, z, w, eps, y=y, rstd=rstd)
+        rn.gated_norm_bwd(x, z, w, dy, rstd, eps, dx=dx, dz=dz, dw=dw, ws=ws)
+        oy.copy_(y, non_blocking=True)
+        ors.copy_(rstd, non_blocking=True)
+        odx.copy_(dx, non_blocking=True)
+        odz.copy_(dz, non_blocking=True)
+        odw.copy_(dw, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e)
+    if dist is not None:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(world * step_b * steps / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 4), "api": "rollout_parity_b200.gated_norm_fwd/bwd"}
+
+
+# ---------------------------------------------------------------------------
+# the fp64 oracle on the host cores
+# ---------------------------------------------------------------------------
+def _oracle_step(orc, x, z, w, dy, eps):
+    orc.gated_norm_fwd(x, z, w, eps)
+    orc.gated_norm_bwd(x, z, w, dy, eps)
+
+
+def cpu_baseline(wl, fwd_b, bwd_b, min_s=10.0, max_s=30.0):
+    import oracle
+    f = workloads.as_f64
+    x, z, w, dy = f(wl.x), f(wl.z), f(wl.w), f(wl.dy)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        _oracle_step(oracle, x, z, w, dy, wl.eps)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_s or el * (reps + 1) / reps > max_s:
+            break
+    return {"value": round((fwd_b + bwd_b) * reps / el / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"fp64 numpy oracle fwd+bwd over all {wl.rows} rows of the workload, "
+                      f"{reps} passes in {el:.1f} s, single thread"}
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(max(1, a.gpus))))
+    if rank != 0:
+        return
+    import oracle
+    wl = workloads.cfg_gated_heads()
+    R, H, eps = wl.rows, wl.width, wl.eps
+    f = workloads.as_f64
+    # size the per-step row sample so the whole run stays near a minute of CPU
+    probe = 4096
+    t0 = time.perf_counter()
+    _oracle_step(oracle, f(wl.x[:probe]), f(wl.z[:probe]), f(wl.w), f(wl.dy[:probe]), eps)
+    per_row = (time.perf_counter() - t0) / probe
+    n = int(60.0 / per_row / max(1, a.steps + a.warmup))
+    n = max(32, min(R, n // 32 * 32))
+    x, z, w, dy = f(wl.x[:n]), f(wl.z[:n]), f(wl.w), f(wl.dy[:n])
+    for _ in range(a.warmup):
+        _oracle_step(oracle, x, z, w, dy, eps)
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        _oracle_step(oracle, x, z, w, dy, eps)
+    el = time.perf_counter() - t0
+    fwd_b, bwd_b = bytes_model(n, H)
+    value = (fwd_b + bwd_b) * a.steps / el / 1e9
+    sample = (f"fp64 numpy oracle fwd+bwd on rows [0, {n}) of the {R}-row workload per step "
+              f"(single thread)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": round(1e3 * el / a.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; no dataset or checkpoint)",
+        "config": {"workload": WORKLOAD, "op": "gated RMSNorm fwd+bwd", "rows": R, "width": H,
+                   "sample_rows_per_step": n},
+        "rows_per_s": round(n * a.steps / el, 1),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,193 @@
+/*
+ * rn.h -- C ABI of librn: batch-invariant zero-centred and gated RMSNorm,
+ * forward and backward, for NVIDIA B200 (sm_100a).
+ *
+ * The operators
+ * -------------
+ * RL-Kernel PR #468, "[WS1][CUDA][Qwen3-Next] Gated RMSNorm CUDA kernel for the
+ * GDN block", section "Summary" defines, per row x of width H:
+ *
+ *   rstd = rsqrt(mean_j(x_j^2) + eps)
+ *   zero-centred:  y_j = x_j * rstd * (1 + w_j)         (weight offset 1)
+ *   gated:         y_j = x_j * rstd * w_j * silu(z_j)   (weight offset 0,
+ *                  norm before gate, one group per row, silu = z * sigmoid(z))
+ *
+ * and the backward (the "Backward" bullet of the same section, and the
+ * calculus of the forward), with g_j = 1 + w_j or w_j * silu(z_j):
+ *
+ *   m     = mean_j(g_j * dy_j * x_j * rstd)
+ *   dx_j  = rstd * (g_j * dy_j - x_j * rstd * m)
+ *   dz_j  = dy_j * x_j * rstd * w_j * s_j * (1 + z_j * (1 - s_j))  (gated)
+ *   dw_j  = sum over rows of dy_j * x_j * rstd [* silu(z_j) when gated]
+ *
+ * Numerical contract (RL-Kernel RFC #415, section 4 "Numerical contract"):
+ *   - every sum accumulates in fp32 and every intermediate is fp32; the only
+ *     narrowing is the round-to-nearest-even store of y, dx, dz;
+ *   - the addition order depends on the width and dtype only: each thread
+ *     adds its own elements in ascending order, a fixed xor butterfly joins
+ *     the lanes of a row, a fixed pairwise tree joins the warps of a row.
+ *     It never depends on the row count, the row's position, the launch
+ *     geometry or the SM count, so a row's y, rstd, dx and dz are bitwise the
+ *     same alone or inside any batch;
+ *   - dw uses no atomics: rows are folded in ascending order inside 32-row
+ *     leaves, and leaves are joined by a level-by-level pairwise tree whose
+ *     shape depends on the row count only (rn_describe prints it); it is
+ *     bitwise the same across runs and launch geometries;
+ *   - unsupported shapes fail closed with a status; there is no fallback.
+ *
+ * Data layout and ownership
+ * -------------------------
+ * x, z, dy, y, dx, dz: row-major contiguous [rows, width] of dtype `dt`
+ *   (RN_BF16 or RN_F32); y, dx, dz take the dtype of x.
+ * w: fp32 [width].  rstd: fp32 [rows].  dw: fp32 [width].
+ * All pointers are DEVICE pointers on the device that is current when the
+ * call is made, and `stream` is a cudaStream_t of that device (NULL = the
+ * legacy default stream).  The caller owns all memory; the library never
+ * allocates, frees or synchronises.  Every call only enqueues work on
+ * `stream` and returns; results are ready when the stream reaches them.
+ *
+ * Errors
+ * ------
+ * Every argument is checked before anything is enqueued.  A failed check
+ * returns its status and enqueues nothing:
+ *   RN_E_ARG       rows < 0 or > 2^36, eps negative or not finite, a required
+ *                  pointer is NULL, or an output overlaps an input or another
+ *                  output;
+ *   RN_E_DTYPE     dt is not RN_BF16 or RN_F32;
+ *   RN_E_WIDTH     width is not a multiple of 8 in [8, 16384];
+ *   RN_E_ALIGN     a tensor pointer is not 16-byte aligned (rstd: 4 bytes);
+ *   RN_E_WORKSPACE the backward's workspace is NULL or smaller than
+ *                  norm_bwd_workspace_bytes(rows, width);
+ *   RN_E_CUDA      a launch failed (rn_last_cuda_error() gives the code).
+ * rows == 0 is valid: the forward enqueues nothing and the backward sets
+ * dw to +0.0.
+ */
+#ifndef RN_H_
+#define RN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RN_OK = 0,
+    RN_E_ARG = 1,
+    RN_E_DTYPE = 2,
+    RN_E_WIDTH = 3,
+    RN_E_ALIGN = 4,
+    RN_E_WORKSPACE = 5,
+    RN_E_CUDA = 6
+} rn_status;
+
+typedef enum {
+    RN_F32 = 0,
+    RN_BF16 = 1
+} rn_dtype;
+
+/* A cudaStream_t, passed as a plain pointer so this header needs no CUDA. */
+typedef void* rn_stream;
+
+/*
+ * Zero-centred RMSNorm forward (PR #468 Summary, with weight offset 1):
+ *   y[r, j] = x[r, j] * rstd[r] * (1 + w[j]).
+ * x: [rows, width] dt, read.  w: [width] fp32, read.  y: [rows, width] dt,
+ * written.  rstd: [rows] fp32, written, or NULL to skip it.
+ */
+rn_status norm_fwd(int64_t rows, int32_t width, float eps, rn_dtype dt,
+                   const void* x, const float* w, void* y, float* rstd,
+                   rn_stream stream);
+
+/*
+ * Gated RMSNorm forward (PR #468 Summary, weight offset 0, act = silu):
+ *   y[r, j] = x[r, j] * rstd[r] * w[j] * silu(z[r, j]).
+ * The offset is never added, so a -0.0 weight keeps its sign.  rstd is
+ * bitwise identical to norm_fwd's for the same x (same reduction).
+ * x, z: [rows, width] dt.  w: [width] fp32.  y: [rows, width] dt.
+ * rstd: [rows] fp32 or NULL.
+ */
+rn_status gated_norm_fwd(int64_t rows, int32_t width, float eps, rn_dtype dt,
+                         const void* x, const void* z, const float* w, void* y,
+                         float* rstd, rn_stream stream);
+
+/*
+ * Bytes of device workspace the backward needs for `rows` x `width`
+ * (fp32 dw partials; independent of dtype and of the launch geometry).
+ * 0 when rows <= 0 or width is unsupported.
+ */
+size_t norm_bwd_workspace_bytes(int64_t rows, int32_t width);
+
+/*
+ * Zero-centred RMSNorm backward.
+ * x, dy: [rows, width] dt, read.  w: [width] fp32, read.
+ * rstd: [rows] fp32 from norm_fwd, read; or NULL to recompute it (bitwise
+ *   the same value norm_fwd writes).
+ * dx: [rows, width] dt, written.  dw: [width] fp32, written (overwritten,
+ *   not accumulated).
+ * ws: device workspace of ws_bytes >= norm_bwd_workspace_bytes(rows, width),
+ *   16-byte aligned; its contents on entry do not matter and are garbage on
+ *   return.
+ */
+rn_status norm_bwd(int64_t rows, int32_t width, float eps, rn_dtype dt,
+                   const void* x, const float* w, const void* dy,
+                   const float* rstd, void* dx, float* dw,
+                   void* ws, size_t ws_bytes, rn_stream stream);
+
+/*
+ * Gated RMSNorm backward: as norm_bwd, plus z ([rows, width] dt, read) and
+ * dz ([rows, width] dt, written).  dz keeps the sign of a -0.0 weight.
+ */
+rn_status gated_norm_bwd(int64_t rows, int32_t width, float eps, rn_dtype dt,
+                         const void* x, const void* z, const float* w,
+                         const void* dy, const float* rstd, void* dx, void* dz,
+                         float* dw, void* ws, size_t ws_bytes, rn_stream stream);
+
+/*
+ * Provenance record (RFC #415 section 4, point 8): a static, NUL-terminated
+ * string naming the kernels, the reduction schedule and tree, and the
+ * accumulator for (width, dt); "unsupported" for an invalid pair.  The
+ * pointer stays valid until the next rn_describe call on the same thread.
+ */
+const char* rn_describe(int32_t width, rn_dtype dt);
+
+/*
+ * Number of kernels one norm_bwd / gated_norm_bwd call with these sizes
+ * enqueues under the current geometry (the backward kernel plus its dw fold
+ * passes); 0 when rows == 0 (dw is cleared with a memset) or the shape is
+ * unsupported.  The forward always enqueues one kernel when rows > 0.
+ */
+int32_t rn_bwd_launches(int64_t rows, int32_t width, rn_dtype dt);
+
+/* Short message for a status code (static string). */
+const char* rn_status_string(rn_status s);
+
+/* The cudaError_t behind this thread's last RN_E_CUDA (0 if none). */
+int rn_last_cuda_error(void);
+
+/*
+ * Test knobs (process-wide; not for production use).  They change how work
+ * is mapped to CTAs -- never the arithmetic -- so results must not change:
+ *   max_ctas        cap on every grid (CTAs loop over the rest); 0 = default.
+ *   leaves_per_cta  32-row leaves one backward CTA folds together (a power
+ *                   of two, clamped to what the width allows); 0 = default.
+ *   fold_rows       rows of partials one fold CTA reduces per pass (a power
+ *                   of two in [8, 256]); 0 = default.
+ * Returns RN_E_ARG for a negative value or a non-power-of-two.
+ */
+rn_status rn_test_set_geometry(int32_t max_ctas, int32_t leaves_per_cta,
+                               int32_t fold_rows);
+
+/*
+ * Test knob: when on, every entry point runs its argument checks and returns
+ * their status without touching the GPU (no CUDA call at all), so the checks
+ * can be exercised on a machine without one.  Off by default.
+ */
+void rn_test_set_validate_only(int32_t on);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RN_H_ */

@@ -1,0 +1,19 @@
+"""Batch-invariant zero-centred and gated RMSNorm (forward + backward) for B200.
+
+The computation lives in librn.so (CUDA kernels for sm_100a behind a C ABI,
+declared in include/rn.h).  This package is its thin binding: ``ops`` has one
+function per C entry point with the same name; ``autograd`` wraps them as
+torch.autograd Functions; ``workloads`` draws seeded synthetic inputs.
+"""
+from ._lib import LIB_PATH, DType, RNError, Status, load  # noqa: F401
+from .ops import (  # noqa: F401
+    gated_norm_bwd,
+    gated_norm_fwd,
+    norm_bwd,
+    norm_bwd_workspace_bytes,
+    norm_fwd,
+    rn_describe,
+    rn_test_set_geometry,
+    rn_test_set_validate_only,
+    workspace,
+)

@@ -1,0 +1,914 @@
+// librn: batch-invariant zero-centred and gated RMSNorm (forward + backward)
+// for B200 (sm_100a).  The operators and their contract are stated in
+// include/rn.h; the sources are RL-Kernel PR #468 ("[WS1][CUDA][Qwen3-Next]
+// Gated RMSNorm CUDA kernel for the GDN block", Summary) and RL-Kernel RFC #415
+// (section 4, "Numerical contract").
+//
+// Design (HBM-bound streaming; no tensor-core work exists on this path):
+//  * A row of width H is owned by a "team" of T threads; each thread owns K
+//    16-byte vectors of the row, vector v = k*T + t, so a team's loads are
+//    contiguous and coalesced.  (T, K) is a function of (H, dtype) only.
+//  * Row reductions (sum of squares, and the backward's dot product) are the
+//    same code everywhere: a thread adds its elements in ascending order with
+//    fused multiply-add into an accumulator that starts at -0.0 (the identity
+//    of IEEE addition, so an empty thread contributes nothing); an xor
+//    butterfly over the team's lanes (offsets min(T,32)/2 ... 1) joins lanes
+//    -- every lane ends with the same bits since a+b == b+a; for T > 32 the
+//    warp results pass through shared memory and every thread applies the
+//    same pairwise tree to them.
+//  * The backward runs one team per 32-row leaf: the team walks its leaf's
+//    rows in ascending order, writes dx (and dz), and keeps the leaf's dw
+//    partial in registers (a left fold started from -0.0, i.e. from the first
+//    row).  The leaves of a CTA (an aligned power-of-two group) are joined in
+//    shared memory by the pairwise tree; the group partials go to the
+//    workspace and a fold kernel joins them with the same tree.  Aligned
+//    power-of-two blocks are perfect subtrees of the level-by-level pairwise
+//    tree, so the bits do not depend on how many leaves a CTA takes, how many
+//    rows a fold pass takes, or the grid size.
+//  * fp32 arithmetic with explicit rounding intrinsics (__fmul_rn, __fadd_rn,
+//    __fmaf_rn, __fdiv_rn, __frcp_rn) wherever the compiler could otherwise
+//    contract or reorder, so the declared order is the executed order.
+//    expf and rsqrtf are CUDA's own (no fast-math build).
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "rn.h"
+
+namespace {
+
+constexpr int kLeafRows = 32;
+constexpr int kFoldRG = 8;          // row groups (warps) per fold CTA
+constexpr int64_t kMaxRows = int64_t(1) << 36;
+constexpr int kMaxGrid = 1 << 20;
+
+// ---------------------------------------------------------------------------
+// element formats: one 16-byte vector holds VE elements
+// ---------------------------------------------------------------------------
+template <int DT>
+struct Fmt;
+
+template <>
+struct Fmt<RN_BF16> {
+  static constexpr int VE = 8;
+  __device__ static __forceinline__ void unpack(const uint4& u, float (&f)[8]) {
+    f[0] = __uint_as_float(u.x << 16); f[1] = __uint_as_float(u.x & 0xffff0000u);
+    f[2] = __uint_as_float(u.y << 16); f[3] = __uint_as_float(u.y & 0xffff0000u);
+    f[4] = __uint_as_float(u.z << 16); f[5] = __uint_as_float(u.z & 0xffff0000u);
+    f[6] = __uint_as_float(u.w << 16); f[7] = __uint_as_float(u.w & 0xffff0000u);
+  }
+  __device__ static __forceinline__ uint32_t pack2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);   // .x (low half) = a
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  __device__ static __forceinline__ uint4 pack(const float (&f)[8]) {
+    return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]),
+                      pack2(f[6], f[7]));
+  }
+};
+
+template <>
+struct Fmt<RN_F32> {
+  static constexpr int VE = 4;
+  __device__ static __forceinline__ void unpack(const uint4& u, float (&f)[4]) {
+    f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+  }
+  __device__ static __forceinline__ uint4 pack(const float (&f)[4]) {
+    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                      __float_as_uint(f[3]));
+  }
+};
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) { return __ldcs(p); }
+__device__ __forceinline__ void st_stream(uint4* p, const uint4& v) { __stcs(p, v); }
+
+// ---------------------------------------------------------------------------
+// arithmetic of one element, written with explicit roundings
+// ---------------------------------------------------------------------------
+// s(z) = 1 / (1 + exp(-z)); silu(z) = z * s(z)   (PR #468 Summary, activation)
+__device__ __forceinline__ float sigmoid_f(float z) {
+  return __frcp_rn(__fadd_rn(1.0f, expf(-z)));
+}
+
+// rstd = rsqrt(ss / H + eps)   (PR #468 Summary, rstd bullet)
+__device__ __forceinline__ float rstd_from_sumsq(float ss, float H, float eps) {
+  return rsqrtf(__fadd_rn(__fdiv_rn(ss, H), eps));
+}
+
+__device__ __forceinline__ float4 add4(const float4& a, const float4& b) {
+  return make_float4(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y), __fadd_rn(a.z, b.z),
+                     __fadd_rn(a.w, b.w));
+}
+
+// ---------------------------------------------------------------------------
+// team reduction: U independent sums at once (one per row in flight)
+// ---------------------------------------------------------------------------
+template <int W>
+__device__ __forceinline__ float pairwise_tree(float (&p)[W]) {
+#pragma unroll
+  for (int s = 1; s < W; s <<= 1) {
+#pragma unroll
+    for (int i = 0; i + s < W; i += 2 * s) p[i] = __fadd_rn(p[i], p[i + s]);
+  }
+  return p[0];
+}
+
+// `red` is this CTA's reduction scratch: 2 phases x teams x U x W floats.
+// For T > 32 all teams of the CTA must call this in lockstep.  `mask` names
+// the lanes of the warp that exist (a CTA may be smaller than a warp).
+template <int T, int U>
+__device__ __forceinline__ void team_sum(float (&v)[U], float* red, int& phase, int team,
+                                         int nteams, unsigned mask) {
+  constexpr int L = T < 32 ? T : 32;
+#pragma unroll
+  for (int o = L / 2; o >= 1; o >>= 1) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) v[u] = __fadd_rn(v[u], __shfl_xor_sync(mask, v[u], o));
+  }
+  if constexpr (T > 32) {
+    constexpr int W = T / 32;
+    const int lane = threadIdx.x & 31;
+    const int wt = (threadIdx.x % T) >> 5;   // warp index inside the team
+    float* buf = red + phase * (nteams * U * W);
+    phase ^= 1;
+    if (lane == 0) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) buf[(team * U + u) * W + wt] = v[u];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float p[W];
+#pragma unroll
+      for (int i = 0; i < W; ++i) p[i] = buf[(team * U + u) * W + i];
+      v[u] = pairwise_tree<W>(p);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// kernels
+// ---------------------------------------------------------------------------
+struct FwdArgs {
+  int64_t rows;
+  int H;
+  float eps;
+  const uint4* x;
+  const uint4* z;
+  const float* w;
+  uint4* y;
+  float* rstd;
+};
+
+struct BwdArgs {
+  int64_t rows;
+  int H;
+  float eps;
+  const uint4* x;
+  const uint4* z;
+  const float* w;
+  const uint4* dy;
+  const float* rstd;
+  uint4* dx;
+  uint4* dz;
+  float* part;      // [groups][H] fp32 group partials (or dw when one group)
+};
+
+template <int T>
+__host__ __device__ constexpr int fwd_block() { return T <= 32 ? 256 : T; }
+template <int T>
+__host__ __device__ constexpr int bwd_max_block() { return T <= 32 ? 8 * T : (T <= 128 ? 256 : T); }
+template <int T>
+__host__ __device__ constexpr int fwd_rows_per_team() { return T <= 32 ? 2 : 1; }
+template <int T>
+__host__ __device__ constexpr int bwd_rows_per_step() { return T <= 32 ? 2 : 1; }
+
+// Loads this thread's gain base: w (gated) or 1 + w (zero-centred).
+template <int VE, int K, int T, bool GATED>
+__device__ __forceinline__ void load_gain(const float* __restrict__ w, int nv, int t,
+                                          float (&g)[K][VE]) {
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const int v = k * T + t;
+#pragma unroll
+    for (int q = 0; q < VE / 4; ++q) {
+      float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (v < nv) f = __ldg(reinterpret_cast<const float4*>(w) + v * (VE / 4) + q);
+      const float a[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) g[k][q * 4 + e] = GATED ? a[e] : __fadd_rn(1.0f, a[e]);
+    }
+  }
+}
+
+template <int DT, int T, int K, bool GATED>
+__global__ void __launch_bounds__(fwd_block<T>())
+k_fwd(const FwdArgs a) {
+  using F = Fmt<DT>;
+  constexpr int VE = F::VE;
+  constexpr int U = fwd_rows_per_team<T>();
+  constexpr int NT = fwd_block<T>() / T;           // teams per CTA
+  constexpr int W = T > 32 ? T / 32 : 1;
+  __shared__ float red[T > 32 ? 2 * NT * U * W : 1];
+  const int team = threadIdx.x / T, t = threadIdx.x % T;
+  const int nv = a.H / VE;
+  const float Hf = float(a.H);
+  const unsigned mask = 0xffffffffu;   // the forward block is always >= 256 threads
+  int phase = 0;
+
+  float gw[K][VE];
+  load_gain<VE, K, T, GATED>(a.w, nv, t, gw);
+
+  const int64_t step = int64_t(gridDim.x) * NT * U;
+  for (int64_t base = int64_t(blockIdx.x) * NT * U; base < a.rows; base += step) {
+    uint4 xr[U][K], zr[U][K];
+    bool act[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t row = base + int64_t(u) * NT + team;
+      act[u] = row < a.rows;
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        const int v = k * T + t;
+        const bool ok = act[u] && v < nv;
+        xr[u][k] = ok ? ld_stream(a.x + row * nv + v) : make_uint4(0, 0, 0, 0);
+        if constexpr (GATED) zr[u][k] = ok ? ld_stream(a.z + row * nv + v) : make_uint4(0, 0, 0, 0);
+      }
+    }
+    // sum of squares: ascending over this thread's elements, fma, from -0.0
+    float ss[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      ss[u] = -0.0f;
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        if (k * T + t < nv) {
+          float f[VE];
+          F::unpack(xr[u][k], f);
+#pragma unroll
+          for (int e = 0; e < VE; ++e) ss[u] = __fmaf_rn(f[e], f[e], ss[u]);
+        }
+      }
+    }
+    team_sum<T, U>(ss, red, phase, team, NT, mask);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t row = base + int64_t(u) * NT + team;
+      const float r = rstd_from_sumsq(ss[u], Hf, a.eps);
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        const int v = k * T + t;
+        if (act[u] && v < nv) {
+          float f[VE], yv[VE];
+          F::unpack(xr[u][k], f);
+          if constexpr (GATED) {
+            float zf[VE];
+            F::unpack(zr[u][k], zf);
+#pragma unroll
+            for (int e = 0; e < VE; ++e) {
+              const float s = sigmoid_f(zf[e]);
+              const float act_z = __fmul_rn(zf[e], s);
+              yv[e] = __fmul_rn(__fmul_rn(__fmul_rn(f[e], r), gw[k][e]), act_z);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < VE; ++e) yv[e] = __fmul_rn(__fmul_rn(f[e], r), gw[k][e]);
+          }
+          st_stream(a.y + row * nv + v, F::pack(yv));
+        }
+      }
+      if (act[u] && t == 0 && a.rstd != nullptr) a.rstd[row] = r;
+    }
+  }
+}
+
+template <int DT, int T, int K, bool GATED>
+__global__ void __launch_bounds__(bwd_max_block<T>())
+k_bwd(const BwdArgs a) {
+  using F = Fmt<DT>;
+  constexpr int VE = F::VE;
+  constexpr int U = bwd_rows_per_step<T>();
+  constexpr int W = T > 32 ? T / 32 : 1;
+  extern __shared__ float dsm[];   // [2][NT][U][W] reduction scratch, then [NT][H] leaves
+  const int NT = blockDim.x / T;   // leaves per CTA (power of two)
+  float* red = dsm;
+  float* leafbuf = dsm + (T > 32 ? 2 * NT * U * W : 0);
+  const int team = threadIdx.x / T, t = threadIdx.x % T;
+  const int nv = a.H / VE;
+  const float Hf = float(a.H);
+  const unsigned mask = blockDim.x >= 32 ? 0xffffffffu : ((1u << blockDim.x) - 1u);
+  int phase = 0;
+
+  float gw[K][VE];
+  load_gain<VE, K, T, GATED>(a.w, nv, t, gw);
+
+  const int64_t n_leaves = (a.rows + kLeafRows - 1) / kLeafRows;
+  const int64_t n_groups = (n_leaves + NT - 1) / NT;
+  for (int64_t grp = blockIdx.x; grp < n_groups; grp += gridDim.x) {
+    const int64_t r0 = (grp * NT + team) * kLeafRows;
+    float acc[K][VE];
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+#pragma unroll
+      for (int e = 0; e < VE; ++e) acc[k][e] = -0.0f;
+
+    for (int i = 0; i < kLeafRows; i += U) {
+      uint4 xr[U][K], zr[U][K], dr[U][K];
+      float rs[U];
+      bool act[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t row = r0 + i + u;
+        act[u] = row < a.rows;
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+          const int v = k * T + t;
+          const bool ok = act[u] && v < nv;
+          xr[u][k] = ok ? ld_stream(a.x + row * nv + v) : make_uint4(0, 0, 0, 0);
+          dr[u][k] = ok ? ld_stream(a.dy + row * nv + v) : make_uint4(0, 0, 0, 0);
+          if constexpr (GATED) zr[u][k] = ok ? ld_stream(a.z + row * nv + v) : make_uint4(0, 0, 0, 0);
+        }
+        rs[u] = (act[u] && a.rstd != nullptr) ? __ldcs(a.rstd + row) : 0.0f;
+      }
+      if (a.rstd == nullptr) {   // uniform branch: recompute exactly as the forward does
+        float ss[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          ss[u] = -0.0f;
+#pragma unroll
+          for (int k = 0; k < K; ++k) {
+            if (k * T + t < nv) {
+              float f[VE];
+              F::unpack(xr[u][k], f);
+#pragma unroll
+              for (int e = 0; e < VE; ++e) ss[u] = __fmaf_rn(f[e], f[e], ss[u]);
+            }
+          }
+        }
+        team_sum<T, U>(ss, red, phase, team, NT, mask);
+#pragma unroll
+        for (int u = 0; u < U; ++u) rs[u] = rstd_from_sumsq(ss[u], Hf, a.eps);
+      }
+
+      // pass 1: the dot sum_j (g_j * dy_j) * xh_j, with xh = x*rstd and
+      // g = 1 + w or w * silu(z); sigmoid(z) is kept for pass 2
+      float sg[U][K][GATED ? VE : 1];
+      float dot[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        dot[u] = -0.0f;
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+          float xf[VE], df[VE], zf[VE];
+          F::unpack(xr[u][k], xf);
+          F::unpack(dr[u][k], df);
+          if constexpr (GATED) F::unpack(zr[u][k], zf);
+          const bool valid = k * T + t < nv;
+#pragma unroll
+          for (int e = 0; e < VE; ++e) {
+            const float xh = __fmul_rn(xf[e], rs[u]);
+            float g;
+            if constexpr (GATED) {
+              sg[u][k][e] = sigmoid_f(zf[e]);
+              g = __fmul_rn(gw[k][e], __fmul_rn(zf[e], sg[u][k][e]));   // w * silu(z)
+            } else {
+              g = gw[k][e];                                              // 1 + w
+            }
+            if (valid) dot[u] = __fmaf_rn(__fmul_rn(g, df[e]), xh, dot[u]);
+          }
+        }
+      }
+      team_sum<T, U>(dot, red, phase, team, NT, mask);
+
+      // pass 2: dx, dz, and the leaf's dw fold (rows in ascending order)
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t row = r0 + i + u;
+        const float m = __fdiv_rn(dot[u], Hf);
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+          const int v = k * T + t;
+          if (act[u] && v < nv) {
+            float xf[VE], df[VE], zf[VE], dxv[VE], dzv[VE];
+            F::unpack(xr[u][k], xf);
+            F::unpack(dr[u][k], df);
+            if constexpr (GATED) F::unpack(zr[u][k], zf);
+#pragma unroll
+            for (int e = 0; e < VE; ++e) {
+              const float xh = __fmul_rn(xf[e], rs[u]);                 // same bits as pass 1
+              const float q = __fmul_rn(df[e], xh);                     // dy * xh
+              if constexpr (GATED) {
+                const float s = sg[u][k][e];
+                const float silu = __fmul_rn(zf[e], s);
+                const float gd = __fmul_rn(__fmul_rn(gw[k][e], silu), df[e]);
+                // dx = rstd * (g*dy - xh*m)
+                dxv[e] = __fmul_rn(rs[u], __fmaf_rn(-xh, m, gd));
+                // dz = dy*xh*w*s*(1 + z*(1-s))
+                const float d1 = __fmaf_rn(zf[e], __fsub_rn(1.0f, s), 1.0f);
+                dzv[e] = __fmul_rn(__fmul_rn(__fmul_rn(q, gw[k][e]), s), d1);
+                acc[k][e] = __fadd_rn(acc[k][e], __fmul_rn(q, silu));
+              } else {
+                const float gd = __fmul_rn(gw[k][e], df[e]);
+                dxv[e] = __fmul_rn(rs[u], __fmaf_rn(-xh, m, gd));
+                acc[k][e] = __fadd_rn(acc[k][e], q);
+              }
+            }
+            st_stream(a.dx + row * nv + v, F::pack(dxv));
+            if constexpr (GATED) st_stream(a.dz + row * nv + v, F::pack(dzv));
+          }
+        }
+      }
+    }
+
+    // join the CTA's leaves (aligned power-of-two group) with the pairwise tree
+    const int64_t rem = n_leaves - grp * NT;
+    const int nl = rem < NT ? int(rem) : NT;
+    float4* out4 = reinterpret_cast<float4*>(a.part + grp * a.H);
+    if (NT == 1) {
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        const int v = k * T + t;
+        if (v < nv) {
+#pragma unroll
+          for (int q = 0; q < VE / 4; ++q)
+            out4[v * (VE / 4) + q] = make_float4(acc[k][4 * q], acc[k][4 * q + 1],
+                                                 acc[k][4 * q + 2], acc[k][4 * q + 3]);
+        }
+      }
+    } else {
+      __syncthreads();   // the previous group's readers of leafbuf are done
+      float4* lb4 = reinterpret_cast<float4*>(leafbuf + team * a.H);
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        const int v = k * T + t;
+        if (v < nv) {
+#pragma unroll
+          for (int q = 0; q < VE / 4; ++q)
+            lb4[v * (VE / 4) + q] = make_float4(acc[k][4 * q], acc[k][4 * q + 1],
+                                                acc[k][4 * q + 2], acc[k][4 * q + 3]);
+        }
+      }
+      __syncthreads();
+      const int H4 = a.H / 4;
+      const float4* all4 = reinterpret_cast<const float4*>(leafbuf);
+      for (int c = threadIdx.x; c < H4; c += blockDim.x) {
+        float4 p[8];
+#pragma unroll
+        for (int l = 0; l < 8; ++l)
+          p[l] = l < NT ? all4[l * H4 + c] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int s = 1; s < 8; s <<= 1) {
+#pragma unroll
+          for (int l = 0; l + s < 8; l += 2 * s)
+            if (l + s < nl) p[l] = add4(p[l], p[l + s]);
+        }
+        out4[c] = p[0];
+      }
+    }
+  }
+}
+
+// One fold pass: out[b] = pairwise tree of in[b*S, min(n, (b+1)*S)), S = kFoldRG * B.
+// CTA = 32 float4 columns x kFoldRG row groups; a thread streams B rows with
+// a binary counter (slot k holds a pending perfect subtree of 2^k rows), the
+// row groups are then joined in shared memory with the same tree.
+template <int B>
+__global__ void __launch_bounds__(32 * kFoldRG)
+k_fold(const float* __restrict__ in, int64_t n, int H, float* __restrict__ out) {
+  constexpr int LB = (B >= 2) + (B >= 4) + (B >= 8) + (B >= 16) + (B >= 32);   // log2 B
+  const int lane = threadIdx.x & 31, rg = threadIdx.x >> 5;
+  const int H4 = H / 4;
+  const int c = blockIdx.y * 32 + lane;
+  const bool col_ok = c < H4;
+  const int64_t start = int64_t(blockIdx.x) * (kFoldRG * B) + int64_t(rg) * B;
+  const int64_t left = n - start;
+  const int cnt = left <= 0 ? 0 : (left >= B ? B : int(left));
+  const float4* in4 = reinterpret_cast<const float4*>(in);
+
+  float4 v[B];
+#pragma unroll
+  for (int i = 0; i < B; ++i)
+    v[i] = (col_ok && i < cnt) ? __ldcg(in4 + (start + i) * H4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+
+  float4 slot[LB + 1];
+#pragma unroll
+  for (int i = 0; i < B; ++i) {
+    if (i < cnt) {
+      float4 cur = v[i];
+#pragma unroll
+      for (int k = 0; k <= LB; ++k) {
+        if ((i >> k) & 1) {
+          cur = add4(slot[k], cur);
+        } else {
+          slot[k] = cur;
+          break;
+        }
+      }
+    }
+  }
+  // remaining pending subtrees, smallest (rightmost) first: acc = slot[k] + acc
+  float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+  bool have = false;
+  if (cnt == B) {
+    res = slot[LB];
+    have = true;
+  } else {
+#pragma unroll
+    for (int k = 0; k < LB; ++k) {
+      if ((cnt >> k) & 1) {
+        res = have ? add4(slot[k], res) : slot[k];
+        have = true;
+      }
+    }
+  }
+  __shared__ float4 sm[kFoldRG][32];
+  sm[rg][lane] = res;
+  __syncthreads();
+  if (rg == 0 && col_ok) {
+    const int64_t left_cta = n - int64_t(blockIdx.x) * (kFoldRG * B);
+    const int64_t ng64 = (left_cta + B - 1) / B;
+    const int ng = ng64 < kFoldRG ? int(ng64) : kFoldRG;
+    float4 p[kFoldRG];
+#pragma unroll
+    for (int g = 0; g < kFoldRG; ++g) p[g] = sm[g][lane];
+#pragma unroll
+    for (int s = 1; s < kFoldRG; s <<= 1) {
+#pragma unroll
+      for (int g = 0; g + s < kFoldRG; g += 2 * s)
+        if (g + s < ng) p[g] = add4(p[g], p[g + s]);
+    }
+    reinterpret_cast<float4*>(out)[int64_t(blockIdx.x) * H4 + c] = p[0];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side: schedule, validation, launch
+// ---------------------------------------------------------------------------
+struct Sched {
+  int T = 0, K = 0;
+};
+
+int pow2ceil(int v) {
+  int p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+bool width_ok(int32_t width) { return width >= 8 && width <= 16384 && width % 8 == 0; }
+
+// (T, K) as a function of the width and dtype only -- this is the reduction
+// schedule, so it must never look at the row count or a pointer.
+bool pick_sched(int32_t width, rn_dtype dt, Sched* s) {
+  if (!width_ok(width) || (dt != RN_BF16 && dt != RN_F32)) return false;
+  const int VE = dt == RN_BF16 ? 8 : 4;
+  const int nv = width / VE;
+  if (nv <= 32) { s->T = pow2ceil(nv); s->K = 1; }
+  else if (nv <= 128) { s->T = 32; s->K = (nv + 31) / 32; }
+  else if (nv <= 512) { s->T = 128; s->K = (nv + 127) / 128; }
+  else if (nv <= 2048) { s->T = 512; s->K = (nv + 511) / 512; }
+  else { s->T = 1024; s->K = (nv + 1023) / 1024; }
+  return true;
+}
+
+int bwd_max_block_rt(int T) { return T <= 32 ? 8 * T : (T <= 128 ? 256 : T); }
+int bwd_rows_per_step_rt(int T) { return T <= 32 ? 2 : 1; }
+int fwd_block_rt(int T) { return T <= 32 ? 256 : T; }
+int fwd_rows_per_cta_rt(int T) { return T <= 32 ? (256 / T) * 2 : 1; }
+
+std::atomic<int> g_max_ctas{0}, g_leaves_per_cta{0}, g_fold_rows{0}, g_validate_only{0};
+thread_local int t_last_cuda = 0;
+thread_local char t_describe[512];
+
+int leaves_per_cta(const Sched& s, int width) {
+  const int maxb = bwd_max_block_rt(s.T);
+  int lpc = maxb / s.T;                                   // default: fill the block
+  if (s.T > 32 && width > 2048) lpc = 1;                  // keep leaf staging <= 16 KB
+  const int req = g_leaves_per_cta.load();
+  if (req > 0) lpc = req < lpc ? req : lpc;
+  if (lpc > 8) lpc = 8;
+  return lpc;
+}
+
+size_t bwd_smem_bytes(const Sched& s, int lpc, int width) {
+  const int U = bwd_rows_per_step_rt(s.T);
+  const int W = s.T > 32 ? s.T / 32 : 1;
+  size_t f = (s.T > 32 ? size_t(2) * lpc * U * W : 0) + (lpc > 1 ? size_t(lpc) * width : 0);
+  return f * sizeof(float);
+}
+
+int grid_cap(int64_t want) {
+  int64_t cap = kMaxGrid;
+  const int req = g_max_ctas.load();
+  if (req > 0 && req < cap) cap = req;
+  if (want < 1) want = 1;
+  return int(want < cap ? want : cap);
+}
+
+int64_t n_leaves_of(int64_t rows) { return (rows + kLeafRows - 1) / kLeafRows; }
+
+size_t ws_bytes_of(int64_t rows, int32_t width) {
+  if (rows <= 0 || rows > kMaxRows || !width_ok(width)) return 0;
+  const int64_t g0 = n_leaves_of(rows);
+  const int64_t g1 = (g0 + kFoldRG - 1) / kFoldRG;
+  return size_t(g0 + g1) * size_t(width) * sizeof(float);
+}
+
+struct Range {
+  const void* p;
+  size_t n;
+};
+
+bool overlap(const Range& a, const Range& b) {
+  if (!a.p || !b.p || a.n == 0 || b.n == 0) return false;
+  const uintptr_t a0 = uintptr_t(a.p), b0 = uintptr_t(b.p);
+  return a0 < b0 + b.n && b0 < a0 + a.n;
+}
+
+bool aligned16(const void* p) { return (uintptr_t(p) & 15u) == 0; }
+
+rn_status common_checks(int64_t rows, int32_t width, float eps, rn_dtype dt) {
+  if (rows < 0 || rows > kMaxRows || !std::isfinite(eps) || eps < 0.0f) return RN_E_ARG;
+  if (dt != RN_BF16 && dt != RN_F32) return RN_E_DTYPE;
+  if (!width_ok(width)) return RN_E_WIDTH;
+  return RN_OK;
+}
+
+// inputs: read-only ranges; outputs: written ranges.  Outputs must not overlap
+// anything else; inputs may overlap one another.
+rn_status check_ranges(const Range* in, int nin, const Range* out, int nout) {
+  for (int i = 0; i < nout; ++i) {
+    for (int j = 0; j < nin; ++j)
+      if (overlap(out[i], in[j])) return RN_E_ARG;
+    for (int j = i + 1; j < nout; ++j)
+      if (overlap(out[i], out[j])) return RN_E_ARG;
+  }
+  return RN_OK;
+}
+
+rn_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    t_last_cuda = int(e);
+    return RN_E_CUDA;
+  }
+  return RN_OK;
+}
+
+// ---- dispatch over the (T, K) pairs pick_sched can return -----------------
+#define RN_TK_LIST(X) \
+  X(1, 1) X(2, 1) X(4, 1) X(8, 1) X(16, 1) X(32, 1) X(32, 2) X(32, 3) X(32, 4) \
+  X(128, 2) X(128, 3) X(128, 4) X(512, 2) X(512, 3) X(512, 4) X(1024, 3) X(1024, 4)
+
+template <int DT, bool GATED>
+rn_status launch_fwd(const Sched& s, const FwdArgs& a, cudaStream_t st) {
+  const int64_t per_cta = fwd_rows_per_cta_rt(s.T);
+  const int grid = grid_cap((a.rows + per_cta - 1) / per_cta);
+  const int block = fwd_block_rt(s.T);
+#define RN_FWD_CASE(T_, K_)                                                     \
+  if (s.T == T_ && s.K == K_) {                                                 \
+    k_fwd<DT, T_, K_, GATED><<<grid, block, 0, st>>>(a);                        \
+    return launch_status();                                                     \
+  }
+  RN_TK_LIST(RN_FWD_CASE)
+#undef RN_FWD_CASE
+  return RN_E_WIDTH;
+}
+
+template <int DT, bool GATED>
+rn_status launch_bwd(const Sched& s, int lpc, const BwdArgs& a, int64_t groups, cudaStream_t st) {
+  const int grid = grid_cap(groups);
+  const int block = lpc * s.T;
+  const size_t smem = bwd_smem_bytes(s, lpc, a.H);
+#define RN_BWD_CASE(T_, K_)                                                     \
+  if (s.T == T_ && s.K == K_) {                                                 \
+    k_bwd<DT, T_, K_, GATED><<<grid, block, smem, st>>>(a);                     \
+    return launch_status();                                                     \
+  }
+  RN_TK_LIST(RN_BWD_CASE)
+#undef RN_BWD_CASE
+  return RN_E_WIDTH;
+}
+
+int fold_rows_default(int64_t n) {
+  int64_t s = 8;
+  while (s < n && s < 256) s <<= 1;
+  return int(s);
+}
+
+int fold_passes(int64_t n) {
+  int passes = 0;
+  while (n > 1) {
+    int S = g_fold_rows.load();
+    if (S <= 0) S = fold_rows_default(n);
+    n = (n + S - 1) / S;
+    ++passes;
+  }
+  return passes;
+}
+
+// Folds n group partials (rows of width H in `a`) into dw, ping-ponging
+// between the two workspace regions a and b.
+rn_status run_fold(float* a, float* b, int64_t n, int H, float* dw, cudaStream_t st) {
+  float* src = a;
+  float* dst = b;
+  while (n > 1) {
+    int S = g_fold_rows.load();
+    if (S <= 0) S = fold_rows_default(n);
+    const int B = S / kFoldRG;
+    const int64_t nout = (n + S - 1) / S;
+    float* o = nout == 1 ? dw : dst;
+    const int gy = (H / 4 + 31) / 32;    // <= 128 column tiles
+    if (nout > 0x7fffffff) return RN_E_ARG;   // unreachable for rows <= 2^36
+    dim3 grid(unsigned(nout), gy);
+    switch (B) {
+      case 1: k_fold<1><<<grid, 32 * kFoldRG, 0, st>>>(src, n, H, o); break;
+      case 2: k_fold<2><<<grid, 32 * kFoldRG, 0, st>>>(src, n, H, o); break;
+      case 4: k_fold<4><<<grid, 32 * kFoldRG, 0, st>>>(src, n, H, o); break;
+      case 8: k_fold<8><<<grid, 32 * kFoldRG, 0, st>>>(src, n, H, o); break;
+      case 16: k_fold<16><<<grid, 32 * kFoldRG, 0, st>>>(src, n, H, o); break;
+      case 32: k_fold<32><<<grid, 32 * kFoldRG, 0, st>>>(src, n, H, o); break;
+      default: return RN_E_ARG;
+    }
+    const rn_status e = launch_status();
+    if (e != RN_OK) return e;
+    n = nout;
+    float* tmp = src;
+    src = dst;
+    dst = tmp;
+  }
+  return RN_OK;
+}
+
+template <bool GATED>
+rn_status bwd_entry(int64_t rows, int32_t width, float eps, rn_dtype dt, const void* x,
+                    const void* z, const float* w, const void* dy, const float* rstd, void* dx,
+                    void* dz, float* dw, void* ws, size_t ws_bytes, rn_stream stream) {
+  rn_status e = common_checks(rows, width, eps, dt);
+  if (e != RN_OK) return e;
+  if (!w || !dw) return RN_E_ARG;
+  if (rows > 0 && (!x || !dy || !dx || (GATED && (!z || !dz)))) return RN_E_ARG;
+  const size_t esz = dt == RN_BF16 ? 2 : 4;
+  const size_t tb = rows > 0 ? size_t(rows) * size_t(width) * esz : 0;
+  const size_t need = ws_bytes_of(rows, width);
+  if (rows > 0) {
+    if (!aligned16(x) || !aligned16(dy) || !aligned16(dx) || !aligned16(w) || !aligned16(dw) ||
+        (GATED && (!aligned16(z) || !aligned16(dz))) || (uintptr_t(rstd) & 3u))
+      return RN_E_ALIGN;
+    if (!ws || ws_bytes < need) return RN_E_WORKSPACE;
+    if (!aligned16(ws)) return RN_E_ALIGN;
+  } else if ((uintptr_t(dw) & 3u) != 0) {
+    return RN_E_ALIGN;
+  }
+  const Range in[] = {{x, tb}, {GATED ? z : nullptr, tb}, {w, size_t(width) * 4},
+                      {dy, tb}, {rstd, rstd ? size_t(rows) * 4 : 0}};
+  const Range out[] = {{dx, tb}, {GATED ? dz : nullptr, tb}, {dw, size_t(width) * 4},
+                       {ws, rows > 0 ? need : 0}};
+  e = check_ranges(in, 5, out, 4);
+  if (e != RN_OK) return e;
+  if (g_validate_only.load()) return RN_OK;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (rows == 0) {
+    if (cudaMemsetAsync(dw, 0, size_t(width) * sizeof(float), st) != cudaSuccess)
+      return launch_status();
+    return RN_OK;
+  }
+  Sched s;
+  pick_sched(width, dt, &s);
+  const int lpc = leaves_per_cta(s, width);
+  const int64_t leaves = n_leaves_of(rows);
+  const int64_t groups = (leaves + lpc - 1) / lpc;
+  float* region_a = static_cast<float*>(ws);
+  float* region_b = region_a + size_t(leaves) * width;
+  BwdArgs a{rows, width, eps, static_cast<const uint4*>(x), static_cast<const uint4*>(z), w,
+            static_cast<const uint4*>(dy), rstd, static_cast<uint4*>(dx), static_cast<uint4*>(dz),
+            groups == 1 ? dw : region_a};
+  if (dt == RN_BF16)
+    e = launch_bwd<RN_BF16, GATED>(s, lpc, a, groups, st);
+  else
+    e = launch_bwd<RN_F32, GATED>(s, lpc, a, groups, st);
+  if (e != RN_OK) return e;
+  if (groups == 1) return RN_OK;
+  return run_fold(region_a, region_b, groups, width, dw, st);
+}
+
+template <bool GATED>
+rn_status fwd_entry(int64_t rows, int32_t width, float eps, rn_dtype dt, const void* x,
+                    const void* z, const float* w, void* y, float* rstd, rn_stream stream) {
+  rn_status e = common_checks(rows, width, eps, dt);
+  if (e != RN_OK) return e;
+  if (!w) return RN_E_ARG;
+  if (rows > 0 && (!x || !y || (GATED && !z))) return RN_E_ARG;
+  const size_t esz = dt == RN_BF16 ? 2 : 4;
+  const size_t tb = rows > 0 ? size_t(rows) * size_t(width) * esz : 0;
+  if (rows > 0 && (!aligned16(x) || !aligned16(y) || !aligned16(w) ||
+                   (GATED && !aligned16(z)) || (uintptr_t(rstd) & 3u)))
+    return RN_E_ALIGN;
+  const Range in[] = {{x, tb}, {GATED ? z : nullptr, tb}, {w, size_t(width) * 4}};
+  const Range out[] = {{y, tb}, {rstd, rstd ? size_t(rows) * 4 : 0}};
+  e = check_ranges(in, 3, out, 2);
+  if (e != RN_OK) return e;
+  if (g_validate_only.load() || rows == 0) return RN_OK;
+  Sched s;
+  pick_sched(width, dt, &s);
+  FwdArgs a{rows, width, eps, static_cast<const uint4*>(x), static_cast<const uint4*>(z), w,
+            static_cast<uint4*>(y), rstd};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == RN_BF16) return launch_fwd<RN_BF16, GATED>(s, a, st);
+  return launch_fwd<RN_F32, GATED>(s, a, st);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// C ABI
+// ---------------------------------------------------------------------------
+extern "C" {
+
+rn_status norm_fwd(int64_t rows, int32_t width, float eps, rn_dtype dt, const void* x,
+                   const float* w, void* y, float* rstd, rn_stream stream) {
+  return fwd_entry<false>(rows, width, eps, dt, x, nullptr, w, y, rstd, stream);
+}
+
+rn_status gated_norm_fwd(int64_t rows, int32_t width, float eps, rn_dtype dt, const void* x,
+                         const void* z, const float* w, void* y, float* rstd, rn_stream stream) {
+  return fwd_entry<true>(rows, width, eps, dt, x, z, w, y, rstd, stream);
+}
+
+size_t norm_bwd_workspace_bytes(int64_t rows, int32_t width) { return ws_bytes_of(rows, width); }
+
+rn_status norm_bwd(int64_t rows, int32_t width, float eps, rn_dtype dt, const void* x,
+                   const float* w, const void* dy, const float* rstd, void* dx, float* dw,
+                   void* ws, size_t ws_bytes, rn_stream stream) {
+  return bwd_entry<false>(rows, width, eps, dt, x, nullptr, w, dy, rstd, dx, nullptr, dw, ws,
+                          ws_bytes, stream);
+}
+
+rn_status gated_norm_bwd(int64_t rows, int32_t width, float eps, rn_dtype dt, const void* x,
+                         const void* z, const float* w, const void* dy, const float* rstd,
+                         void* dx, void* dz, float* dw, void* ws, size_t ws_bytes,
+                         rn_stream stream) {
+  return bwd_entry<true>(rows, width, eps, dt, x, z, w, dy, rstd, dx, dz, dw, ws, ws_bytes,
+                         stream);
+}
+
+const char* rn_describe(int32_t width, rn_dtype dt) {
+  Sched s;
+  if (!pick_sched(width, dt, &s)) return "unsupported";
+  const int VE = dt == RN_BF16 ? 8 : 4;
+  const int lpc = leaves_per_cta(s, width);
+  std::snprintf(t_describe, sizeof t_describe,
+                "backend=cuda-sm100a lib=librn kernels=k_fwd,k_bwd,k_fold dtype=%s width=%d "
+                "acc=fp32 team_threads=%d vectors_per_thread=%d elems_per_vector=%d "
+                "thread_order=ascending-fma-from-neg0 lane_join=xor-butterfly(%d..1) "
+                "warp_join=%s dw_tree=leaf32-ascending-fold+level-pairwise "
+                "leaves_per_cta=%d fast_math=off atomics=none",
+                dt == RN_BF16 ? "bf16" : "f32", width, s.T, s.K, VE, (s.T < 32 ? s.T : 32) / 2,
+                s.T > 32 ? "smem-pairwise" : "none", lpc);
+  return t_describe;
+}
+
+int32_t rn_bwd_launches(int64_t rows, int32_t width, rn_dtype dt) {
+  Sched s;
+  if (rows <= 0 || rows > kMaxRows || !pick_sched(width, dt, &s)) return 0;
+  const int lpc = leaves_per_cta(s, width);
+  const int64_t groups = (n_leaves_of(rows) + lpc - 1) / lpc;
+  return 1 + fold_passes(groups);
+}
+
+const char* rn_status_string(rn_status s) {
+  switch (s) {
+    case RN_OK: return "ok";
+    case RN_E_ARG: return "invalid argument (rows, eps, NULL pointer or overlapping buffers)";
+    case RN_E_DTYPE: return "unsupported dtype";
+    case RN_E_WIDTH: return "unsupported width (need a multiple of 8 in [8, 16384])";
+    case RN_E_ALIGN: return "misaligned pointer (need 16 bytes; rstd 4 bytes)";
+    case RN_E_WORKSPACE: return "workspace missing or too small";
+    case RN_E_CUDA: return "CUDA launch failed";
+  }
+  return "unknown status";
+}
+
+int rn_last_cuda_error(void) { return t_last_cuda; }
+
+rn_status rn_test_set_geometry(int32_t max_ctas, int32_t leaves_per_cta_req, int32_t fold_rows) {
+  auto pow2 = [](int v) { return v > 0 && (v & (v - 1)) == 0; };
+  if (max_ctas < 0 || leaves_per_cta_req < 0 || fold_rows < 0) return RN_E_ARG;
+  if (leaves_per_cta_req > 0 && !pow2(leaves_per_cta_req)) return RN_E_ARG;
+  if (fold_rows > 0 && (!pow2(fold_rows) || fold_rows < 8 || fold_rows > 256)) return RN_E_ARG;
+  g_max_ctas.store(max_ctas);
+  g_leaves_per_cta.store(leaves_per_cta_req);
+  g_fold_rows.store(fold_rows);
+  return RN_OK;
+}
+
+void rn_test_set_validate_only(int32_t on) { g_validate_only.store(on ? 1 : 0); }
+
+}  // extern "C"

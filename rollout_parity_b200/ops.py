@@ -1,0 +1,177 @@
+"""Python binding of librn, one function per C entry point, same names.
+
+These functions only marshal arguments: they check that torch tensors can be
+described by plain pointers (CUDA, contiguous, the right dtype and shape),
+allocate outputs the caller did not pass (torch is used for device memory and
+streams only), and call the C ABI on the tensors' device and current stream.
+Every step of the computation runs in librn's kernels; a failed status raises
+RNError.
+"""
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from ._lib import DType, check, load
+
+_DT = {torch.bfloat16: DType.BF16, torch.float32: DType.F32}
+
+
+def _dt(x: torch.Tensor) -> DType:
+    if x.dtype not in _DT:
+        raise TypeError(f"x dtype {x.dtype} not supported (bf16 or fp32)")
+    return _DT[x.dtype]
+
+
+def _mat(name: str, t: Optional[torch.Tensor], like: torch.Tensor) -> torch.Tensor:
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.device != like.device or t.dtype != like.dtype or tuple(t.shape) != tuple(like.shape):
+        raise ValueError(f"{name} must be {tuple(like.shape)} {like.dtype} on {like.device}, "
+                         f"got {tuple(t.shape)} {t.dtype} on {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _vec(name: str, t: Optional[torch.Tensor], n: int, device) -> torch.Tensor:
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.device != device or t.dtype != torch.float32 or tuple(t.shape) != (n,) \
+            or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous fp32 [{n}] tensor on {device}")
+    return t
+
+
+def _rows_width(x: torch.Tensor) -> Tuple[int, int]:
+    if x.dim() != 2:
+        raise ValueError("x must be [rows, width]")
+    if not x.is_cuda:
+        raise ValueError("x must be a CUDA tensor")
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    return int(x.shape[0]), int(x.shape[1])
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(x: torch.Tensor, stream) -> int:
+    s = torch.cuda.current_stream(x.device) if stream is None else stream
+    return s.cuda_stream
+
+
+def norm_bwd_workspace_bytes(rows: int, width: int) -> int:
+    return int(load().norm_bwd_workspace_bytes(rows, width))
+
+
+def workspace(rows: int, width: int, device) -> torch.Tensor:
+    """A device buffer large enough for the backward's dw partials."""
+    n = norm_bwd_workspace_bytes(rows, width)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def norm_fwd(x: torch.Tensor, w: torch.Tensor, eps: float = 1e-6, *,
+             y: Optional[torch.Tensor] = None, rstd: Optional[torch.Tensor] = None,
+             want_rstd: bool = True, stream=None):
+    """Zero-centred RMSNorm forward.  Returns (y, rstd); rstd is None when
+    want_rstd is False and none was passed."""
+    rows, width = _rows_width(x)
+    _vec("w", w, width, x.device)
+    y = torch.empty_like(x) if y is None else _mat("y", y, x)
+    if rstd is None and want_rstd:
+        rstd = torch.empty(rows, dtype=torch.float32, device=x.device)
+    if rstd is not None:
+        _vec("rstd", rstd, rows, x.device)
+    with torch.cuda.device(x.device):
+        check("norm_fwd", load().norm_fwd(rows, width, eps, _dt(x), _ptr(x), _ptr(w), _ptr(y),
+                                          _ptr(rstd), _stream(x, stream)))
+    return y, rstd
+
+
+def gated_norm_fwd(x: torch.Tensor, z: torch.Tensor, w: torch.Tensor, eps: float = 1e-6, *,
+                   y: Optional[torch.Tensor] = None, rstd: Optional[torch.Tensor] = None,
+                   want_rstd: bool = True, stream=None):
+    """Gated RMSNorm forward.  Returns (y, rstd)."""
+    rows, width = _rows_width(x)
+    _mat("z", z, x)
+    _vec("w", w, width, x.device)
+    y = torch.empty_like(x) if y is None else _mat("y", y, x)
+    if rstd is None and want_rstd:
+        rstd = torch.empty(rows, dtype=torch.float32, device=x.device)
+    if rstd is not None:
+        _vec("rstd", rstd, rows, x.device)
+    with torch.cuda.device(x.device):
+        check("gated_norm_fwd",
+              load().gated_norm_fwd(rows, width, eps, _dt(x), _ptr(x), _ptr(z), _ptr(w), _ptr(y),
+                                    _ptr(rstd), _stream(x, stream)))
+    return y, rstd
+
+
+def _ws(rows, width, device, ws):
+    if ws is None:
+        ws = workspace(rows, width, device)
+    if ws.device != device or not ws.is_contiguous():
+        raise ValueError("ws must be a contiguous buffer on the tensors' device")
+    return ws, ws.numel() * ws.element_size()
+
+
+def norm_bwd(x: torch.Tensor, w: torch.Tensor, dy: torch.Tensor,
+             rstd: Optional[torch.Tensor] = None, eps: float = 1e-6, *,
+             dx: Optional[torch.Tensor] = None, dw: Optional[torch.Tensor] = None,
+             ws: Optional[torch.Tensor] = None, stream=None):
+    """Zero-centred RMSNorm backward.  Returns (dx, dw).  rstd=None recomputes it."""
+    rows, width = _rows_width(x)
+    _vec("w", w, width, x.device)
+    _mat("dy", dy, x)
+    if rstd is not None:
+        _vec("rstd", rstd, rows, x.device)
+    dx = torch.empty_like(x) if dx is None else _mat("dx", dx, x)
+    dw = torch.empty(width, dtype=torch.float32, device=x.device) if dw is None else \
+        _vec("dw", dw, width, x.device)
+    ws, nws = _ws(rows, width, x.device, ws)
+    with torch.cuda.device(x.device):
+        check("norm_bwd", load().norm_bwd(rows, width, eps, _dt(x), _ptr(x), _ptr(w), _ptr(dy),
+                                          _ptr(rstd), _ptr(dx), _ptr(dw), _ptr(ws), nws,
+                                          _stream(x, stream)))
+    return dx, dw
+
+
+def gated_norm_bwd(x: torch.Tensor, z: torch.Tensor, w: torch.Tensor, dy: torch.Tensor,
+                   rstd: Optional[torch.Tensor] = None, eps: float = 1e-6, *,
+                   dx: Optional[torch.Tensor] = None, dz: Optional[torch.Tensor] = None,
+                   dw: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                   stream=None):
+    """Gated RMSNorm backward.  Returns (dx, dz, dw).  rstd=None recomputes it."""
+    rows, width = _rows_width(x)
+    _mat("z", z, x)
+    _vec("w", w, width, x.device)
+    _mat("dy", dy, x)
+    if rstd is not None:
+        _vec("rstd", rstd, rows, x.device)
+    dx = torch.empty_like(x) if dx is None else _mat("dx", dx, x)
+    dz = torch.empty_like(x) if dz is None else _mat("dz", dz, x)
+    dw = torch.empty(width, dtype=torch.float32, device=x.device) if dw is None else \
+        _vec("dw", dw, width, x.device)
+    ws, nws = _ws(rows, width, x.device, ws)
+    with torch.cuda.device(x.device):
+        check("gated_norm_bwd",
+              load().gated_norm_bwd(rows, width, eps, _dt(x), _ptr(x), _ptr(z), _ptr(w), _ptr(dy),
+                                    _ptr(rstd), _ptr(dx), _ptr(dz), _ptr(dw), _ptr(ws), nws,
+                                    _stream(x, stream)))
+    return dx, dz, dw
+
+
+def rn_describe(width: int, dtype=torch.bfloat16) -> str:
+    dt = _DT[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    return load().rn_describe(width, dt).decode()
+
+
+def rn_test_set_geometry(max_ctas: int = 0, leaves_per_cta: int = 0, fold_rows: int = 0) -> None:
+    check("rn_test_set_geometry", load().rn_test_set_geometry(max_ctas, leaves_per_cta, fold_rows))
+
+
+def rn_test_set_validate_only(on: bool) -> None:
+    load().rn_test_set_validate_only(1 if on else 0)

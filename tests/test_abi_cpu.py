@@ -1,0 +1,258 @@
+"""The C ABI without a GPU: the library loads, exports every function
+include/rn.h declares, and its argument checks return the documented status
+without touching CUDA (validate-only mode; the fake pointers below are never
+dereferenced)."""
+import contextlib
+import os
+import re
+import subprocess
+
+import pytest
+
+import rollout_parity_b200 as rn
+from rollout_parity_b200 import build as rn_build
+from rollout_parity_b200._lib import SIGNATURES, DType, Status
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rn.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(
+        r"^(?:rn_status|size_t|const char\s*\*|int32_t|int|void)\s+(\w+)\s*\(", text,
+        flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    rn_build.build()
+    return rn.load()
+
+
+@contextlib.contextmanager
+def validate_only(lib):
+    lib.rn_test_set_validate_only(1)
+    try:
+        yield
+    finally:
+        lib.rn_test_set_validate_only(0)
+
+
+def test_header_declares_the_expected_api():
+    assert header_functions() == sorted(SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", rn.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if ln.strip()}
+    for name in header_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+# fake device addresses, 4 GiB apart so nothing overlaps unless a test says so
+BASE = 1 << 40
+def P(i, off=0):
+    return BASE + (i << 32) + off
+
+
+R, H = 64, 128
+X, Z, W, Y, RS, DY, DX, DZ, DW, WS = range(10)
+
+
+def fwd(lib, rows=R, width=H, eps=1e-6, dt=DType.BF16, x=None, w=None, y=None, rstd=None):
+    return lib.norm_fwd(rows, width, eps, dt, P(X) if x is None else x, P(W) if w is None else w,
+                        P(Y) if y is None else y, P(RS) if rstd is None else rstd, None)
+
+
+def gfwd(lib, rows=R, width=H, eps=1e-6, dt=DType.BF16, x=None, z=None, w=None, y=None,
+         rstd=None):
+    return lib.gated_norm_fwd(rows, width, eps, dt, P(X) if x is None else x,
+                              P(Z) if z is None else z, P(W) if w is None else w,
+                              P(Y) if y is None else y, P(RS) if rstd is None else rstd, None)
+
+
+def gbwd(lib, rows=R, width=H, eps=1e-6, dt=DType.BF16, ws_bytes=None, **kw):
+    ptr = dict(x=P(X), z=P(Z), w=P(W), dy=P(DY), rstd=P(RS), dx=P(DX), dz=P(DZ), dw=P(DW),
+               ws=P(WS))
+    ptr.update(kw)
+    nws = lib.norm_bwd_workspace_bytes(rows, width) if ws_bytes is None else ws_bytes
+    return lib.gated_norm_bwd(rows, width, eps, dt, ptr["x"], ptr["z"], ptr["w"], ptr["dy"],
+                              ptr["rstd"], ptr["dx"], ptr["dz"], ptr["dw"], ptr["ws"], nws, None)
+
+
+def bwd(lib, rows=R, width=H, eps=1e-6, dt=DType.BF16, ws_bytes=None, **kw):
+    ptr = dict(x=P(X), w=P(W), dy=P(DY), rstd=P(RS), dx=P(DX), dw=P(DW), ws=P(WS))
+    ptr.update(kw)
+    nws = lib.norm_bwd_workspace_bytes(rows, width) if ws_bytes is None else ws_bytes
+    return lib.norm_bwd(rows, width, eps, dt, ptr["x"], ptr["w"], ptr["dy"], ptr["rstd"],
+                        ptr["dx"], ptr["dw"], ptr["ws"], nws, None)
+
+
+FWD_CASES = [
+    ("valid", {}, Status.OK),
+    ("valid f32", dict(dt=DType.F32), Status.OK),
+    ("rstd NULL", dict(rstd=0), Status.OK),
+    ("rstd 4-byte aligned", dict(rstd=P(RS, 4)), Status.OK),
+    ("rows 0, no tensors", dict(rows=0, x=0, y=0), Status.OK),
+    ("rows < 0", dict(rows=-1), Status.E_ARG),
+    ("rows too large", dict(rows=(1 << 36) + 1), Status.E_ARG),
+    ("eps < 0", dict(eps=-1e-6), Status.E_ARG),
+    ("eps nan", dict(eps=float("nan")), Status.E_ARG),
+    ("eps inf", dict(eps=float("inf")), Status.E_ARG),
+    ("dtype", dict(dt=7), Status.E_DTYPE),
+    ("width 0", dict(width=0), Status.E_WIDTH),
+    ("width 4", dict(width=4), Status.E_WIDTH),
+    ("width 12", dict(width=12), Status.E_WIDTH),
+    ("width 16392", dict(width=16392), Status.E_WIDTH),
+    ("width < 0", dict(width=-8), Status.E_WIDTH),
+    ("x NULL", dict(x=0), Status.E_ARG),
+    ("w NULL", dict(w=0), Status.E_ARG),
+    ("y NULL", dict(y=0), Status.E_ARG),
+    ("x misaligned", dict(x=P(X, 2)), Status.E_ALIGN),
+    ("w misaligned", dict(w=P(W, 4)), Status.E_ALIGN),
+    ("y misaligned", dict(y=P(Y, 8)), Status.E_ALIGN),
+    ("rstd misaligned", dict(rstd=P(RS, 2)), Status.E_ALIGN),
+    ("y aliases x", dict(y=P(X)), Status.E_ARG),
+    ("y overlaps x tail", dict(y=P(X, R * H * 2 - 16)), Status.E_ARG),
+    ("y just after x", dict(y=P(X, R * H * 2)), Status.OK),
+    ("rstd inside y", dict(rstd=P(Y, 64)), Status.E_ARG),
+    ("y overlaps w", dict(y=P(W, -16)), Status.E_ARG),
+]
+
+
+@pytest.mark.parametrize("name,kw,want", FWD_CASES, ids=[c[0] for c in FWD_CASES])
+def test_norm_fwd_checks(lib, name, kw, want):
+    with validate_only(lib):
+        assert fwd(lib, **kw) == want
+
+
+GFWD_CASES = [
+    ("valid", {}, Status.OK),
+    ("z NULL", dict(z=0), Status.E_ARG),
+    ("z misaligned", dict(z=P(Z, 2)), Status.E_ALIGN),
+    ("z == x is allowed", dict(z=P(X)), Status.OK),
+    ("y aliases z", dict(y=P(Z)), Status.E_ARG),
+    ("rows 0", dict(rows=0, x=0, z=0, y=0), Status.OK),
+]
+
+
+@pytest.mark.parametrize("name,kw,want", GFWD_CASES, ids=[c[0] for c in GFWD_CASES])
+def test_gated_norm_fwd_checks(lib, name, kw, want):
+    with validate_only(lib):
+        assert gfwd(lib, **kw) == want
+
+
+GBWD_CASES = [
+    ("valid", {}, Status.OK),
+    ("rstd NULL recomputes", dict(rstd=0), Status.OK),
+    ("ws NULL", dict(ws=0), Status.E_WORKSPACE),
+    ("ws too small", dict(ws_bytes=1024), Status.E_WORKSPACE),
+    ("ws misaligned", dict(ws=P(WS, 8)), Status.E_ALIGN),
+    ("ws overlaps dx", dict(ws=P(DX, 256)), Status.E_ARG),
+    ("ws overlaps x", dict(ws=P(X)), Status.E_ARG),
+    ("dw NULL", dict(dw=0), Status.E_ARG),
+    ("dz NULL", dict(dz=0), Status.E_ARG),
+    ("dx aliases dy", dict(dx=P(DY)), Status.E_ARG),
+    ("dz aliases dx", dict(dz=P(DX)), Status.E_ARG),
+    ("dw overlaps w", dict(dw=P(W)), Status.E_ARG),
+    ("dw inside dz", dict(dw=P(DZ, 4096)), Status.E_ARG),
+    ("dy misaligned", dict(dy=P(DY, 2)), Status.E_ALIGN),
+    ("dw misaligned", dict(dw=P(DW, 4)), Status.E_ALIGN),
+    ("rows 0 only needs dw", dict(rows=0, x=0, z=0, dy=0, dx=0, dz=0, ws=0, rstd=0), Status.OK),
+    ("rows 0 still needs dw", dict(rows=0, dw=0), Status.E_ARG),
+    ("width", dict(width=20), Status.E_WIDTH),
+    ("dtype", dict(dt=2), Status.E_DTYPE),
+]
+
+
+@pytest.mark.parametrize("name,kw,want", GBWD_CASES, ids=[c[0] for c in GBWD_CASES])
+def test_gated_norm_bwd_checks(lib, name, kw, want):
+    with validate_only(lib):
+        assert gbwd(lib, **kw) == want
+
+
+BWD_CASES = [
+    ("valid", {}, Status.OK),
+    ("ws too small by one byte", dict(ws_bytes="need-1"), Status.E_WORKSPACE),
+    ("dx aliases x", dict(dx=P(X)), Status.E_ARG),
+    ("rstd overlaps dx", dict(rstd=P(DX, 16)), Status.E_ARG),
+]
+
+
+@pytest.mark.parametrize("name,kw,want", BWD_CASES, ids=[c[0] for c in BWD_CASES])
+def test_norm_bwd_checks(lib, name, kw, want):
+    if kw.get("ws_bytes") == "need-1":
+        kw = dict(kw, ws_bytes=lib.norm_bwd_workspace_bytes(R, H) - 1)
+    with validate_only(lib):
+        assert bwd(lib, **kw) == want
+
+
+@pytest.mark.parametrize("rows", [1, 31, 32, 33, 256, 257, 4096, 262144, 1 << 30])
+@pytest.mark.parametrize("width", [8, 128, 2048, 8192, 16384])
+def test_workspace_bytes(lib, rows, width):
+    leaves = -(-rows // 32)
+    assert lib.norm_bwd_workspace_bytes(rows, width) == (leaves + -(-leaves // 8)) * width * 4
+
+
+def test_workspace_bytes_invalid(lib):
+    assert lib.norm_bwd_workspace_bytes(0, 128) == 0
+    assert lib.norm_bwd_workspace_bytes(-5, 128) == 0
+    assert lib.norm_bwd_workspace_bytes(64, 100) == 0
+
+
+@pytest.mark.parametrize("width,dt,team", [(128, DType.BF16, 16), (128, DType.F32, 32),
+                                           (8, DType.BF16, 1), (2048, DType.BF16, 128),
+                                           (8192, DType.BF16, 512), (5120, DType.BF16, 512),
+                                           (16384, DType.F32, 1024)])
+def test_describe(lib, width, dt, team):
+    d = lib.rn_describe(width, dt).decode()
+    assert f"team_threads={team} " in d
+    assert "acc=fp32" in d and "atomics=none" in d and "fast_math=off" in d
+
+
+def test_describe_unsupported(lib):
+    assert lib.rn_describe(100, DType.BF16) == b"unsupported"
+    assert lib.rn_describe(128, 9) == b"unsupported"
+
+
+def test_geometry_knob_checks(lib):
+    try:
+        assert lib.rn_test_set_geometry(-1, 0, 0) == Status.E_ARG
+        assert lib.rn_test_set_geometry(0, 3, 0) == Status.E_ARG
+        assert lib.rn_test_set_geometry(0, 0, 4) == Status.E_ARG
+        assert lib.rn_test_set_geometry(0, 0, 512) == Status.E_ARG
+        assert lib.rn_test_set_geometry(0, 0, 24) == Status.E_ARG
+        assert lib.rn_test_set_geometry(7, 2, 64) == Status.OK
+    finally:
+        assert lib.rn_test_set_geometry(0, 0, 0) == Status.OK
+
+
+def test_bwd_launch_count(lib):
+    # 262144 rows of width 128: 8192 leaves, 8 per CTA -> 1024 partials -> 2 fold passes
+    assert lib.rn_bwd_launches(262144, 128, DType.BF16) == 3
+    assert lib.rn_bwd_launches(256, 128, DType.BF16) == 1      # one CTA writes dw itself
+    assert lib.rn_bwd_launches(0, 128, DType.BF16) == 0
+    assert lib.rn_bwd_launches(64, 100, DType.BF16) == 0
+    try:
+        lib.rn_test_set_geometry(0, 1, 8)                         # 8192 leaves, 8 rows/pass
+        assert lib.rn_bwd_launches(262144, 128, DType.BF16) == 1 + 5
+    finally:
+        lib.rn_test_set_geometry(0, 0, 0)
+
+
+def test_status_strings(lib):
+    for s in Status:
+        assert lib.rn_status_string(int(s))
+    assert lib.rn_last_cuda_error() == 0
+
+
+def test_binding_rejects_host_tensors(lib):
+    import torch
+    x = torch.zeros(4, 128, dtype=torch.bfloat16)
+    w = torch.zeros(128)
+    with pytest.raises(ValueError):
+        rn.norm_fwd(x, w)
