@@ -57,6 +57,9 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-invariance", action="store_true")
+    ap.add_argument("--buffer-sets", type=int, default=SETS,
+                    help="rotating input sets (fewer only for profiler captures)")
     return ap.parse_args()
 
 
@@ -182,7 +185,8 @@ def run_ours(a):
                                 device_id=dev)
     lib = rn.load()
 
-    host = [workloads.cfg_gated_heads(seed=1000 * rank + s) for s in range(SETS)]
+    nsets = max(1, a.buffer_sets)
+    host = [workloads.cfg_gated_heads(seed=1000 * rank + s) for s in range(nsets)]
     R, H, eps = host[0].rows, host[0].width, host[0].eps
     fwd_b, bwd_b = bytes_model(R, H)
     step_b = fwd_b + bwd_b
@@ -210,8 +214,8 @@ def run_ours(a):
     for p in P:                       # every set gets its rstd before any backward
         check("gated_norm_fwd", fwd(p))
     for k in range(a.warmup):
-        check("gated_norm_fwd", fwd(P[k % SETS]))
-        check("gated_norm_bwd", bwd(P[(k + 2) % SETS]))
+        check("gated_norm_fwd", fwd(P[k % nsets]))
+        check("gated_norm_bwd", bwd(P[(k + 2) % nsets]))
     torch.cuda.synchronize()
 
     K = a.steps
@@ -227,9 +231,9 @@ def run_ours(a):
     for k in range(K):
         e = ev[k]
         e[0].record(stream)
-        s1 = fwd(P[k % SETS])
+        s1 = fwd(P[k % nsets])
         e[1].record(stream)
-        s2 = bwd(P[(k + 2) % SETS])
+        s2 = bwd(P[(k + 2) % nsets])
         e[2].record(stream)
         if s1 or s2:
             check("gated_norm_fwd", s1)
@@ -251,8 +255,10 @@ def run_ours(a):
     value = world * step_b * K / (ms / 1e3) / 1e9
     launches = K * (1 + lib.rn_bwd_launches(R, H, bf16))
 
-    inv = invariance_checks(rn, sets[0], R, H, eps) if rank == 0 else None
-    e2e = run_e2e(rn, host[0], dev, a.e2e_steps, step_b, world, dist)
+    inv = invariance_checks(rn, sets[0], R, H, eps) if rank == 0 and not a.no_invariance \
+        else None
+    e2e = run_e2e(rn, host[0], dev, a.e2e_steps, step_b, world, dist) if a.e2e_steps > 0 \
+        else None
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         cpu = cpu_baseline(host[0], fwd_b, bwd_b)
@@ -273,9 +279,10 @@ def run_ours(a):
                        "outliers": "1% of channels x50 in x, z, dy", "eps": eps,
                        "io_dtype": "bf16 x/z/dy/y/dx/dz, fp32 w/rstd/dw", "accumulate": "fp32",
                        "bytes_per_step": step_b, "parallelism": f"replicas x{world}",
-                       "l2": "4 rotating buffer sets (fwd on k%4, bwd on (k+2)%4): every "
-                             "buffer is re-touched only after >= 512 MB of other traffic "
-                             "(L2 is 126 MB); no flush kernel"},
+                       "l2": (f"{nsets} rotating buffer sets (fwd on k%{nsets}, bwd on "
+                              f"(k+2)%{nsets}): every buffer is re-touched only after >= 512 MB "
+                              "of other traffic (L2 is 126 MB); no flush kernel")
+                       if nsets == SETS else f"{nsets} buffer set(s): profiling layout"},
             "rows_per_s": round(world * R * K / (ms / 1e3), 1),
             "pct_of_peak": round(100.0 * value / world / peak, 2),
             "fwd_us": round(1e3 * fwd_mean, 2), "bwd_us": round(1e3 * bwd_mean, 2),

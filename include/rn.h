@@ -186,6 +186,15 @@ rn_status rn_test_set_geometry(int32_t max_ctas, int32_t leaves_per_cta,
  */
 void rn_test_set_validate_only(int32_t on);
 
+/*
+ * Test entry point: out[i] = the reciprocal the sigmoid uses, for inputs
+ * d[i] in [1, 2] (n floats, device pointers; steps = 1 or 2 Newton steps;
+ * RN_E_ARG otherwise).  Lets a test compare it with IEEE division over every
+ * float in [1, 2].
+ */
+rn_status rn_test_rcp_1to2(int64_t n, const float* d, float* out, int32_t steps,
+                           rn_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

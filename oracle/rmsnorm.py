@@ -139,7 +139,13 @@ def gated_norm_bwd(x, z, w, dy, eps: float):
 # rounding that cancellation amplifies.
 # ---------------------------------------------------------------------------
 def dx_cancellation_scale(x, w, dy, eps: float, z=None) -> np.ndarray:
-    """max(|rho * g * dy|, |rho * xh * m|) per element (the two terms of dx)."""
+    """max(|rho * g * dy|, |rho * xh| * mean_k |g_k * dy_k * xh_k|) per element.
+
+    The two terms of dx are rho*g*dy and rho*xh*m.  m is a sum over the row, so
+    its rounding error scales with the sum of the magnitudes of its terms, not
+    with |m| (the dot-product error bound, Higham, "Accuracy and Stability of
+    Numerical Algorithms", 2nd ed., section 3.1); the second term therefore uses
+    mean_k |g_k dy_k xh_k| in place of |m|."""
     x, dy = _rows(x), _rows(dy)
     w = np.asarray(w, dtype=np.float64)
     rho = rstd(x, eps)
@@ -148,9 +154,9 @@ def dx_cancellation_scale(x, w, dy, eps: float, z=None) -> np.ndarray:
         g = np.broadcast_to((1.0 + w)[None, :], x.shape)
     else:
         g = w[None, :] * silu(_rows(z))
-    m = np.sum(g * dy * xh, axis=1) / x.shape[1]
+    m_abs = np.sum(np.abs(g * dy * xh), axis=1) / x.shape[1]
     a = np.abs(rho[:, None] * g * dy)
-    b = np.abs(rho[:, None] * xh * m[:, None])
+    b = np.abs(rho[:, None] * xh * m_abs[:, None])
     return np.maximum(a, b)
 
 

@@ -51,6 +51,7 @@ SIGNATURES = {
     "rn_last_cuda_error": (ctypes.c_int, []),
     "rn_test_set_geometry": (c_i32, [c_i32, c_i32, c_i32]),
     "rn_test_set_validate_only": (None, [c_i32]),
+    "rn_test_rcp_1to2": (c_i32, [c_i64, c_vp, c_vp, c_i32, c_vp]),
 }
 
 _lib = None

@@ -92,14 +92,37 @@ __device__ __forceinline__ void st_stream(uint4* p, const uint4& v) { __stcs(p, 
 // ---------------------------------------------------------------------------
 // arithmetic of one element, written with explicit roundings
 // ---------------------------------------------------------------------------
+// 1/d for d in [1, 2]: the hardware approximation (rcp.approx, within 1 ulp)
+// refined by Newton-Raphson steps written as fused multiply-adds, e = 1 - d*y,
+// y' = y + y*e (Markstein, "Computation of elementary functions on the IBM
+// RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990).  The domain
+// needs no special cases (no zero, infinity, NaN or subnormal).  A GPU test
+// compares it with IEEE division for every float in [1, 2].
+template <int STEPS>
+__device__ __forceinline__ float rcp_1to2(float d) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(d));
+#pragma unroll
+  for (int i = 0; i < STEPS; ++i) y = __fmaf_rn(y, __fmaf_rn(-d, y, 1.0f), y);
+  return y;
+}
+constexpr int kRcpSteps = 1;   // one step is already IEEE-exact on [1, 2]
+
 // s(z) = 1 / (1 + exp(-z)); silu(z) = z * s(z)   (PR #468 Summary, activation)
+// Evaluated as 1/(1+e) for z >= 0 and e/(1+e) for z < 0 with e = exp(-|z|) in
+// (0, 1]: the same function, but exp never overflows, so for z < -88.7 the
+// sigmoid is the fp32 subnormal e^z rather than 1/inf = 0 (outlier gates reach
+// there, and x*rstd*w*z*s(z) can still be a normal bf16 number).
 __device__ __forceinline__ float sigmoid_f(float z) {
-  return __frcp_rn(__fadd_rn(1.0f, expf(-z)));
+  const float e = expf(-fabsf(z));
+  const float r = rcp_1to2<kRcpSteps>(__fadd_rn(1.0f, e));
+  return z >= 0.0f ? r : __fmul_rn(e, r);
 }
 
-// rstd = rsqrt(ss / H + eps)   (PR #468 Summary, rstd bullet)
-__device__ __forceinline__ float rstd_from_sumsq(float ss, float H, float eps) {
-  return rsqrtf(__fadd_rn(__fdiv_rn(ss, H), eps));
+// sum / H with an IEEE division; when H is a power of two this is the exact
+// scaling sum * (1/H), which gives the same bits with one multiply.
+__device__ __forceinline__ float mean_of(float sum, int H, float inv_h, bool h_pow2) {
+  return h_pow2 ? __fmul_rn(sum, inv_h) : __fdiv_rn(sum, float(H));
 }
 
 __device__ __forceinline__ float4 add4(const float4& a, const float4& b) {
@@ -158,8 +181,9 @@ __device__ __forceinline__ void team_sum(float (&v)[U], float* red, int& phase, 
 // ---------------------------------------------------------------------------
 struct FwdArgs {
   int64_t rows;
-  int H;
-  float eps;
+  int H, nv;
+  float eps, inv_h;
+  int h_pow2;
   const uint4* x;
   const uint4* z;
   const float* w;
@@ -169,8 +193,9 @@ struct FwdArgs {
 
 struct BwdArgs {
   int64_t rows;
-  int H;
-  float eps;
+  int H, nv;
+  float eps, inv_h;
+  int h_pow2;
   const uint4* x;
   const uint4* z;
   const float* w;
@@ -183,12 +208,21 @@ struct BwdArgs {
 
 template <int T>
 __host__ __device__ constexpr int fwd_block() { return T <= 32 ? 256 : T; }
-template <int T>
-__host__ __device__ constexpr int bwd_max_block() { return T <= 32 ? 8 * T : (T <= 128 ? 256 : T); }
+template <int T, int K>
+__host__ __device__ constexpr int fwd_min_blocks() { return T <= 16 ? 3 : 1; }
 template <int T>
 __host__ __device__ constexpr int fwd_rows_per_team() { return T <= 32 ? 2 : 1; }
 template <int T>
-__host__ __device__ constexpr int bwd_rows_per_step() { return T <= 32 ? 2 : 1; }
+__host__ __device__ constexpr int bwd_max_block() { return T <= 32 ? 8 * T : (T <= 128 ? 256 : T); }
+// enough resident CTAs that one wave holds every 32-row leaf of a ~256K-row
+// batch at width 128 (1024 CTAs of 128 threads on 148 SMs)
+template <int T, int K>
+__host__ __device__ constexpr int bwd_min_blocks() {
+  return K != 1 ? 1 : (T <= 16 ? 112 / T : (T == 32 ? 3 : 1));
+}
+// sub-warp teams read w from shared memory (saves registers for occupancy)
+template <int T>
+__host__ __device__ constexpr bool bwd_w_in_smem() { return T <= 32; }
 
 // Loads this thread's gain base: w (gated) or 1 + w (zero-centred).
 template <int VE, int K, int T, bool GATED>
@@ -208,8 +242,87 @@ __device__ __forceinline__ void load_gain(const float* __restrict__ w, int nv, i
   }
 }
 
-template <int DT, int T, int K, bool GATED>
-__global__ void __launch_bounds__(fwd_block<T>())
+// A thread's K vectors of one row; `p` points at the row's vector t.
+template <int T, int K, bool EXACT>
+__device__ __forceinline__ void load_row(uint4 (&r)[K], const uint4* __restrict__ p, int nv,
+                                         int t, bool act) {
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const bool ok = act && (EXACT || k * T + t < nv);
+    r[k] = ok ? ld_stream(p + k * T) : make_uint4(0, 0, 0, 0);
+  }
+}
+
+// Sum of squares of this thread's elements: ascending, fma, from -0.0.
+template <int DT, int T, int K, bool EXACT>
+__device__ __forceinline__ float thread_sumsq(const uint4 (&x)[K], int nv, int t) {
+  using F = Fmt<DT>;
+  float ss = -0.0f;
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    if (EXACT || k * T + t < nv) {
+      float f[F::VE];
+      F::unpack(x[k], f);
+#pragma unroll
+      for (int e = 0; e < F::VE; ++e) ss = __fmaf_rn(f[e], f[e], ss);
+    }
+  }
+  return ss;
+}
+
+// Writes the partial of this CTA's group of NT leaves (an aligned
+// power-of-two block, nl of them present) to `out`: the leaves' partials
+// (this thread's columns in acc) go through shared memory and are joined by
+// the level-by-level pairwise tree; with one leaf, acc is the partial.
+template <int VE, int K, int T, bool EXACT>
+__device__ __forceinline__ void join_leaves(const float (&acc)[K][VE], int NT, int nl, int team,
+                                            int t, int nv, int H, float* leafbuf, float* out) {
+  float4* out4 = reinterpret_cast<float4*>(out);
+  if (NT == 1) {
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const int v = k * T + t;
+      if (EXACT || v < nv) {
+#pragma unroll
+        for (int q = 0; q < VE / 4; ++q)
+          out4[v * (VE / 4) + q] = make_float4(acc[k][4 * q], acc[k][4 * q + 1],
+                                               acc[k][4 * q + 2], acc[k][4 * q + 3]);
+      }
+    }
+    return;
+  }
+  __syncthreads();   // the previous group's readers of leafbuf are done
+  float4* lb4 = reinterpret_cast<float4*>(leafbuf + team * H);
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const int v = k * T + t;
+    if (EXACT || v < nv) {
+#pragma unroll
+      for (int q = 0; q < VE / 4; ++q)
+        lb4[v * (VE / 4) + q] = make_float4(acc[k][4 * q], acc[k][4 * q + 1],
+                                            acc[k][4 * q + 2], acc[k][4 * q + 3]);
+    }
+  }
+  __syncthreads();
+  const int H4 = H / 4;
+  const float4* all4 = reinterpret_cast<const float4*>(leafbuf);
+  for (int c = threadIdx.x; c < H4; c += blockDim.x) {
+    float4 p[8];
+#pragma unroll
+    for (int l = 0; l < 8; ++l)
+      p[l] = l < NT ? all4[l * H4 + c] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int s = 1; s < 8; s <<= 1) {
+#pragma unroll
+      for (int l = 0; l + s < 8; l += 2 * s)
+        if (l + s < nl) p[l] = add4(p[l], p[l + s]);
+    }
+    out4[c] = p[0];
+  }
+}
+
+template <int DT, int T, int K, bool GATED, bool EXACT>
+__global__ void __launch_bounds__(fwd_block<T>(), fwd_min_blocks<T, K>())
 k_fwd(const FwdArgs a) {
   using F = Fmt<DT>;
   constexpr int VE = F::VE;
@@ -218,8 +331,7 @@ k_fwd(const FwdArgs a) {
   constexpr int W = T > 32 ? T / 32 : 1;
   __shared__ float red[T > 32 ? 2 * NT * U * W : 1];
   const int team = threadIdx.x / T, t = threadIdx.x % T;
-  const int nv = a.H / VE;
-  const float Hf = float(a.H);
+  const int nv = a.nv;
   const unsigned mask = 0xffffffffu;   // the forward block is always >= 256 threads
   int phase = 0;
 
@@ -230,42 +342,25 @@ k_fwd(const FwdArgs a) {
   for (int64_t base = int64_t(blockIdx.x) * NT * U; base < a.rows; base += step) {
     uint4 xr[U][K], zr[U][K];
     bool act[U];
+    int64_t off[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int64_t row = base + int64_t(u) * NT + team;
       act[u] = row < a.rows;
-#pragma unroll
-      for (int k = 0; k < K; ++k) {
-        const int v = k * T + t;
-        const bool ok = act[u] && v < nv;
-        xr[u][k] = ok ? ld_stream(a.x + row * nv + v) : make_uint4(0, 0, 0, 0);
-        if constexpr (GATED) zr[u][k] = ok ? ld_stream(a.z + row * nv + v) : make_uint4(0, 0, 0, 0);
-      }
+      off[u] = row * nv + t;
+      load_row<T, K, EXACT>(xr[u], a.x + off[u], nv, t, act[u]);
+      if constexpr (GATED) load_row<T, K, EXACT>(zr[u], a.z + off[u], nv, t, act[u]);
     }
-    // sum of squares: ascending over this thread's elements, fma, from -0.0
     float ss[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      ss[u] = -0.0f;
-#pragma unroll
-      for (int k = 0; k < K; ++k) {
-        if (k * T + t < nv) {
-          float f[VE];
-          F::unpack(xr[u][k], f);
-#pragma unroll
-          for (int e = 0; e < VE; ++e) ss[u] = __fmaf_rn(f[e], f[e], ss[u]);
-        }
-      }
-    }
+    for (int u = 0; u < U; ++u) ss[u] = thread_sumsq<DT, T, K, EXACT>(xr[u], nv, t);
     team_sum<T, U>(ss, red, phase, team, NT, mask);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int64_t row = base + int64_t(u) * NT + team;
-      const float r = rstd_from_sumsq(ss[u], Hf, a.eps);
+      const float r = rsqrtf(__fadd_rn(mean_of(ss[u], a.H, a.inv_h, a.h_pow2), a.eps));
 #pragma unroll
       for (int k = 0; k < K; ++k) {
-        const int v = k * T + t;
-        if (act[u] && v < nv) {
+        if (act[u] && (EXACT || k * T + t < nv)) {
           float f[VE], yv[VE];
           F::unpack(xr[u][k], f);
           if constexpr (GATED) {
@@ -273,41 +368,250 @@ k_fwd(const FwdArgs a) {
             F::unpack(zr[u][k], zf);
 #pragma unroll
             for (int e = 0; e < VE; ++e) {
-              const float s = sigmoid_f(zf[e]);
-              const float act_z = __fmul_rn(zf[e], s);
+              const float act_z = __fmul_rn(zf[e], sigmoid_f(zf[e]));
               yv[e] = __fmul_rn(__fmul_rn(__fmul_rn(f[e], r), gw[k][e]), act_z);
             }
           } else {
 #pragma unroll
             for (int e = 0; e < VE; ++e) yv[e] = __fmul_rn(__fmul_rn(f[e], r), gw[k][e]);
           }
-          st_stream(a.y + row * nv + v, F::pack(yv));
+          st_stream(a.y + off[u] + k * T, F::pack(yv));
         }
       }
-      if (act[u] && t == 0 && a.rstd != nullptr) a.rstd[row] = r;
+      if (act[u] && t == 0 && a.rstd != nullptr) a.rstd[base + int64_t(u) * NT + team] = r;
     }
   }
 }
 
-template <int DT, int T, int K, bool GATED>
-__global__ void __launch_bounds__(bwd_max_block<T>())
+template <int DT, int T, int K, bool GATED, bool EXACT>
+__global__ void __launch_bounds__(bwd_max_block<T>(), bwd_min_blocks<T, K>())
 k_bwd(const BwdArgs a) {
   using F = Fmt<DT>;
   constexpr int VE = F::VE;
-  constexpr int U = bwd_rows_per_step<T>();
   constexpr int W = T > 32 ? T / 32 : 1;
-  extern __shared__ float dsm[];   // [2][NT][U][W] reduction scratch, then [NT][H] leaves
+  constexpr bool WS = bwd_w_in_smem<T>();
+  // dynamic shared memory: [H] gain (WS), [2][NT][W] reduction scratch (T > 32),
+  // then [NT][H] leaf partials (NT > 1)
+  extern __shared__ float dsm[];
   const int NT = blockDim.x / T;   // leaves per CTA (power of two)
-  float* red = dsm;
-  float* leafbuf = dsm + (T > 32 ? 2 * NT * U * W : 0);
+  float* gsm = dsm;
+  float* red = dsm + (WS ? a.H : 0);
+  float* leafbuf = red + (T > 32 ? 2 * NT * W : 0);
   const int team = threadIdx.x / T, t = threadIdx.x % T;
-  const int nv = a.H / VE;
-  const float Hf = float(a.H);
+  const int nv = a.nv;
   const unsigned mask = blockDim.x >= 32 ? 0xffffffffu : ((1u << blockDim.x) - 1u);
+  const bool have_rstd = a.rstd != nullptr;
   int phase = 0;
 
-  float gw[K][VE];
-  load_gain<VE, K, T, GATED>(a.w, nv, t, gw);
+  float gw_r[WS ? 1 : K][WS ? 1 : VE];
+  if constexpr (WS) {
+    for (int c = threadIdx.x; c < a.H; c += blockDim.x)
+      gsm[c] = GATED ? __ldg(a.w + c) : __fadd_rn(1.0f, __ldg(a.w + c));
+    __syncthreads();
+  } else {
+    load_gain<VE, K, T, GATED>(a.w, nv, t, gw_r);
+  }
+  // this thread's gain for vector k: from registers, or from shared memory
+  auto gain = [&](int k, float (&g)[VE]) {
+    if constexpr (WS) {
+      const float4* p = reinterpret_cast<const float4*>(gsm) + (k * T + t) * (VE / 4);
+#pragma unroll
+      for (int q = 0; q < VE / 4; ++q) {
+        const float4 f = p[q];
+        g[4 * q] = f.x; g[4 * q + 1] = f.y; g[4 * q + 2] = f.z; g[4 * q + 3] = f.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < VE; ++e) g[e] = gw_r[WS ? 0 : k][WS ? 0 : e];
+    }
+  };
+
+  // one row: fetch (issued a row ahead of its use)
+  auto fetch = [&](int64_t row, bool act, uint4 (&x)[K], uint4 (&z)[K], uint4 (&d)[K],
+                   float& r) {
+    const int64_t off = row * nv + t;
+    load_row<T, K, EXACT>(x, a.x + off, nv, t, act);
+    load_row<T, K, EXACT>(d, a.dy + off, nv, t, act);
+    if constexpr (GATED) load_row<T, K, EXACT>(z, a.z + off, nv, t, act);
+    r = (act && have_rstd) ? __ldcs(a.rstd + row) : 0.0f;
+  };
+
+  float acc[K][VE];
+
+  // one row: dot, dx, dz, and the leaf's dw fold (called in ascending row order)
+  auto process = [&](int64_t row, bool act, const uint4 (&x)[K], const uint4 (&z)[K],
+                     const uint4 (&d)[K], float rs) {
+    if (!have_rstd) {   // uniform branch: recompute exactly as the forward does
+      float ss[1] = {thread_sumsq<DT, T, K, EXACT>(x, nv, t)};
+      team_sum<T, 1>(ss, red, phase, team, NT, mask);
+      rs = rsqrtf(__fadd_rn(mean_of(ss[0], a.H, a.inv_h, a.h_pow2), a.eps));
+    }
+    // pass 1: dot = sum_j (g_j * dy_j) * xh_j, xh = x*rstd, g = 1+w or w*silu(z)
+    float sg[K][GATED ? VE : 1];
+    float dot[1] = {-0.0f};
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      float xf[VE], df[VE], zf[VE], gk[VE];
+      F::unpack(x[k], xf);
+      F::unpack(d[k], df);
+      if constexpr (GATED) F::unpack(z[k], zf);
+      gain(k, gk);
+#pragma unroll
+      for (int e = 0; e < VE; ++e) {
+        const float xh = __fmul_rn(xf[e], rs);
+        float g;
+        if constexpr (GATED) {
+          sg[k][e] = sigmoid_f(zf[e]);
+          g = __fmul_rn(gk[e], __fmul_rn(zf[e], sg[k][e]));      // w * silu(z)
+        } else {
+          g = gk[e];                                             // 1 + w
+        }
+        if (EXACT || k * T + t < nv) dot[0] = __fmaf_rn(__fmul_rn(g, df[e]), xh, dot[0]);
+      }
+    }
+    team_sum<T, 1>(dot, red, phase, team, NT, mask);
+    const float m = mean_of(dot[0], a.H, a.inv_h, a.h_pow2);
+    // pass 2
+    const int64_t off = row * nv + t;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      if (act && (EXACT || k * T + t < nv)) {
+        float xf[VE], df[VE], zf[VE], dxv[VE], dzv[VE], gk[VE];
+        F::unpack(x[k], xf);
+        F::unpack(d[k], df);
+        if constexpr (GATED) F::unpack(z[k], zf);
+        gain(k, gk);
+#pragma unroll
+        for (int e = 0; e < VE; ++e) {
+          const float xh = __fmul_rn(xf[e], rs);                  // same bits as pass 1
+          const float q = __fmul_rn(df[e], xh);                   // dy * xh
+          if constexpr (GATED) {
+            const float s = sg[k][e];
+            const float silu = __fmul_rn(zf[e], s);
+            const float gd = __fmul_rn(__fmul_rn(gk[e], silu), df[e]);
+            dxv[e] = __fmul_rn(rs, __fmaf_rn(-xh, m, gd));       // rstd*(g*dy - xh*m)
+            const float d1 = __fmaf_rn(zf[e], __fsub_rn(1.0f, s), 1.0f);
+            dzv[e] = __fmul_rn(__fmul_rn(__fmul_rn(q, gk[e]), s), d1);
+            acc[k][e] = __fadd_rn(acc[k][e], __fmul_rn(q, silu));
+          } else {
+            const float gd = __fmul_rn(gk[e], df[e]);
+            dxv[e] = __fmul_rn(rs, __fmaf_rn(-xh, m, gd));
+            acc[k][e] = __fadd_rn(acc[k][e], q);
+          }
+        }
+        st_stream(a.dx + off + k * T, F::pack(dxv));
+        if constexpr (GATED) st_stream(a.dz + off + k * T, F::pack(dzv));
+      }
+    }
+  };
+
+  const int64_t n_leaves = (a.rows + kLeafRows - 1) / kLeafRows;
+  const int64_t n_groups = (n_leaves + NT - 1) / NT;
+  for (int64_t grp = blockIdx.x; grp < n_groups; grp += gridDim.x) {
+    const int64_t r0 = (grp * NT + team) * kLeafRows;
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+#pragma unroll
+      for (int e = 0; e < VE; ++e) acc[k][e] = -0.0f;
+
+    uint4 ax[K], az[K], ad[K], bx[K], bz[K], bd[K];
+    float ar, br;
+    fetch(r0, r0 < a.rows, ax, az, ad, ar);
+    for (int i = 0; i < kLeafRows; i += 2) {
+      const int64_t row = r0 + i;
+      fetch(row + 1, row + 1 < a.rows, bx, bz, bd, br);
+      process(row, row < a.rows, ax, az, ad, ar);
+      fetch(row + 2, i + 2 < kLeafRows && row + 2 < a.rows, ax, az, ad, ar);
+      process(row + 1, row + 1 < a.rows, bx, bz, bd, br);
+    }
+
+    // join the CTA's leaves (aligned power-of-two group) with the pairwise tree
+    const int64_t rem = n_leaves - grp * NT;
+    join_leaves<VE, K, T, EXACT>(acc, NT, rem < NT ? int(rem) : NT, team, t, nv, a.H, leafbuf,
+                                 a.part + grp * a.H);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Backward for sub-warp teams (T <= 16, K <= 2: widths up to 256 bf16 / 128
+// fp32).  Same arithmetic and order as k_bwd; the difference is the data
+// path: each thread stages its own x, dy (z) vectors and rstd through shared
+// memory with cp.async, kBwdStages - 1 rows ahead of the row it computes, so
+// no registers hold prefetched rows and pass 2 keeps xh, g*dy and s from
+// pass 1 instead of recomputing them.  Every thread reads back only what it
+// copied itself (cp.async.wait_group makes its own copies visible to it), so
+// the pipeline needs no barrier.
+// ---------------------------------------------------------------------------
+constexpr int kBwdStages = 3;
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
+  const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+template <int T>
+__host__ __device__ constexpr int bwds_min_blocks() { return T <= 8 ? 7 : (T == 16 ? 6 : 1); }
+
+template <int DT, int T, int K, bool GATED, bool EXACT>
+__global__ void __launch_bounds__(8 * T, bwds_min_blocks<T>())
+k_bwd_s(const BwdArgs a) {
+  using F = Fmt<DT>;
+  constexpr int VE = F::VE;
+  constexpr int S = kBwdStages;
+  constexpr int NTEN = GATED ? 3 : 2;   // staged tensors: x, dy (, z)
+  // dynamic shared memory: gain [H] | stages [S][NTEN][K][blockDim] uint4 |
+  // leaf partials [NT][H] | rstd stages [S][blockDim]
+  extern __shared__ float dsm[];
+  const int bd = blockDim.x;
+  const int NT = bd / T;
+  const int tid = threadIdx.x;
+  float* gsm = dsm;
+  uint4* stg = reinterpret_cast<uint4*>(dsm + a.H);
+  float* leafbuf = reinterpret_cast<float*>(stg + S * NTEN * K * bd);
+  float* rsm = leafbuf + (NT > 1 ? NT * a.H : 0);
+  const int team = tid / T, t = tid % T;
+  const int nv = a.nv;
+  const unsigned mask = bd >= 32 ? 0xffffffffu : ((1u << bd) - 1u);
+  const bool have_rstd = a.rstd != nullptr;
+  int phase = 0;   // unused: T <= 32 reduces with shuffles only
+
+  for (int c = tid; c < a.H; c += bd) gsm[c] = GATED ? __ldg(a.w + c) : __fadd_rn(1.0f, __ldg(a.w + c));
+  __syncthreads();
+  auto gain = [&](int k, float (&g)[VE]) {
+    const float4* p = reinterpret_cast<const float4*>(gsm) + (k * T + t) * (VE / 4);
+#pragma unroll
+    for (int q = 0; q < VE / 4; ++q) {
+      const float4 f = p[q];
+      g[4 * q] = f.x; g[4 * q + 1] = f.y; g[4 * q + 2] = f.z; g[4 * q + 3] = f.w;
+    }
+  };
+  auto slot = [&](int sl, int ten, int k) -> uint4* { return stg + ((sl * NTEN + ten) * K + k) * bd + tid; };
+
+  // stage row `row` (if act) into slot sl, then close the copy group
+  auto issue = [&](int64_t row, bool act, int sl) {
+    if (act) {
+      const int64_t off = row * nv + t;
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        if (EXACT || k * T + t < nv) {
+          cp_async16(slot(sl, 0, k), a.x + off + k * T);
+          cp_async16(slot(sl, 1, k), a.dy + off + k * T);
+          if constexpr (GATED) cp_async16(slot(sl, 2, k), a.z + off + k * T);
+        }
+      }
+      if (have_rstd) cp_async4(rsm + sl * bd + tid, a.rstd + row);
+    }
+    cp_async_commit();
+  };
 
   const int64_t n_leaves = (a.rows + kLeafRows - 1) / kLeafRows;
   const int64_t n_groups = (n_leaves + NT - 1) / NT;
@@ -319,159 +623,95 @@ k_bwd(const BwdArgs a) {
 #pragma unroll
       for (int e = 0; e < VE; ++e) acc[k][e] = -0.0f;
 
-    for (int i = 0; i < kLeafRows; i += U) {
-      uint4 xr[U][K], zr[U][K], dr[U][K];
-      float rs[U];
-      bool act[U];
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t row = r0 + i + u;
-        act[u] = row < a.rows;
-#pragma unroll
-        for (int k = 0; k < K; ++k) {
-          const int v = k * T + t;
-          const bool ok = act[u] && v < nv;
-          xr[u][k] = ok ? ld_stream(a.x + row * nv + v) : make_uint4(0, 0, 0, 0);
-          dr[u][k] = ok ? ld_stream(a.dy + row * nv + v) : make_uint4(0, 0, 0, 0);
-          if constexpr (GATED) zr[u][k] = ok ? ld_stream(a.z + row * nv + v) : make_uint4(0, 0, 0, 0);
-        }
-        rs[u] = (act[u] && a.rstd != nullptr) ? __ldcs(a.rstd + row) : 0.0f;
+    for (int i = 0; i < S - 1; ++i) issue(r0 + i, r0 + i < a.rows, i);
+    int sl = 0;
+    for (int i = 0; i < kLeafRows; ++i) {
+      const int64_t row = r0 + i;
+      const bool act = row < a.rows;
+      {
+        const int ahead = i + S - 1;
+        int sa = sl + S - 1;
+        if (sa >= S) sa -= S;
+        issue(r0 + ahead, ahead < kLeafRows && r0 + ahead < a.rows, sa);
       }
-      if (a.rstd == nullptr) {   // uniform branch: recompute exactly as the forward does
-        float ss[U];
+      cp_async_wait<S - 1>();
+      uint4 xr[K], dr[K], zr[K];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          ss[u] = -0.0f;
+      for (int k = 0; k < K; ++k) {
+        xr[k] = *slot(sl, 0, k);
+        dr[k] = *slot(sl, 1, k);
+        if constexpr (GATED) zr[k] = *slot(sl, 2, k);
+      }
+      float rs;
+      if (have_rstd) {
+        rs = rsm[sl * bd + tid];
+      } else {   // uniform branch: recompute exactly as the forward does
+        float ss[1] = {thread_sumsq<DT, T, K, EXACT>(xr, nv, t)};
+        team_sum<T, 1>(ss, nullptr, phase, team, NT, mask);
+        rs = rsqrtf(__fadd_rn(mean_of(ss[0], a.H, a.inv_h, a.h_pow2), a.eps));
+      }
+      // pass 1: keep xh, g*dy and s for pass 2
+      float xh[K][VE], gd[K][VE], sg[K][GATED ? VE : 1];
+      float dot[1] = {-0.0f};
 #pragma unroll
-          for (int k = 0; k < K; ++k) {
-            if (k * T + t < nv) {
-              float f[VE];
-              F::unpack(xr[u][k], f);
+      for (int k = 0; k < K; ++k) {
+        float xf[VE], df[VE], zf[VE], gk[VE];
+        F::unpack(xr[k], xf);
+        F::unpack(dr[k], df);
+        if constexpr (GATED) F::unpack(zr[k], zf);
+        gain(k, gk);
 #pragma unroll
-              for (int e = 0; e < VE; ++e) ss[u] = __fmaf_rn(f[e], f[e], ss[u]);
-            }
+        for (int e = 0; e < VE; ++e) {
+          xh[k][e] = __fmul_rn(xf[e], rs);
+          float g;
+          if constexpr (GATED) {
+            sg[k][e] = sigmoid_f(zf[e]);
+            g = __fmul_rn(gk[e], __fmul_rn(zf[e], sg[k][e]));   // w * silu(z)
+          } else {
+            g = gk[e];                                          // 1 + w
           }
+          gd[k][e] = __fmul_rn(g, df[e]);
+          if (EXACT || k * T + t < nv) dot[0] = __fmaf_rn(gd[k][e], xh[k][e], dot[0]);
         }
-        team_sum<T, U>(ss, red, phase, team, NT, mask);
-#pragma unroll
-        for (int u = 0; u < U; ++u) rs[u] = rstd_from_sumsq(ss[u], Hf, a.eps);
       }
-
-      // pass 1: the dot sum_j (g_j * dy_j) * xh_j, with xh = x*rstd and
-      // g = 1 + w or w * silu(z); sigmoid(z) is kept for pass 2
-      float sg[U][K][GATED ? VE : 1];
-      float dot[U];
+      team_sum<T, 1>(dot, nullptr, phase, team, NT, mask);
+      const float m = mean_of(dot[0], a.H, a.inv_h, a.h_pow2);
+      // pass 2: dx, dz, and the leaf's dw fold (rows in ascending order)
+      const int64_t off = row * nv + t;
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        dot[u] = -0.0f;
-#pragma unroll
-        for (int k = 0; k < K; ++k) {
-          float xf[VE], df[VE], zf[VE];
-          F::unpack(xr[u][k], xf);
-          F::unpack(dr[u][k], df);
-          if constexpr (GATED) F::unpack(zr[u][k], zf);
-          const bool valid = k * T + t < nv;
+      for (int k = 0; k < K; ++k) {
+        if (act && (EXACT || k * T + t < nv)) {
+          float df[VE], zf[VE], dxv[VE], dzv[VE], gk[VE];
+          F::unpack(dr[k], df);
+          if constexpr (GATED) {
+            F::unpack(zr[k], zf);
+            gain(k, gk);
+          }
 #pragma unroll
           for (int e = 0; e < VE; ++e) {
-            const float xh = __fmul_rn(xf[e], rs[u]);
-            float g;
+            dxv[e] = __fmul_rn(rs, __fmaf_rn(-xh[k][e], m, gd[k][e]));   // rstd*(g*dy - xh*m)
+            const float q = __fmul_rn(df[e], xh[k][e]);                   // dy * xh
             if constexpr (GATED) {
-              sg[u][k][e] = sigmoid_f(zf[e]);
-              g = __fmul_rn(gw[k][e], __fmul_rn(zf[e], sg[u][k][e]));   // w * silu(z)
+              const float sv = sg[k][e];
+              const float d1 = __fmaf_rn(zf[e], __fsub_rn(1.0f, sv), 1.0f);
+              dzv[e] = __fmul_rn(__fmul_rn(__fmul_rn(q, gk[e]), sv), d1);   // dy*xh*w*s*(1+z(1-s))
+              acc[k][e] = __fadd_rn(acc[k][e], __fmul_rn(q, __fmul_rn(zf[e], sv)));
             } else {
-              g = gw[k][e];                                              // 1 + w
+              acc[k][e] = __fadd_rn(acc[k][e], q);
             }
-            if (valid) dot[u] = __fmaf_rn(__fmul_rn(g, df[e]), xh, dot[u]);
           }
+          st_stream(a.dx + off + k * T, F::pack(dxv));
+          if constexpr (GATED) st_stream(a.dz + off + k * T, F::pack(dzv));
         }
       }
-      team_sum<T, U>(dot, red, phase, team, NT, mask);
-
-      // pass 2: dx, dz, and the leaf's dw fold (rows in ascending order)
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t row = r0 + i + u;
-        const float m = __fdiv_rn(dot[u], Hf);
-#pragma unroll
-        for (int k = 0; k < K; ++k) {
-          const int v = k * T + t;
-          if (act[u] && v < nv) {
-            float xf[VE], df[VE], zf[VE], dxv[VE], dzv[VE];
-            F::unpack(xr[u][k], xf);
-            F::unpack(dr[u][k], df);
-            if constexpr (GATED) F::unpack(zr[u][k], zf);
-#pragma unroll
-            for (int e = 0; e < VE; ++e) {
-              const float xh = __fmul_rn(xf[e], rs[u]);                 // same bits as pass 1
-              const float q = __fmul_rn(df[e], xh);                     // dy * xh
-              if constexpr (GATED) {
-                const float s = sg[u][k][e];
-                const float silu = __fmul_rn(zf[e], s);
-                const float gd = __fmul_rn(__fmul_rn(gw[k][e], silu), df[e]);
-                // dx = rstd * (g*dy - xh*m)
-                dxv[e] = __fmul_rn(rs[u], __fmaf_rn(-xh, m, gd));
-                // dz = dy*xh*w*s*(1 + z*(1-s))
-                const float d1 = __fmaf_rn(zf[e], __fsub_rn(1.0f, s), 1.0f);
-                dzv[e] = __fmul_rn(__fmul_rn(__fmul_rn(q, gw[k][e]), s), d1);
-                acc[k][e] = __fadd_rn(acc[k][e], __fmul_rn(q, silu));
-              } else {
-                const float gd = __fmul_rn(gw[k][e], df[e]);
-                dxv[e] = __fmul_rn(rs[u], __fmaf_rn(-xh, m, gd));
-                acc[k][e] = __fadd_rn(acc[k][e], q);
-              }
-            }
-            st_stream(a.dx + row * nv + v, F::pack(dxv));
-            if constexpr (GATED) st_stream(a.dz + row * nv + v, F::pack(dzv));
-          }
-        }
-      }
+      if (++sl == S) sl = 0;
     }
+    cp_async_wait<0>();   // no copy may be in flight into slots the next group reuses
 
-    // join the CTA's leaves (aligned power-of-two group) with the pairwise tree
     const int64_t rem = n_leaves - grp * NT;
-    const int nl = rem < NT ? int(rem) : NT;
-    float4* out4 = reinterpret_cast<float4*>(a.part + grp * a.H);
-    if (NT == 1) {
-#pragma unroll
-      for (int k = 0; k < K; ++k) {
-        const int v = k * T + t;
-        if (v < nv) {
-#pragma unroll
-          for (int q = 0; q < VE / 4; ++q)
-            out4[v * (VE / 4) + q] = make_float4(acc[k][4 * q], acc[k][4 * q + 1],
-                                                 acc[k][4 * q + 2], acc[k][4 * q + 3]);
-        }
-      }
-    } else {
-      __syncthreads();   // the previous group's readers of leafbuf are done
-      float4* lb4 = reinterpret_cast<float4*>(leafbuf + team * a.H);
-#pragma unroll
-      for (int k = 0; k < K; ++k) {
-        const int v = k * T + t;
-        if (v < nv) {
-#pragma unroll
-          for (int q = 0; q < VE / 4; ++q)
-            lb4[v * (VE / 4) + q] = make_float4(acc[k][4 * q], acc[k][4 * q + 1],
-                                                acc[k][4 * q + 2], acc[k][4 * q + 3]);
-        }
-      }
-      __syncthreads();
-      const int H4 = a.H / 4;
-      const float4* all4 = reinterpret_cast<const float4*>(leafbuf);
-      for (int c = threadIdx.x; c < H4; c += blockDim.x) {
-        float4 p[8];
-#pragma unroll
-        for (int l = 0; l < 8; ++l)
-          p[l] = l < NT ? all4[l * H4 + c] : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int s = 1; s < 8; s <<= 1) {
-#pragma unroll
-          for (int l = 0; l + s < 8; l += 2 * s)
-            if (l + s < nl) p[l] = add4(p[l], p[l + s]);
-        }
-        out4[c] = p[0];
-      }
-    }
+    join_leaves<VE, K, T, EXACT>(acc, NT, rem < NT ? int(rem) : NT, team, t, nv, a.H, leafbuf,
+                                 a.part + grp * a.H);
   }
 }
 
@@ -548,6 +788,15 @@ k_fold(const float* __restrict__ in, int64_t n, int H, float* __restrict__ out) 
   }
 }
 
+// Test kernel: the reciprocal used by the sigmoid, for checking against IEEE
+// division over every float in [1, 2].
+__global__ void k_test_rcp(const float* __restrict__ d, float* __restrict__ out, int64_t n,
+                           int steps) {
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n;
+       i += int64_t(gridDim.x) * blockDim.x)
+    out[i] = steps == 1 ? rcp_1to2<1>(d[i]) : rcp_1to2<2>(d[i]);
+}
+
 // ---------------------------------------------------------------------------
 // host side: schedule, validation, launch
 // ---------------------------------------------------------------------------
@@ -569,7 +818,9 @@ bool pick_sched(int32_t width, rn_dtype dt, Sched* s) {
   if (!width_ok(width) || (dt != RN_BF16 && dt != RN_F32)) return false;
   const int VE = dt == RN_BF16 ? 8 : 4;
   const int nv = width / VE;
-  if (nv <= 32) { s->T = pow2ceil(nv); s->K = 1; }
+  // up to 32 vectors: two vectors (32 B) per thread, so a 128-wide bf16 row
+  // is 8 lanes x 16 elements
+  if (nv <= 32) { s->T = pow2ceil(nv) / 2 > 1 ? pow2ceil(nv) / 2 : 1; s->K = (nv + s->T - 1) / s->T; }
   else if (nv <= 128) { s->T = 32; s->K = (nv + 31) / 32; }
   else if (nv <= 512) { s->T = 128; s->K = (nv + 127) / 128; }
   else if (nv <= 2048) { s->T = 512; s->K = (nv + 511) / 512; }
@@ -578,7 +829,6 @@ bool pick_sched(int32_t width, rn_dtype dt, Sched* s) {
 }
 
 int bwd_max_block_rt(int T) { return T <= 32 ? 8 * T : (T <= 128 ? 256 : T); }
-int bwd_rows_per_step_rt(int T) { return T <= 32 ? 2 : 1; }
 int fwd_block_rt(int T) { return T <= 32 ? 256 : T; }
 int fwd_rows_per_cta_rt(int T) { return T <= 32 ? (256 / T) * 2 : 1; }
 
@@ -586,6 +836,22 @@ std::atomic<int> g_max_ctas{0}, g_leaves_per_cta{0}, g_fold_rows{0}, g_validate_
 thread_local int t_last_cuda = 0;
 thread_local char t_describe[512];
 
+
+bool bwd_pipelined(const Sched& s) { return s.T <= 16; }
+
+size_t bwd_smem_bytes(const Sched& s, int lpc, int width, bool gated) {
+  const size_t leaves = lpc > 1 ? size_t(lpc) * width * sizeof(float) : 0;
+  if (bwd_pipelined(s)) {   // k_bwd_s: gain, staged rows, leaf partials, staged rstd
+    const size_t bd = size_t(lpc) * s.T;
+    return size_t(width) * sizeof(float) + size_t(kBwdStages) * (gated ? 3 : 2) * s.K * bd * 16 +
+           leaves + size_t(kBwdStages) * bd * sizeof(float);
+  }
+  const int W = s.T > 32 ? s.T / 32 : 1;
+  size_t f = (s.T <= 32 ? size_t(width) : 0) + (s.T > 32 ? size_t(2) * lpc * W : 0);
+  return f * sizeof(float) + leaves;
+}
+
+// (sized for the gated op's staging, so both ops use the same geometry)
 int leaves_per_cta(const Sched& s, int width) {
   const int maxb = bwd_max_block_rt(s.T);
   int lpc = maxb / s.T;                                   // default: fill the block
@@ -593,14 +859,8 @@ int leaves_per_cta(const Sched& s, int width) {
   const int req = g_leaves_per_cta.load();
   if (req > 0) lpc = req < lpc ? req : lpc;
   if (lpc > 8) lpc = 8;
+  while (lpc > 1 && bwd_smem_bytes(s, lpc, width, true) > 48 * 1024) lpc /= 2;
   return lpc;
-}
-
-size_t bwd_smem_bytes(const Sched& s, int lpc, int width) {
-  const int U = bwd_rows_per_step_rt(s.T);
-  const int W = s.T > 32 ? s.T / 32 : 1;
-  size_t f = (s.T > 32 ? size_t(2) * lpc * U * W : 0) + (lpc > 1 ? size_t(lpc) * width : 0);
-  return f * sizeof(float);
 }
 
 int grid_cap(int64_t want) {
@@ -663,17 +923,23 @@ rn_status launch_status() {
 
 // ---- dispatch over the (T, K) pairs pick_sched can return -----------------
 #define RN_TK_LIST(X) \
-  X(1, 1) X(2, 1) X(4, 1) X(8, 1) X(16, 1) X(32, 1) X(32, 2) X(32, 3) X(32, 4) \
+  X(1, 1) X(1, 2) X(2, 2) X(4, 2) X(8, 2) X(16, 2) X(32, 2) X(32, 3) X(32, 4) \
   X(128, 2) X(128, 3) X(128, 4) X(512, 2) X(512, 3) X(512, 4) X(1024, 3) X(1024, 4)
+// the sub-warp teams, which use the pipelined backward k_bwd_s
+#define RN_TK_SMALL(X) X(1, 1) X(1, 2) X(2, 2) X(4, 2) X(8, 2) X(16, 2)
 
 template <int DT, bool GATED>
 rn_status launch_fwd(const Sched& s, const FwdArgs& a, cudaStream_t st) {
   const int64_t per_cta = fwd_rows_per_cta_rt(s.T);
   const int grid = grid_cap((a.rows + per_cta - 1) / per_cta);
   const int block = fwd_block_rt(s.T);
+  const bool exact = a.nv == s.T * s.K;
 #define RN_FWD_CASE(T_, K_)                                                     \
   if (s.T == T_ && s.K == K_) {                                                 \
-    k_fwd<DT, T_, K_, GATED><<<grid, block, 0, st>>>(a);                        \
+    if (exact)                                                                  \
+      k_fwd<DT, T_, K_, GATED, true><<<grid, block, 0, st>>>(a);                \
+    else                                                                        \
+      k_fwd<DT, T_, K_, GATED, false><<<grid, block, 0, st>>>(a);               \
     return launch_status();                                                     \
   }
   RN_TK_LIST(RN_FWD_CASE)
@@ -685,20 +951,42 @@ template <int DT, bool GATED>
 rn_status launch_bwd(const Sched& s, int lpc, const BwdArgs& a, int64_t groups, cudaStream_t st) {
   const int grid = grid_cap(groups);
   const int block = lpc * s.T;
-  const size_t smem = bwd_smem_bytes(s, lpc, a.H);
+  const size_t smem = bwd_smem_bytes(s, lpc, a.H, GATED);
+  const bool exact = a.nv == s.T * s.K;
+  if (bwd_pipelined(s)) {
+#define RN_BWDS_CASE(T_, K_)                                                    \
+    if (s.T == T_ && s.K == K_) {                                               \
+      if (exact)                                                                \
+        k_bwd_s<DT, T_, K_, GATED, true><<<grid, block, smem, st>>>(a);         \
+      else                                                                      \
+        k_bwd_s<DT, T_, K_, GATED, false><<<grid, block, smem, st>>>(a);        \
+      return launch_status();                                                   \
+    }
+    RN_TK_SMALL(RN_BWDS_CASE)
+#undef RN_BWDS_CASE
+    return RN_E_WIDTH;
+  }
 #define RN_BWD_CASE(T_, K_)                                                     \
-  if (s.T == T_ && s.K == K_) {                                                 \
-    k_bwd<DT, T_, K_, GATED><<<grid, block, smem, st>>>(a);                     \
-    return launch_status();                                                     \
+  if constexpr (T_ > 16) {                                                      \
+    if (s.T == T_ && s.K == K_) {                                               \
+      if (exact)                                                                \
+        k_bwd<DT, T_, K_, GATED, true><<<grid, block, smem, st>>>(a);           \
+      else                                                                      \
+        k_bwd<DT, T_, K_, GATED, false><<<grid, block, smem, st>>>(a);          \
+      return launch_status();                                                   \
+    }                                                                           \
   }
   RN_TK_LIST(RN_BWD_CASE)
 #undef RN_BWD_CASE
   return RN_E_WIDTH;
 }
 
+// rows of partials per fold CTA: one pass when there are few, else passes of
+// 32 so the first pass spreads over many CTAs (each thread then streams 4 rows)
 int fold_rows_default(int64_t n) {
+  if (n > 256) return 32;
   int64_t s = 8;
-  while (s < n && s < 256) s <<= 1;
+  while (s < n) s <<= 1;
   return int(s);
 }
 
@@ -787,7 +1075,10 @@ rn_status bwd_entry(int64_t rows, int32_t width, float eps, rn_dtype dt, const v
   const int64_t groups = (leaves + lpc - 1) / lpc;
   float* region_a = static_cast<float*>(ws);
   float* region_b = region_a + size_t(leaves) * width;
-  BwdArgs a{rows, width, eps, static_cast<const uint4*>(x), static_cast<const uint4*>(z), w,
+  const int VE = dt == RN_BF16 ? 8 : 4;
+  const bool pow2 = (width & (width - 1)) == 0;
+  BwdArgs a{rows, width, width / VE, eps, 1.0f / float(width), pow2 ? 1 : 0,
+            static_cast<const uint4*>(x), static_cast<const uint4*>(z), w,
             static_cast<const uint4*>(dy), rstd, static_cast<uint4*>(dx), static_cast<uint4*>(dz),
             groups == 1 ? dw : region_a};
   if (dt == RN_BF16)
@@ -818,7 +1109,10 @@ rn_status fwd_entry(int64_t rows, int32_t width, float eps, rn_dtype dt, const v
   if (g_validate_only.load() || rows == 0) return RN_OK;
   Sched s;
   pick_sched(width, dt, &s);
-  FwdArgs a{rows, width, eps, static_cast<const uint4*>(x), static_cast<const uint4*>(z), w,
+  const int VE = dt == RN_BF16 ? 8 : 4;
+  const bool pow2 = (width & (width - 1)) == 0;
+  FwdArgs a{rows, width, width / VE, eps, 1.0f / float(width), pow2 ? 1 : 0,
+            static_cast<const uint4*>(x), static_cast<const uint4*>(z), w,
             static_cast<uint4*>(y), rstd};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dt == RN_BF16) return launch_fwd<RN_BF16, GATED>(s, a, st);
@@ -910,5 +1204,15 @@ rn_status rn_test_set_geometry(int32_t max_ctas, int32_t leaves_per_cta_req, int
 }
 
 void rn_test_set_validate_only(int32_t on) { g_validate_only.store(on ? 1 : 0); }
+
+rn_status rn_test_rcp_1to2(int64_t n, const float* d, float* out, int32_t steps,
+                           rn_stream stream) {
+  if (n < 0 || (n > 0 && (!d || !out)) || (steps != 1 && steps != 2)) return RN_E_ARG;
+  if (n == 0 || g_validate_only.load()) return RN_OK;
+  const int64_t blocks = (n + 255) / 256;
+  k_test_rcp<<<int(blocks < 4096 ? blocks : 4096), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      d, out, n, steps);
+  return launch_status();
+}
 
 }  // extern "C"

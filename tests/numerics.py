@@ -6,8 +6,10 @@ the bar is 2 bf16 ulp per bf16 element and relative L2 <= 1e-4 for fp32 tensors)
   * bf16 y:        |gpu - ref| <= 2 ulp_bf16(|ref|)
   * bf16 dx, dz:   |gpu - ref| <= 2 ulp_bf16(|ref|) + 2**-16 * T
     where T is the size of the largest term that cancels in that element
-    (the oracle's cancellation scale); fp32 rounding of those terms is
-    amplified by the cancellation, and no bf16 rounding can hide it.
+    (the oracle's cancellation scale; for dx's mean term it is built from the
+    magnitudes of the row sum's terms, which bound that sum's rounding error);
+    fp32 rounding of those terms is amplified by the cancellation, and no bf16
+    rounding can hide it.
   * fp32 tensors:  ||gpu - ref||_2 / ||ref||_2 <= 1e-4
 """
 from __future__ import annotations
