@@ -130,6 +130,43 @@ __device__ __forceinline__ float4 add4(const float4& a, const float4& b) {
                      __fadd_rn(a.w, b.w));
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before its predecessor ends; griddep_wait() blocks
+// until the predecessor grid has completed and its writes are visible (it
+// returns at once for a normal launch).  griddep_trigger() lets the next such
+// kernel be scheduled.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void griddep_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
+// Gain vectors in "thread-major" order: float4 number (k*(VE/4) + q)*T + t is
+// the q-th float4 of thread t's k-th vector, so the threads of a team read
+// consecutive 16-byte words (no bank conflicts).  Holds K*T*VE floats.
+template <int VE, int K, int T, bool GATED>
+__device__ __forceinline__ void stage_gain(const float* __restrict__ w, int nv, float* gsm) {
+  float4* g4 = reinterpret_cast<float4*>(gsm);
+  constexpr int N = K * (VE / 4) * T;
+  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+    const int k = i / ((VE / 4) * T), q = (i / T) % (VE / 4), t = i % T;
+    const int v = k * T + t;
+    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (v < nv) f = __ldg(reinterpret_cast<const float4*>(w) + v * (VE / 4) + q);
+    if (!GATED) f = make_float4(__fadd_rn(1.0f, f.x), __fadd_rn(1.0f, f.y), __fadd_rn(1.0f, f.z),
+                                __fadd_rn(1.0f, f.w));
+    g4[i] = f;
+  }
+}
+template <int VE, int K, int T>
+__device__ __forceinline__ void read_gain(const float* gsm, int k, int t, float (&g)[VE]) {
+  const float4* g4 = reinterpret_cast<const float4*>(gsm);
+#pragma unroll
+  for (int q = 0; q < VE / 4; ++q) {
+    const float4 f = g4[(k * (VE / 4) + q) * T + t];
+    g[4 * q] = f.x; g[4 * q + 1] = f.y; g[4 * q + 2] = f.z; g[4 * q + 3] = f.w;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // team reduction: U independent sums at once (one per row in flight)
 // ---------------------------------------------------------------------------
@@ -253,21 +290,25 @@ __device__ __forceinline__ void load_row(uint4 (&r)[K], const uint4* __restrict_
   }
 }
 
-// Sum of squares of this thread's elements: ascending, fma, from -0.0.
+// Sum of squares of this thread's elements: each 16-byte vector folded in
+// ascending order with fma from -0.0, then the thread's K vector sums joined
+// by the pairwise tree (a vector the row does not reach contributes -0.0, the
+// identity).  K independent chains instead of one K*VE-long chain.
 template <int DT, int T, int K, bool EXACT>
 __device__ __forceinline__ float thread_sumsq(const uint4 (&x)[K], int nv, int t) {
   using F = Fmt<DT>;
-  float ss = -0.0f;
+  float p[K];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
+    p[k] = -0.0f;
     if (EXACT || k * T + t < nv) {
       float f[F::VE];
       F::unpack(x[k], f);
 #pragma unroll
-      for (int e = 0; e < F::VE; ++e) ss = __fmaf_rn(f[e], f[e], ss);
+      for (int e = 0; e < F::VE; ++e) p[k] = __fmaf_rn(f[e], f[e], p[k]);
     }
   }
-  return ss;
+  return pairwise_tree<K>(p);
 }
 
 // Writes the partial of this CTA's group of NT leaves (an aligned
@@ -402,6 +443,7 @@ k_bwd(const BwdArgs a) {
   const unsigned mask = blockDim.x >= 32 ? 0xffffffffu : ((1u << blockDim.x) - 1u);
   const bool have_rstd = a.rstd != nullptr;
   int phase = 0;
+  griddep_trigger();   // the dw fold may be scheduled; it waits for this grid
 
   float gw_r[WS ? 1 : K][WS ? 1 : VE];
   if constexpr (WS) {
@@ -448,9 +490,10 @@ k_bwd(const BwdArgs a) {
     }
     // pass 1: dot = sum_j (g_j * dy_j) * xh_j, xh = x*rstd, g = 1+w or w*silu(z)
     float sg[K][GATED ? VE : 1];
-    float dot[1] = {-0.0f};
+    float dp[K];   // per-vector dot partials, joined by the pairwise tree
 #pragma unroll
     for (int k = 0; k < K; ++k) {
+      dp[k] = -0.0f;
       float xf[VE], df[VE], zf[VE], gk[VE];
       F::unpack(x[k], xf);
       F::unpack(d[k], df);
@@ -466,9 +509,10 @@ k_bwd(const BwdArgs a) {
         } else {
           g = gk[e];                                             // 1 + w
         }
-        if (EXACT || k * T + t < nv) dot[0] = __fmaf_rn(__fmul_rn(g, df[e]), xh, dot[0]);
+        if (EXACT || k * T + t < nv) dp[k] = __fmaf_rn(__fmul_rn(g, df[e]), xh, dp[k]);
       }
     }
+    float dot[1] = {pairwise_tree<K>(dp)};
     team_sum<T, 1>(dot, red, phase, team, NT, mask);
     const float m = mean_of(dot[0], a.H, a.inv_h, a.h_pow2);
     // pass 2
@@ -533,7 +577,7 @@ k_bwd(const BwdArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Backward for sub-warp teams (T <= 16, K <= 2: widths up to 256 bf16 / 128
+// Backward for sub-warp teams (T <= 8, K <= 4: widths up to 256 bf16 / 128
 // fp32).  Same arithmetic and order as k_bwd; the difference is the data
 // path: each thread stages its own x, dy (z) vectors and rstd through shared
 // memory with cp.async, kBwdStages - 1 rows ahead of the row it computes, so
@@ -558,24 +602,26 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-template <int T>
-__host__ __device__ constexpr int bwds_min_blocks() { return T <= 8 ? 7 : (T == 16 ? 6 : 1); }
+// enough resident CTAs for one wave of 1024 (262144 rows of 128: 8192 leaves,
+// 8 per CTA) on 148 SMs, within the register file
+template <int T, int K>
+__host__ __device__ constexpr int bwds_min_blocks() { return T <= 4 ? 7 : (K <= 2 ? 7 : 4); }
 
 template <int DT, int T, int K, bool GATED, bool EXACT>
-__global__ void __launch_bounds__(8 * T, bwds_min_blocks<T>())
+__global__ void __launch_bounds__(8 * T, bwds_min_blocks<T, K>())
 k_bwd_s(const BwdArgs a) {
   using F = Fmt<DT>;
   constexpr int VE = F::VE;
   constexpr int S = kBwdStages;
   constexpr int NTEN = GATED ? 3 : 2;   // staged tensors: x, dy (, z)
-  // dynamic shared memory: gain [H] | stages [S][NTEN][K][blockDim] uint4 |
+  // dynamic shared memory: gain [K*T*VE] | stages [S][NTEN][K][blockDim] uint4 |
   // leaf partials [NT][H] | rstd stages [S][blockDim]
   extern __shared__ float dsm[];
   const int bd = blockDim.x;
   const int NT = bd / T;
   const int tid = threadIdx.x;
   float* gsm = dsm;
-  uint4* stg = reinterpret_cast<uint4*>(dsm + a.H);
+  uint4* stg = reinterpret_cast<uint4*>(dsm + K * T * VE);
   float* leafbuf = reinterpret_cast<float*>(stg + S * NTEN * K * bd);
   float* rsm = leafbuf + (NT > 1 ? NT * a.H : 0);
   const int team = tid / T, t = tid % T;
@@ -584,16 +630,10 @@ k_bwd_s(const BwdArgs a) {
   const bool have_rstd = a.rstd != nullptr;
   int phase = 0;   // unused: T <= 32 reduces with shuffles only
 
-  for (int c = tid; c < a.H; c += bd) gsm[c] = GATED ? __ldg(a.w + c) : __fadd_rn(1.0f, __ldg(a.w + c));
+  griddep_trigger();   // the dw fold may be scheduled; it waits for this grid
+  stage_gain<VE, K, T, GATED>(a.w, nv, gsm);
   __syncthreads();
-  auto gain = [&](int k, float (&g)[VE]) {
-    const float4* p = reinterpret_cast<const float4*>(gsm) + (k * T + t) * (VE / 4);
-#pragma unroll
-    for (int q = 0; q < VE / 4; ++q) {
-      const float4 f = p[q];
-      g[4 * q] = f.x; g[4 * q + 1] = f.y; g[4 * q + 2] = f.z; g[4 * q + 3] = f.w;
-    }
-  };
+  auto gain = [&](int k, float (&g)[VE]) { read_gain<VE, K, T>(gsm, k, t, g); };
   auto slot = [&](int sl, int ten, int k) -> uint4* { return stg + ((sl * NTEN + ten) * K + k) * bd + tid; };
 
   // stage row `row` (if act) into slot sl, then close the copy group
@@ -653,9 +693,10 @@ k_bwd_s(const BwdArgs a) {
       }
       // pass 1: keep xh, g*dy and s for pass 2
       float xh[K][VE], gd[K][VE], sg[K][GATED ? VE : 1];
-      float dot[1] = {-0.0f};
+      float dp[K];   // per-vector dot partials, joined by the pairwise tree
 #pragma unroll
       for (int k = 0; k < K; ++k) {
+        dp[k] = -0.0f;
         float xf[VE], df[VE], zf[VE], gk[VE];
         F::unpack(xr[k], xf);
         F::unpack(dr[k], df);
@@ -672,9 +713,10 @@ k_bwd_s(const BwdArgs a) {
             g = gk[e];                                          // 1 + w
           }
           gd[k][e] = __fmul_rn(g, df[e]);
-          if (EXACT || k * T + t < nv) dot[0] = __fmaf_rn(gd[k][e], xh[k][e], dot[0]);
+          if (EXACT || k * T + t < nv) dp[k] = __fmaf_rn(gd[k][e], xh[k][e], dp[k]);
         }
       }
+      float dot[1] = {pairwise_tree<K>(dp)};
       team_sum<T, 1>(dot, nullptr, phase, team, NT, mask);
       const float m = mean_of(dot[0], a.H, a.inv_h, a.h_pow2);
       // pass 2: dx, dz, and the leaf's dw fold (rows in ascending order)
@@ -715,6 +757,109 @@ k_bwd_s(const BwdArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Forward for sub-warp teams (T <= 8), persistent: the grid is one wave of
+// CTAs and each team walks rows (blockIdx.x + i*gridDim.x)*NT + team, staging
+// x (and z) through shared memory with cp.async kFwdStages - 1 rows ahead.
+// Per row the arithmetic is k_fwd's, in the same order.
+// ---------------------------------------------------------------------------
+constexpr int kFwdStages = 3;
+template <int K>
+__host__ __device__ constexpr int fwds_block() { return K <= 2 ? 128 : 64; }
+
+template <int DT, int T, int K, bool GATED, bool EXACT>
+__global__ void __launch_bounds__(fwds_block<K>(), K <= 2 ? 4 : 8)
+k_fwd_s(const FwdArgs a) {
+  constexpr int kFwdsBlock = fwds_block<K>();
+  using F = Fmt<DT>;
+  constexpr int VE = F::VE;
+  constexpr int S = kFwdStages;
+  constexpr int NTEN = GATED ? 2 : 1;   // staged tensors: x (, z)
+  constexpr int NT = kFwdsBlock / T;
+  // dynamic shared memory: gain [K*T*VE] (thread-major) | stages [S][NTEN][K][block] uint4
+  extern __shared__ float dsm[];
+  float* gsm = dsm;
+  uint4* stg = reinterpret_cast<uint4*>(dsm + K * T * VE);
+  const int tid = threadIdx.x, team = tid / T, t = tid % T;
+  const int nv = a.nv;
+  const unsigned mask = 0xffffffffu;
+  int phase = 0;   // unused: sub-warp teams reduce with shuffles only
+
+  stage_gain<VE, K, T, GATED>(a.w, nv, gsm);
+  __syncthreads();
+
+  auto slot = [&](int sl, int ten, int k) -> uint4* {
+    return stg + ((sl * NTEN + ten) * K + k) * kFwdsBlock + tid;
+  };
+  const int64_t nblk = (a.rows + NT - 1) / NT;
+  const int64_t iters = nblk > blockIdx.x ? (nblk - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  auto row_of = [&](int64_t i) { return (int64_t(blockIdx.x) + i * gridDim.x) * NT + team; };
+  auto issue = [&](int64_t i, int sl) {
+    if (i < iters) {
+      const int64_t row = row_of(i);
+      if (row < a.rows) {
+        const int64_t off = row * nv + t;
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+          if (EXACT || k * T + t < nv) {
+            cp_async16(slot(sl, 0, k), a.x + off + k * T);
+            if constexpr (GATED) cp_async16(slot(sl, 1, k), a.z + off + k * T);
+          }
+        }
+      }
+    }
+    cp_async_commit();
+  };
+
+#pragma unroll
+  for (int i = 0; i < S - 1; ++i) issue(i, i);
+  int sl = 0;
+  for (int64_t i = 0; i < iters; ++i) {
+    {
+      int sa = sl + S - 1;
+      if (sa >= S) sa -= S;
+      issue(i + S - 1, sa);
+    }
+    cp_async_wait<S - 1>();
+    uint4 xr[K], zr[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      xr[k] = *slot(sl, 0, k);
+      if constexpr (GATED) zr[k] = *slot(sl, 1, k);
+    }
+    const int64_t row = row_of(i);
+    const bool act = row < a.rows;
+    float ss[1] = {thread_sumsq<DT, T, K, EXACT>(xr, nv, t)};
+    team_sum<T, 1>(ss, nullptr, phase, team, NT, mask);
+    const float r = rsqrtf(__fadd_rn(mean_of(ss[0], a.H, a.inv_h, a.h_pow2), a.eps));
+    const int64_t off = row * nv + t;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      if (act && (EXACT || k * T + t < nv)) {
+        float f[VE], yv[VE], gk[VE];
+        F::unpack(xr[k], f);
+        read_gain<VE, K, T>(gsm, k, t, gk);
+        if constexpr (GATED) {
+          float zf[VE];
+          F::unpack(zr[k], zf);
+#pragma unroll
+          for (int e = 0; e < VE; ++e) {
+            const float act_z = __fmul_rn(zf[e], sigmoid_f(zf[e]));
+            yv[e] = __fmul_rn(__fmul_rn(__fmul_rn(f[e], r), gk[e]), act_z);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < VE; ++e) yv[e] = __fmul_rn(__fmul_rn(f[e], r), gk[e]);
+        }
+        st_stream(a.y + off + k * T, F::pack(yv));
+      }
+    }
+    if (act && t == 0 && a.rstd != nullptr) a.rstd[row] = r;
+    if (++sl == S) sl = 0;
+  }
+  cp_async_wait<0>();
+}
+
 // One fold pass: out[b] = pairwise tree of in[b*S, min(n, (b+1)*S)), S = kFoldRG * B.
 // CTA = 32 float4 columns x kFoldRG row groups; a thread streams B rows with
 // a binary counter (slot k holds a pending perfect subtree of 2^k rows), the
@@ -723,6 +868,8 @@ template <int B>
 __global__ void __launch_bounds__(32 * kFoldRG)
 k_fold(const float* __restrict__ in, int64_t n, int H, float* __restrict__ out) {
   constexpr int LB = (B >= 2) + (B >= 4) + (B >= 8) + (B >= 16) + (B >= 32);   // log2 B
+  griddep_trigger();   // a following fold pass may be scheduled
+  griddep_wait();      // the partials of the previous kernel are complete and visible
   const int lane = threadIdx.x & 31, rg = threadIdx.x >> 5;
   const int H4 = H / 4;
   const int c = blockIdx.y * 32 + lane;
@@ -818,9 +965,9 @@ bool pick_sched(int32_t width, rn_dtype dt, Sched* s) {
   if (!width_ok(width) || (dt != RN_BF16 && dt != RN_F32)) return false;
   const int VE = dt == RN_BF16 ? 8 : 4;
   const int nv = width / VE;
-  // up to 32 vectors: two vectors (32 B) per thread, so a 128-wide bf16 row
-  // is 8 lanes x 16 elements
-  if (nv <= 32) { s->T = pow2ceil(nv) / 2 > 1 ? pow2ceil(nv) / 2 : 1; s->K = (nv + s->T - 1) / s->T; }
+  // up to 32 vectors: up to four vectors (64 B) per thread, so a 128-wide
+  // bf16 row is 4 lanes x 32 elements
+  if (nv <= 32) { s->T = pow2ceil(nv) / 4 > 1 ? pow2ceil(nv) / 4 : 1; s->K = (nv + s->T - 1) / s->T; }
   else if (nv <= 128) { s->T = 32; s->K = (nv + 31) / 32; }
   else if (nv <= 512) { s->T = 128; s->K = (nv + 127) / 128; }
   else if (nv <= 2048) { s->T = 512; s->K = (nv + 511) / 512; }
@@ -843,7 +990,8 @@ size_t bwd_smem_bytes(const Sched& s, int lpc, int width, bool gated) {
   const size_t leaves = lpc > 1 ? size_t(lpc) * width * sizeof(float) : 0;
   if (bwd_pipelined(s)) {   // k_bwd_s: gain, staged rows, leaf partials, staged rstd
     const size_t bd = size_t(lpc) * s.T;
-    return size_t(width) * sizeof(float) + size_t(kBwdStages) * (gated ? 3 : 2) * s.K * bd * 16 +
+    // gain: K*T*VE floats (VE <= 8)
+    return size_t(s.K) * s.T * 8 * sizeof(float) + size_t(kBwdStages) * (gated ? 3 : 2) * s.K * bd * 16 +
            leaves + size_t(kBwdStages) * bd * sizeof(float);
   }
   const int W = s.T > 32 ? s.T / 32 : 1;
@@ -923,24 +1071,83 @@ rn_status launch_status() {
 
 // ---- dispatch over the (T, K) pairs pick_sched can return -----------------
 #define RN_TK_LIST(X) \
-  X(1, 1) X(1, 2) X(2, 2) X(4, 2) X(8, 2) X(16, 2) X(32, 2) X(32, 3) X(32, 4) \
-  X(128, 2) X(128, 3) X(128, 4) X(512, 2) X(512, 3) X(512, 4) X(1024, 3) X(1024, 4)
-// the sub-warp teams, which use the pipelined backward k_bwd_s
-#define RN_TK_SMALL(X) X(1, 1) X(1, 2) X(2, 2) X(4, 2) X(8, 2) X(16, 2)
+  X(32, 2) X(32, 3) X(32, 4) X(128, 2) X(128, 3) X(128, 4) X(512, 2) X(512, 3) X(512, 4) \
+  X(1024, 3) X(1024, 4)
+// the sub-warp teams, which use the pipelined kernels k_fwd_s and k_bwd_s
+#define RN_TK_SMALL(X) \
+  X(1, 1) X(1, 2) X(1, 3) X(1, 4) X(2, 3) X(2, 4) X(4, 3) X(4, 4) X(8, 3) X(8, 4)
+
+int sm_count() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  if (dev < 64) {
+    const int c = cached[dev].load();
+    if (c > 0) return c;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  if (dev < 64) cached[dev].store(n);
+  return n;
+}
+
+// Resident CTAs per SM of a kernel (cached per instantiation and smem size).
+template <typename Kern>
+int blocks_per_sm(Kern kernel, int block, size_t smem) {
+  int nb = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, block, smem) != cudaSuccess ||
+      nb <= 0) {
+    (void)cudaGetLastError();
+    nb = 1;
+  }
+  return nb;
+}
+
+template <int DT, int T, int K, bool GATED, bool EXACT>
+rn_status launch_fwd_s(const FwdArgs& a, cudaStream_t st) {
+  constexpr int NTEN = GATED ? 2 : 1;
+  constexpr int kFwdsBlock = fwds_block<K>();
+  const size_t smem = size_t(K) * T * (DT == RN_BF16 ? 8 : 4) * sizeof(float) +
+                      size_t(kFwdStages) * NTEN * K * kFwdsBlock * 16;
+  static std::atomic<int> per_sm{0};
+  int nb = per_sm.load();
+  if (nb <= 0) {
+    nb = blocks_per_sm(k_fwd_s<DT, T, K, GATED, EXACT>, kFwdsBlock, smem);
+    per_sm.store(nb);
+  }
+  const int64_t nblk = (a.rows + kFwdsBlock / T - 1) / (kFwdsBlock / T);
+  const int64_t wave = int64_t(nb) * sm_count();
+  const int grid = grid_cap(nblk < wave ? nblk : wave);
+  k_fwd_s<DT, T, K, GATED, EXACT><<<grid, kFwdsBlock, smem, st>>>(a);
+  return launch_status();
+}
 
 template <int DT, bool GATED>
 rn_status launch_fwd(const Sched& s, const FwdArgs& a, cudaStream_t st) {
+  if (s.T <= 16) {
+    const bool ex = a.nv == s.T * s.K;
+#define RN_FWDS_CASE(T_, K_)                                                    \
+    if (s.T == T_ && s.K == K_)                                                 \
+      return ex ? launch_fwd_s<DT, T_, K_, GATED, true>(a, st)                  \
+                : launch_fwd_s<DT, T_, K_, GATED, false>(a, st);
+    RN_TK_SMALL(RN_FWDS_CASE)
+#undef RN_FWDS_CASE
+    return RN_E_WIDTH;
+  }
   const int64_t per_cta = fwd_rows_per_cta_rt(s.T);
   const int grid = grid_cap((a.rows + per_cta - 1) / per_cta);
   const int block = fwd_block_rt(s.T);
   const bool exact = a.nv == s.T * s.K;
 #define RN_FWD_CASE(T_, K_)                                                     \
-  if (s.T == T_ && s.K == K_) {                                                 \
-    if (exact)                                                                  \
-      k_fwd<DT, T_, K_, GATED, true><<<grid, block, 0, st>>>(a);                \
-    else                                                                        \
-      k_fwd<DT, T_, K_, GATED, false><<<grid, block, 0, st>>>(a);               \
-    return launch_status();                                                     \
+  if constexpr (T_ > 16) {                                                      \
+    if (s.T == T_ && s.K == K_) {                                               \
+      if (exact)                                                                \
+        k_fwd<DT, T_, K_, GATED, true><<<grid, block, 0, st>>>(a);              \
+      else                                                                      \
+        k_fwd<DT, T_, K_, GATED, false><<<grid, block, 0, st>>>(a);             \
+      return launch_status();                                                   \
+    }                                                                           \
   }
   RN_TK_LIST(RN_FWD_CASE)
 #undef RN_FWD_CASE
@@ -1003,9 +1210,45 @@ int fold_passes(int64_t n) {
 
 // Folds n group partials (rows of width H in `a`) into dw, ping-ponging
 // between the two workspace regions a and b.
+// One fold pass, launched with programmatic stream serialization so that its
+// launch overlaps the end of the kernel it depends on (k_fold waits for it
+// with griddepcontrol.wait).  If the launch with the attribute is refused,
+// it is retried as an ordinary launch.
+template <int B>
+rn_status launch_fold_b(dim3 grid, cudaStream_t st, const float* in, int64_t n, int H, float* out) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(32 * kFoldRG);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k_fold<B>, in, n, H, out) == cudaSuccess) return launch_status();
+  (void)cudaGetLastError();
+  k_fold<B><<<grid, 32 * kFoldRG, 0, st>>>(in, n, H, out);
+  return launch_status();
+}
+
+rn_status launch_fold(int B, dim3 grid, cudaStream_t st, const float* in, int64_t n, int H,
+                      float* out) {
+  switch (B) {
+    case 1: return launch_fold_b<1>(grid, st, in, n, H, out);
+    case 2: return launch_fold_b<2>(grid, st, in, n, H, out);
+    case 4: return launch_fold_b<4>(grid, st, in, n, H, out);
+    case 8: return launch_fold_b<8>(grid, st, in, n, H, out);
+    case 16: return launch_fold_b<16>(grid, st, in, n, H, out);
+    case 32: return launch_fold_b<32>(grid, st, in, n, H, out);
+    default: return RN_E_ARG;
+  }
+}
+
 rn_status run_fold(float* a, float* b, int64_t n, int H, float* dw, cudaStream_t st) {
   float* src = a;
   float* dst = b;
+  rn_status e = RN_OK;
   while (n > 1) {
     int S = g_fold_rows.load();
     if (S <= 0) S = fold_rows_default(n);
@@ -1015,16 +1258,7 @@ rn_status run_fold(float* a, float* b, int64_t n, int H, float* dw, cudaStream_t
     const int gy = (H / 4 + 31) / 32;    // <= 128 column tiles
     if (nout > 0x7fffffff) return RN_E_ARG;   // unreachable for rows <= 2^36
     dim3 grid(unsigned(nout), gy);
-    switch (B) {
-      case 1: k_fold<1><<<grid, 32 * kFoldRG, 0, st>>>(src, n, H, o); break;
-      case 2: k_fold<2><<<grid, 32 * kFoldRG, 0, st>>>(src, n, H, o); break;
-      case 4: k_fold<4><<<grid, 32 * kFoldRG, 0, st>>>(src, n, H, o); break;
-      case 8: k_fold<8><<<grid, 32 * kFoldRG, 0, st>>>(src, n, H, o); break;
-      case 16: k_fold<16><<<grid, 32 * kFoldRG, 0, st>>>(src, n, H, o); break;
-      case 32: k_fold<32><<<grid, 32 * kFoldRG, 0, st>>>(src, n, H, o); break;
-      default: return RN_E_ARG;
-    }
-    const rn_status e = launch_status();
+    e = launch_fold(B, grid, st, src, n, H, o);
     if (e != RN_OK) return e;
     n = nout;
     float* tmp = src;

@@ -204,7 +204,7 @@ def test_workspace_bytes_invalid(lib):
     assert lib.norm_bwd_workspace_bytes(64, 100) == 0
 
 
-@pytest.mark.parametrize("width,dt,team", [(128, DType.BF16, 8), (128, DType.F32, 16),
+@pytest.mark.parametrize("width,dt,team", [(128, DType.BF16, 4), (128, DType.F32, 8),
                                            (8, DType.BF16, 1), (2048, DType.BF16, 128),
                                            (8192, DType.BF16, 512), (5120, DType.BF16, 512),
                                            (16384, DType.F32, 1024)])
