@@ -145,6 +145,41 @@ rn_status gated_norm_bwd(int64_t rows, int32_t width, float eps, rn_dtype dt,
                          float* dw, void* ws, size_t ws_bytes, rn_stream stream);
 
 /*
+ * Gated RMSNorm backward that allocates nothing: the same computation,
+ * arguments and results as gated_norm_bwd, but the dw-partial scratch is a
+ * fixed 8 MiB block of static device memory inside this library instead of a
+ * caller-supplied workspace.  (The paper has no counterpart of this call; it
+ * is an addition of this library.)
+ *
+ * Who needs it: hosts that hand a library only the input and output buffers of
+ * each call and own every other byte of device memory -- plugin interfaces,
+ * runtimes with a fixed memory plan, code that must not call cudaMalloc
+ * because it would synchronise the device or fall outside the host's memory
+ * accounting.  Such a caller has no workspace to pass and cannot allocate one.
+ *
+ * Limits and sharing:
+ *  - the scratch holds 8 MiB (8388608 bytes), so a call needs
+ *    norm_bwd_workspace_bytes(rows, width) <= 8388608 (e.g. 262144 rows of
+ *    width 128 use 4.7 MiB); larger shapes return RN_E_WORKSPACE and enqueue
+ *    nothing;
+ *  - every GPU on which this library runs kernels keeps the 8 MiB until the
+ *    process exits;
+ *  - the first call on each device looks up the scratch's device address (with
+ *    that device current) and keeps it; make that first call before any
+ *    stream capture;
+ *  - all calls on a device share the one scratch, which keeps whatever the last
+ *    call left there (nothing in it needs to start at zero).  Calls that can
+ *    run at the same time on the GPU -- on different streams, or from several
+ *    host threads -- race on it and give wrong dw; order them on one stream.
+ * The call never allocates or frees memory (no cudaMalloc/cudaFree, no
+ * allocating library routine).
+ */
+rn_status gated_norm_bwd_static_ws(int64_t rows, int32_t width, float eps, rn_dtype dt,
+                                   const void* x, const void* z, const float* w,
+                                   const void* dy, const float* rstd, void* dx, void* dz,
+                                   float* dw, rn_stream stream);
+
+/*
  * Provenance record (RFC #415 section 4, point 8): a static, NUL-terminated
  * string naming the kernels, the reduction schedule and tree, and the
  * accumulator for (width, dt); "unsupported" for an invalid pair.  The

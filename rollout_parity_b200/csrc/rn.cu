@@ -35,6 +35,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <mutex>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -1450,3 +1451,72 @@ rn_status rn_test_rcp_1to2(int64_t n, const float* d, float* out, int32_t steps,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Gated backward whose dw scratch lives in this library's own static device
+// memory, for callers that cannot allocate device memory (see the note on
+// gated_norm_bwd_static_ws in rn.h).  It only supplies the workspace pointer;
+// the work itself is gated_norm_bwd's, unchanged.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;   // 8 MiB on each GPU
+
+// Static dw-partial scratch.  Every GPU on which this library's kernels run
+// holds one copy until the process exits.  In host code this name refers to a
+// host-side stand-in, never to the device memory: its device address comes
+// from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::atomic<void*> g_static_scratch_addr[64];
+std::mutex g_static_scratch_mu;
+
+// Device address of g_static_scratch on the current device, looked up with that
+// device current the first time a call runs on it, then reused.
+rn_status static_scratch_address(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    t_last_cuda = int(e);
+    return RN_E_CUDA;
+  }
+  if (dev < 0 || dev >= 64) return RN_E_ARG;
+  void* p = g_static_scratch_addr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+    p = g_static_scratch_addr[dev].load(std::memory_order_relaxed);
+    if (p == nullptr) {
+      e = cudaGetSymbolAddress(&p, g_static_scratch);
+      if (e != cudaSuccess || p == nullptr) {
+        t_last_cuda = int(e);
+        return RN_E_CUDA;
+      }
+      g_static_scratch_addr[dev].store(p, std::memory_order_release);
+    }
+  }
+  *out = p;
+  return RN_OK;
+}
+
+}  // namespace
+
+extern "C" rn_status gated_norm_bwd_static_ws(int64_t rows, int32_t width, float eps,
+                                              rn_dtype dt, const void* x, const void* z,
+                                              const float* w, const void* dy, const float* rstd,
+                                              void* dx, void* dz, float* dw, rn_stream stream) {
+  rn_status e = common_checks(rows, width, eps, dt);
+  if (e != RN_OK) return e;
+  if (ws_bytes_of(rows, width) > kStaticScratchBytes) return RN_E_WORKSPACE;   // too large
+  void* ws = nullptr;
+  if (rows > 0) {
+    if (g_validate_only.load()) {
+      // checks only: any non-null, aligned stand-in lets the remaining checks run
+      ws = reinterpret_cast<void*>(uintptr_t(256));
+    } else {
+      e = static_scratch_address(&ws);
+      if (e != RN_OK) return e;
+    }
+  }
+  return bwd_entry<true>(rows, width, eps, dt, x, z, w, dy, rstd, dx, dz, dw, ws,
+                         kStaticScratchBytes, stream);
+}
