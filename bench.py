@@ -60,6 +60,10 @@ def parse():
     ap.add_argument("--no-invariance", action="store_true")
     ap.add_argument("--buffer-sets", type=int, default=SETS,
                     help="rotating input sets (fewer only for profiler captures)")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(workloads.CONFIGS),
+                    help="which synthetic workload one step runs (default: the headline)")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every call from Python instead of replaying a CUDA graph")
     return ap.parse_args()
 
 
@@ -159,6 +163,14 @@ class Clocks:
                 "samples": len(inside), "samples_outside_window": len(rows) - len(inside)}
 
 
+def graph_steps(k):
+    """Steps per captured graph: a divisor of k (so exactly k steps run), at most
+    256, preferring multiples of the buffer rotation (4)."""
+    divs = [d for d in range(1, min(k, 256) + 1) if k % d == 0]
+    rot = [d for d in divs if d % SETS == 0]
+    return max(rot) if rot else max(divs)
+
+
 def dist_setup(n):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if n > 1 or world > 1:
@@ -186,15 +198,19 @@ def run_ours(a):
     lib = rn.load()
 
     nsets = max(1, a.buffer_sets)
-    host = [workloads.cfg_gated_heads(seed=1000 * rank + s) for s in range(nsets)]
+    make = workloads.CONFIGS[a.workload]
+    host = [make(seed=1000 * rank + s) for s in range(nsets)]
     R, H, eps = host[0].rows, host[0].width, host[0].eps
-    fwd_b, bwd_b = bytes_model(R, H)
+    gated = host[0].gated
+    dtc = int(DType.BF16 if host[0].dtype == "bf16" else DType.F32)
+    esize = 2 if host[0].dtype == "bf16" else 4
+    fwd_b, bwd_b = bytes_model(R, H, esize=esize, gated=gated)
     step_b = fwd_b + bwd_b
     nws = lib.norm_bwd_workspace_bytes(R, H)
     sets = []
     for wl in host:
         d = wl.to(dev)
-        sets.append(dict(x=d.x, z=d.z, w=d.w, dy=d.dy, y=torch.empty_like(d.x),
+        sets.append(dict(x=d.x, z=d.z if gated else d.x, w=d.w, dy=d.dy, y=torch.empty_like(d.x),
                          rstd=torch.empty(R, dtype=torch.float32, device=dev),
                          dx=torch.empty_like(d.x), dz=torch.empty_like(d.x),
                          dw=torch.empty(H, dtype=torch.float32, device=dev),
@@ -202,14 +218,19 @@ def run_ours(a):
     P = [{k: v.data_ptr() for k, v in s.items()} for s in sets]
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
-    bf16 = int(DType.BF16)
 
-    def fwd(p):
-        return lib.gated_norm_fwd(R, H, eps, bf16, p["x"], p["z"], p["w"], p["y"], p["rstd"], sp)
+    def fwd(p, stp=sp):
+        if gated:
+            return lib.gated_norm_fwd(R, H, eps, dtc, p["x"], p["z"], p["w"], p["y"], p["rstd"],
+                                      stp)
+        return lib.norm_fwd(R, H, eps, dtc, p["x"], p["w"], p["y"], p["rstd"], stp)
 
-    def bwd(p):
-        return lib.gated_norm_bwd(R, H, eps, bf16, p["x"], p["z"], p["w"], p["dy"], p["rstd"],
-                                  p["dx"], p["dz"], p["dw"], p["ws"], nws, sp)
+    def bwd(p, stp=sp):
+        if gated:
+            return lib.gated_norm_bwd(R, H, eps, dtc, p["x"], p["z"], p["w"], p["dy"], p["rstd"],
+                                      p["dx"], p["dz"], p["dw"], p["ws"], nws, stp)
+        return lib.norm_bwd(R, H, eps, dtc, p["x"], p["w"], p["dy"], p["rstd"], p["dx"], p["dw"],
+                            p["ws"], nws, stp)
 
     for p in P:                       # every set gets its rstd before any backward
         check("gated_norm_fwd", fwd(p))
@@ -219,7 +240,31 @@ def run_ours(a):
     torch.cuda.synchronize()
 
     K = a.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    G = K if a.no_graph else graph_steps(K)
+    # per-call events: the last G steps of the timed region
+    ev = [[torch.cuda.Event(enable_timing=True, external=not a.no_graph) for _ in range(3)]
+          for _ in range(G)]
+    graph = None
+    if not a.no_graph:
+        # one CUDA graph holds G steps (calls and their event records); the
+        # timed region replays it K / G times
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.graph(graph, stream=cap):
+            csp = cap.cuda_stream
+            for j in range(G):
+                ev[j][0].record(cap)
+                s1 = fwd(P[j % nsets], csp)
+                ev[j][1].record(cap)
+                s2 = bwd(P[(j + 2) % nsets], csp)
+                ev[j][2].record(cap)
+                if s1 or s2:
+                    raise RuntimeError(f"capture failed: status {s1}, {s2}")
+        stream.wait_stream(cap)
+        for _ in range(max(1, a.warmup // G)):
+            graph.replay()
+        torch.cuda.synchronize()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = Clocks(dev)
     clocks.start()
@@ -228,16 +273,20 @@ def run_ours(a):
     torch.cuda.synchronize()
     clocks.mark("t0")
     t_start.record(stream)
-    for k in range(K):
-        e = ev[k]
-        e[0].record(stream)
-        s1 = fwd(P[k % nsets])
-        e[1].record(stream)
-        s2 = bwd(P[(k + 2) % nsets])
-        e[2].record(stream)
-        if s1 or s2:
-            check("gated_norm_fwd", s1)
-            check("gated_norm_bwd", s2)
+    if graph is not None:
+        for _ in range(K // G):
+            graph.replay()
+    else:
+        for k in range(K):
+            e = ev[k]
+            e[0].record(stream)
+            s1 = fwd(P[k % nsets])
+            e[1].record(stream)
+            s2 = bwd(P[(k + 2) % nsets])
+            e[2].record(stream)
+            if s1 or s2:
+                check("gated_norm_fwd", s1)
+                check("gated_norm_bwd", s2)
     t_end.record(stream)
     torch.cuda.synchronize()
     clocks.mark("t1")
@@ -245,18 +294,18 @@ def run_ours(a):
         dist.barrier()
     clk = clocks.stop()
     ms = t_start.elapsed_time(t_end)
-    fwd_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
-    bwd_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
+    fwd_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(G)]
+    bwd_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(G)]
     if dist is not None:
         t = torch.tensor([ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     ms_step = ms / K
     value = world * step_b * K / (ms / 1e3) / 1e9
-    launches = K * (1 + lib.rn_bwd_launches(R, H, bf16))
+    launches = K * (1 + lib.rn_bwd_launches(R, H, dtc))
 
-    inv = invariance_checks(rn, sets[0], R, H, eps) if rank == 0 and not a.no_invariance \
-        else None
+    inv = invariance_checks(rn, sets[0], R, H, eps, gated) \
+        if rank == 0 and not a.no_invariance else None
     e2e = run_e2e(rn, host[0], dev, a.e2e_steps, step_b, world, dist) if a.e2e_steps > 0 \
         else None
     cpu = None
@@ -269,16 +318,21 @@ def run_ours(a):
         fwd_mean = float(np.mean(fwd_ms))
         achieved = bwd_b / (bwd_mean / 1e3) / 1e9
         traffic = profiled_traffic()
+        desc = {WORKLOAD: {"layout": "8192 tokens x 32 heads, row = token*32 + head",
+                           "outliers": "1% of channels x50 in x, z, dy"}}.get(a.workload, {})
+        opname = "gated RMSNorm fwd+bwd" if gated else "zero-centred RMSNorm fwd+bwd"
+        iod = host[0].dtype
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": a.warmup, "ms_per_step": round(ms_step, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": iod,
             "data": "synthetic (seeded; no dataset or checkpoint)",
-            "config": {"workload": WORKLOAD, "op": "gated RMSNorm fwd+bwd", "rows": R,
-                       "width": H, "layout": "8192 tokens x 32 heads, row = token*32 + head",
-                       "outliers": "1% of channels x50 in x, z, dy", "eps": eps,
-                       "io_dtype": "bf16 x/z/dy/y/dx/dz, fp32 w/rstd/dw", "accumulate": "fp32",
+            "config": {"workload": a.workload, "op": opname, "rows": R, "width": H, **desc,
+                       "eps": eps, "io_dtype": f"{iod} x/z/dy/y/dx/dz, fp32 w/rstd/dw",
+                       "accumulate": "fp32",
                        "bytes_per_step": step_b, "parallelism": f"replicas x{world}",
+                       "launch": ("python loop" if a.no_graph else
+                                  f"CUDA graph of {G} steps replayed {K // G} times"),
                        "l2": (f"{nsets} rotating buffer sets (fwd on k%{nsets}, bwd on "
                               f"(k+2)%{nsets}): every buffer is re-touched only after >= 512 MB "
                               "of other traffic (L2 is 126 MB); no flush kernel")
@@ -289,7 +343,9 @@ def run_ours(a):
             "fwd_gbs": round(fwd_b / (fwd_mean / 1e3) / 1e9, 1),
             "bwd_gbs": round(achieved, 1),
             "invariance": inv,
-            "roofline": {"bound": "hbm", "kernel": "gated_norm_bwd call (k_bwd + k_fold passes)",
+            "roofline": {"bound": "hbm",
+                         "kernel": ("gated_norm_bwd" if gated else "norm_bwd") +
+                                   " call (k_bwd + k_fold passes)",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_source": src,
                          "traffic": traffic, "algorithmic_bytes": bwd_b},
@@ -302,28 +358,34 @@ def run_ours(a):
         dist.destroy_process_group()
 
 
-def invariance_checks(rn, s, R, H, eps):
+def invariance_checks(rn, s, R, H, eps, gated=True):
     """Bitwise: rows inside the full batch vs the same rows as their own batch,
     and dw across repeats and launch geometries."""
-    y, rstd = rn.gated_norm_fwd(s["x"], s["z"], s["w"], eps)
-    dx, dz, dw = rn.gated_norm_bwd(s["x"], s["z"], s["w"], s["dy"], rstd, eps)
+    def fb(x, z, dy):
+        if gated:
+            y, r = rn.gated_norm_fwd(x, z, s["w"], eps)
+            dx, dz, dw = rn.gated_norm_bwd(x, z, s["w"], dy, r, eps)
+            return [y, r, dx, dz], dw
+        y, r = rn.norm_fwd(x, s["w"], eps)
+        dx, dw = rn.norm_bwd(x, s["w"], dy, r, eps)
+        return [y, r, dx], dw
+
+    bits = lambda t: t.view(torch.int16 if t.dtype == torch.bfloat16 else torch.int32)
+    full, dw = fb(s["x"], s["z"], s["dy"])
     checks, bad = 0, 0
-    for st, n in ((12345, 1), (70001, 7), (R // 2 - 5, 4099), (R - 33, 33)):
+    for st, n in ((R // 3, 1), (R // 5, 7), (R // 2 - 5, min(4099, R // 2)), (R - 33, 33)):
+        if st < 0 or st + n > R:
+            continue
         sl = slice(st, st + n)
-        c = {k: s[k][sl].clone() for k in ("x", "z", "dy")}
-        y2, r2 = rn.gated_norm_fwd(c["x"], c["z"], s["w"], eps)
-        dx2, dz2, _ = rn.gated_norm_bwd(c["x"], c["z"], s["w"], c["dy"], r2, eps)
-        for a, b in ((y[sl], y2), (rstd[sl], r2), (dx[sl], dx2), (dz[sl], dz2)):
+        part, _ = fb(s["x"][sl].clone(), s["z"][sl].clone(), s["dy"][sl].clone())
+        for a_, b_ in zip([t[sl] for t in full], part):
             checks += 1
-            bad += int(not torch.equal(a.view(torch.int16 if a.dtype == torch.bfloat16
-                                              else torch.int32),
-                                       b.view(torch.int16 if b.dtype == torch.bfloat16
-                                              else torch.int32)))
+            bad += int(not torch.equal(bits(a_), bits(b_)))
     for geo in ((0, 0, 0), (148, 1, 8), (7, 2, 64), (0, 0, 0)):
         rn.rn_test_set_geometry(*geo)
-        _, _, dw2 = rn.gated_norm_bwd(s["x"], s["z"], s["w"], s["dy"], rstd, eps)
+        _, dw2 = fb(s["x"], s["z"], s["dy"])
         checks += 1
-        bad += int(not torch.equal(dw.view(torch.int32), dw2.view(torch.int32)))
+        bad += int(not torch.equal(bits(dw), bits(dw2)))
     rn.rn_test_set_geometry(0, 0, 0)
     torch.cuda.synchronize()
     return {"result": "pass" if bad == 0 else "fail", "bitwise_checks": checks, "failed": bad}
@@ -331,8 +393,10 @@ def invariance_checks(rn, s, R, H, eps):
 
 def run_e2e(rn, wl, dev, steps, step_b, world, dist):
     R, H, eps = wl.rows, wl.width, wl.eps
+    gated = wl.gated
     pin = lambda t: t.pin_memory()
-    hx, hz, hdy, hw = pin(wl.x), pin(wl.z), pin(wl.dy), pin(wl.w)
+    hx, hdy, hw = pin(wl.x), pin(wl.dy), pin(wl.w)
+    hz = pin(wl.z) if gated else None
     oy, ors = torch.empty_like(hx).pin_memory(), torch.empty(R, dtype=torch.float32).pin_memory()
     odx, odz = torch.empty_like(hx).pin_memory(), torch.empty_like(hx).pin_memory()
     odw = torch.empty(H, dtype=torch.float32).pin_memory()
@@ -345,20 +409,27 @@ def run_e2e(rn, wl, dev, steps, step_b, world, dist):
     dx, dz = torch.empty_like(x), torch.empty_like(x)
     dw = torch.empty(H, dtype=torch.float32, device=dev)
     ws = rn.workspace(R, H, dev)
-    h2d = sum(t.numel() * t.element_size() for t in (hx, hz, hdy, hw))
-    d2h = sum(t.numel() * t.element_size() for t in (oy, ors, odx, odz, odw))
+    h2d = sum(t.numel() * t.element_size() for t in (hx, hz, hdy, hw) if t is not None)
+    d2h = sum(t.numel() * t.element_size() for t in ((oy, ors, odx, odz, odw) if gated else
+                                                     (oy, ors, odx, odw)))
 
     def step():
         x.copy_(hx, non_blocking=True)
-        z.copy_(hz, non_blocking=True)
+        if gated:
+            z.copy_(hz, non_blocking=True)
         dy.copy_(hdy, non_blocking=True)
         w.copy_(hw, non_blocking=True)
-        rn.gated_norm_fwd(x, z, w, eps, y=y, rstd=rstd)
-        rn.gated_norm_bwd(x, z, w, dy, rstd, eps, dx=dx, dz=dz, dw=dw, ws=ws)
+        if gated:
+            rn.gated_norm_fwd(x, z, w, eps, y=y, rstd=rstd)
+            rn.gated_norm_bwd(x, z, w, dy, rstd, eps, dx=dx, dz=dz, dw=dw, ws=ws)
+        else:
+            rn.norm_fwd(x, w, eps, y=y, rstd=rstd)
+            rn.norm_bwd(x, w, dy, rstd, eps, dx=dx, dw=dw, ws=ws)
         oy.copy_(y, non_blocking=True)
         ors.copy_(rstd, non_blocking=True)
         odx.copy_(dx, non_blocking=True)
-        odz.copy_(dz, non_blocking=True)
+        if gated:
+            odz.copy_(dz, non_blocking=True)
         odw.copy_(dw, non_blocking=True)
 
     for _ in range(3):
@@ -379,13 +450,18 @@ def run_e2e(rn, wl, dev, steps, step_b, world, dist):
         ms = float(t.item())
     return {"value": round(world * step_b * steps / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": round(ms / steps, 4), "api": "rollout_parity_b200.gated_norm_fwd/bwd"}
+            "ms_per_step": round(ms / steps, 4),
+            "api": "rollout_parity_b200." + ("gated_norm_fwd/bwd" if gated else "norm_fwd/bwd")}
 
 
 # ---------------------------------------------------------------------------
 # the fp64 oracle on the host cores
 # ---------------------------------------------------------------------------
 def _oracle_step(orc, x, z, w, dy, eps):
+    if z is None:
+        orc.norm_fwd(x, w, eps)
+        orc.norm_bwd(x, w, dy, eps)
+        return
     orc.gated_norm_fwd(x, z, w, eps)
     orc.gated_norm_bwd(x, z, w, dy, eps)
 
@@ -394,6 +470,13 @@ def cpu_baseline(wl, fwd_b, bwd_b, min_s=10.0, max_s=30.0):
     import oracle
     f = workloads.as_f64
     x, z, w, dy = f(wl.x), f(wl.z), f(wl.w), f(wl.dy)
+    if wl.rows * wl.width > (1 << 26):        # bound host memory and time: a row sample
+        n = max(32, (1 << 26) // wl.width)
+        x, dy = x[:n], dy[:n]
+        z = None if z is None else z[:n]
+        fwd_b, bwd_b = bytes_model(n, wl.width, 2 if wl.dtype == "bf16" else 4, wl.gated)
+    else:
+        n = wl.rows
     reps, t0 = 0, time.perf_counter()
     while True:
         _oracle_step(oracle, x, z, w, dy, wl.eps)
@@ -403,8 +486,8 @@ def cpu_baseline(wl, fwd_b, bwd_b, min_s=10.0, max_s=30.0):
             break
     return {"value": round((fwd_b + bwd_b) * reps / el / 1e9, 4), "unit": "GB/s", "cores": 1,
             "kind": "oracle",
-            "sample": f"fp64 numpy oracle fwd+bwd over all {wl.rows} rows of the workload, "
-                      f"{reps} passes in {el:.1f} s, single thread"}
+            "sample": f"fp64 numpy oracle fwd+bwd over rows [0, {n}) of the {wl.rows}-row "
+                      f"workload, {reps} passes in {el:.1f} s, single thread"}
 
 
 def run_reference(a):
@@ -413,24 +496,27 @@ def run_reference(a):
     if rank != 0:
         return
     import oracle
-    wl = workloads.cfg_gated_heads()
+    wl = workloads.CONFIGS[a.workload]()
     R, H, eps = wl.rows, wl.width, wl.eps
     f = workloads.as_f64
+    fz = (lambda t: None) if not wl.gated else f
     # size the per-step row sample so the whole run stays near a minute of CPU
-    probe = 4096
+    probe = min(R, max(32, 4096 * 128 // H))
     t0 = time.perf_counter()
-    _oracle_step(oracle, f(wl.x[:probe]), f(wl.z[:probe]), f(wl.w), f(wl.dy[:probe]), eps)
+    _oracle_step(oracle, f(wl.x[:probe]), fz(wl.z[:probe] if wl.gated else None), f(wl.w),
+                 f(wl.dy[:probe]), eps)
     per_row = (time.perf_counter() - t0) / probe
     n = int(60.0 / per_row / max(1, a.steps + a.warmup))
     n = max(32, min(R, n // 32 * 32))
-    x, z, w, dy = f(wl.x[:n]), f(wl.z[:n]), f(wl.w), f(wl.dy[:n])
+    x, w, dy = f(wl.x[:n]), f(wl.w), f(wl.dy[:n])
+    z = f(wl.z[:n]) if wl.gated else None
     for _ in range(a.warmup):
         _oracle_step(oracle, x, z, w, dy, eps)
     t0 = time.perf_counter()
     for _ in range(a.steps):
         _oracle_step(oracle, x, z, w, dy, eps)
     el = time.perf_counter() - t0
-    fwd_b, bwd_b = bytes_model(n, H)
+    fwd_b, bwd_b = bytes_model(n, H, 2 if wl.dtype == "bf16" else 4, wl.gated)
     value = (fwd_b + bwd_b) * a.steps / el / 1e9
     sample = (f"fp64 numpy oracle fwd+bwd on rows [0, {n}) of the {R}-row workload per step "
               f"(single thread)")
@@ -440,8 +526,9 @@ def run_reference(a):
         "ms_per_step": round(1e3 * el / a.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded; no dataset or checkpoint)",
-        "config": {"workload": WORKLOAD, "op": "gated RMSNorm fwd+bwd", "rows": R, "width": H,
-                   "sample_rows_per_step": n},
+        "config": {"workload": a.workload,
+                   "op": "gated RMSNorm fwd+bwd" if wl.gated else "zero-centred RMSNorm fwd+bwd",
+                   "rows": R, "width": H, "sample_rows_per_step": n},
         "rows_per_s": round(n * a.steps / el, 1),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": sample},

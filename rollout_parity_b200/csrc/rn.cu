@@ -376,6 +376,8 @@ k_fwd(const FwdArgs a) {
   const int nv = a.nv;
   const unsigned mask = 0xffffffffu;   // the forward block is always >= 256 threads
   int phase = 0;
+  griddep_trigger();   // the next kernel may be scheduled
+  griddep_wait();      // the previous kernel's writes are complete and visible
 
   float gw[K][VE];
   load_gain<VE, K, T, GATED>(a.w, nv, t, gw);
@@ -444,7 +446,8 @@ k_bwd(const BwdArgs a) {
   const unsigned mask = blockDim.x >= 32 ? 0xffffffffu : ((1u << blockDim.x) - 1u);
   const bool have_rstd = a.rstd != nullptr;
   int phase = 0;
-  griddep_trigger();   // the dw fold may be scheduled; it waits for this grid
+  griddep_trigger();   // the next kernel (the dw fold) may be scheduled
+  griddep_wait();      // the previous kernel's writes are complete and visible
 
   float gw_r[WS ? 1 : K][WS ? 1 : VE];
   if constexpr (WS) {
@@ -631,7 +634,8 @@ k_bwd_s(const BwdArgs a) {
   const bool have_rstd = a.rstd != nullptr;
   int phase = 0;   // unused: T <= 32 reduces with shuffles only
 
-  griddep_trigger();   // the dw fold may be scheduled; it waits for this grid
+  griddep_trigger();   // the next kernel (the dw fold) may be scheduled
+  griddep_wait();      // the previous kernel's writes are complete and visible
   stage_gain<VE, K, T, GATED>(a.w, nv, gsm);
   __syncthreads();
   auto gain = [&](int k, float (&g)[VE]) { read_gain<VE, K, T>(gsm, k, t, g); };
@@ -786,6 +790,8 @@ k_fwd_s(const FwdArgs a) {
   const unsigned mask = 0xffffffffu;
   int phase = 0;   // unused: sub-warp teams reduce with shuffles only
 
+  griddep_trigger();   // the next kernel may be scheduled
+  griddep_wait();      // the previous kernel's writes are complete and visible
   stage_gain<VE, K, T, GATED>(a.w, nv, gsm);
   __syncthreads();
 
@@ -1105,6 +1111,29 @@ int blocks_per_sm(Kern kernel, int block, size_t smem) {
   return nb;
 }
 
+// Launches `kern` with programmatic stream serialization: it may be scheduled
+// while the kernel before it in the stream finishes, and waits for it
+// (griddepcontrol.wait) before touching global memory.  If the launch with
+// the attribute is refused it is retried as an ordinary launch.
+template <typename... KArgs, typename... Args>
+rn_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, args...) == cudaSuccess) return launch_status();
+  (void)cudaGetLastError();
+  kern<<<grid, block, smem, st>>>(args...);
+  return launch_status();
+}
+
 template <int DT, int T, int K, bool GATED, bool EXACT>
 rn_status launch_fwd_s(const FwdArgs& a, cudaStream_t st) {
   constexpr int NTEN = GATED ? 2 : 1;
@@ -1120,8 +1149,7 @@ rn_status launch_fwd_s(const FwdArgs& a, cudaStream_t st) {
   const int64_t nblk = (a.rows + kFwdsBlock / T - 1) / (kFwdsBlock / T);
   const int64_t wave = int64_t(nb) * sm_count();
   const int grid = grid_cap(nblk < wave ? nblk : wave);
-  k_fwd_s<DT, T, K, GATED, EXACT><<<grid, kFwdsBlock, smem, st>>>(a);
-  return launch_status();
+  return launch_pdl(k_fwd_s<DT, T, K, GATED, EXACT>, dim3(grid), dim3(kFwdsBlock), smem, st, a);
 }
 
 template <int DT, bool GATED>
@@ -1144,10 +1172,9 @@ rn_status launch_fwd(const Sched& s, const FwdArgs& a, cudaStream_t st) {
   if constexpr (T_ > 16) {                                                      \
     if (s.T == T_ && s.K == K_) {                                               \
       if (exact)                                                                \
-        k_fwd<DT, T_, K_, GATED, true><<<grid, block, 0, st>>>(a);              \
+        return launch_pdl(k_fwd<DT, T_, K_, GATED, true>, dim3(grid), dim3(block), 0, st, a);  \
       else                                                                      \
-        k_fwd<DT, T_, K_, GATED, false><<<grid, block, 0, st>>>(a);             \
-      return launch_status();                                                   \
+        return launch_pdl(k_fwd<DT, T_, K_, GATED, false>, dim3(grid), dim3(block), 0, st, a); \
     }                                                                           \
   }
   RN_TK_LIST(RN_FWD_CASE)
@@ -1165,10 +1192,9 @@ rn_status launch_bwd(const Sched& s, int lpc, const BwdArgs& a, int64_t groups, 
 #define RN_BWDS_CASE(T_, K_)                                                    \
     if (s.T == T_ && s.K == K_) {                                               \
       if (exact)                                                                \
-        k_bwd_s<DT, T_, K_, GATED, true><<<grid, block, smem, st>>>(a);         \
+        return launch_pdl(k_bwd_s<DT, T_, K_, GATED, true>, dim3(grid), dim3(block), smem, st, a); \
       else                                                                      \
-        k_bwd_s<DT, T_, K_, GATED, false><<<grid, block, smem, st>>>(a);        \
-      return launch_status();                                                   \
+        return launch_pdl(k_bwd_s<DT, T_, K_, GATED, false>, dim3(grid), dim3(block), smem, st, a); \
     }
     RN_TK_SMALL(RN_BWDS_CASE)
 #undef RN_BWDS_CASE
@@ -1178,10 +1204,9 @@ rn_status launch_bwd(const Sched& s, int lpc, const BwdArgs& a, int64_t groups, 
   if constexpr (T_ > 16) {                                                      \
     if (s.T == T_ && s.K == K_) {                                               \
       if (exact)                                                                \
-        k_bwd<DT, T_, K_, GATED, true><<<grid, block, smem, st>>>(a);           \
+        return launch_pdl(k_bwd<DT, T_, K_, GATED, true>, dim3(grid), dim3(block), smem, st, a); \
       else                                                                      \
-        k_bwd<DT, T_, K_, GATED, false><<<grid, block, smem, st>>>(a);          \
-      return launch_status();                                                   \
+        return launch_pdl(k_bwd<DT, T_, K_, GATED, false>, dim3(grid), dim3(block), smem, st, a); \
     }                                                                           \
   }
   RN_TK_LIST(RN_BWD_CASE)
@@ -1217,20 +1242,7 @@ int fold_passes(int64_t n) {
 // it is retried as an ordinary launch.
 template <int B>
 rn_status launch_fold_b(dim3 grid, cudaStream_t st, const float* in, int64_t n, int H, float* out) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(32 * kFoldRG);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, k_fold<B>, in, n, H, out) == cudaSuccess) return launch_status();
-  (void)cudaGetLastError();
-  k_fold<B><<<grid, 32 * kFoldRG, 0, st>>>(in, n, H, out);
-  return launch_status();
+  return launch_pdl(k_fold<B>, grid, dim3(32 * kFoldRG), 0, st, in, n, H, out);
 }
 
 rn_status launch_fold(int B, dim3 grid, cudaStream_t st, const float* in, int64_t n, int H,
