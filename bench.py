@@ -240,28 +240,46 @@ def run_ours(a):
     torch.cuda.synchronize()
 
     K = a.steps
+    exchange = None
+    if world > 1:
+        # data parallel: the ranks' dw are joined every step by an all-gather and
+        # the same pairwise fold, so the step's dw is that of the whole N-rank batch
+        from rollout_parity_b200 import parallel
+        parallel.check_shard_rows(R, device=dev)
+        exchange = parallel.fold_gathered_dw
+        a.no_graph = True      # NCCL calls stay outside graph capture
     G = K if a.no_graph else graph_steps(K)
-    # per-call events: the last G steps of the timed region
+    # per-call events for the roofline: G steps recorded in a separate graph (or,
+    # without graphs, every step of the timed loop)
     ev = [[torch.cuda.Event(enable_timing=True, external=not a.no_graph) for _ in range(3)]
           for _ in range(G)]
-    graph = None
+    graph = graph_ev = None
     if not a.no_graph:
-        # one CUDA graph holds G steps (calls and their event records); the
-        # timed region replays it K / G times
-        graph = torch.cuda.CUDAGraph()
+        # graph: G steps of calls only; it is what the timed region replays K / G times.
+        # graph_ev: the same G steps with event records between the calls.
         cap = torch.cuda.Stream(dev)
-        cap.wait_stream(stream)
-        with torch.cuda.graph(graph, stream=cap):
-            csp = cap.cuda_stream
-            for j in range(G):
-                ev[j][0].record(cap)
-                s1 = fwd(P[j % nsets], csp)
-                ev[j][1].record(cap)
-                s2 = bwd(P[(j + 2) % nsets], csp)
-                ev[j][2].record(cap)
-                if s1 or s2:
-                    raise RuntimeError(f"capture failed: status {s1}, {s2}")
-        stream.wait_stream(cap)
+
+        def capture(with_events):
+            g = torch.cuda.CUDAGraph()
+            cap.wait_stream(stream)
+            with torch.cuda.graph(g, stream=cap):
+                csp = cap.cuda_stream
+                for j in range(G):
+                    if with_events:
+                        ev[j][0].record(cap)
+                    s1 = fwd(P[j % nsets], csp)
+                    if with_events:
+                        ev[j][1].record(cap)
+                    s2 = bwd(P[(j + 2) % nsets], csp)
+                    if with_events:
+                        ev[j][2].record(cap)
+                    if s1 or s2:
+                        raise RuntimeError(f"capture failed: status {s1}, {s2}")
+            stream.wait_stream(cap)
+            return g
+
+        graph = capture(False)
+        graph_ev = capture(True)
         for _ in range(max(1, a.warmup // G)):
             graph.replay()
         torch.cuda.synchronize()
@@ -283,6 +301,8 @@ def run_ours(a):
             s1 = fwd(P[k % nsets])
             e[1].record(stream)
             s2 = bwd(P[(k + 2) % nsets])
+            if exchange is not None:
+                exchange(sets[(k + 2) % nsets]["dw"])
             e[2].record(stream)
             if s1 or s2:
                 check("gated_norm_fwd", s1)
@@ -294,6 +314,10 @@ def run_ours(a):
         dist.barrier()
     clk = clocks.stop()
     ms = t_start.elapsed_time(t_end)
+    if graph_ev is not None:   # per-call timings, right after the timed region
+        for _ in range(2):
+            graph_ev.replay()
+        torch.cuda.synchronize()
     fwd_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(G)]
     bwd_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(G)]
     if dist is not None:
@@ -330,9 +354,15 @@ def run_ours(a):
             "config": {"workload": a.workload, "op": opname, "rows": R, "width": H, **desc,
                        "eps": eps, "io_dtype": f"{iod} x/z/dy/y/dx/dz, fp32 w/rstd/dw",
                        "accumulate": "fp32",
-                       "bytes_per_step": step_b, "parallelism": f"replicas x{world}",
+                       "bytes_per_step": step_b,
+                       "parallelism": (f"data parallel x{world}: rows split across ranks, dw "
+                                       "all-gathered and folded each step" if world > 1
+                                       else "one GPU"),
                        "launch": ("python loop" if a.no_graph else
                                   f"CUDA graph of {G} steps replayed {K // G} times"),
+                       "per_call_timing": ("events in the timed loop" if a.no_graph else
+                                           f"events in a copy of the graph replayed after "
+                                           f"the timed region ({G} steps)"),
                        "l2": (f"{nsets} rotating buffer sets (fwd on k%{nsets}, bwd on "
                               f"(k+2)%{nsets}): every buffer is re-touched only after >= 512 MB "
                               "of other traffic (L2 is 126 MB); no flush kernel")

@@ -145,6 +145,19 @@ rn_status gated_norm_bwd(int64_t rows, int32_t width, float eps, rn_dtype dt,
                          float* dw, void* ws, size_t ws_bytes, rn_stream stream);
 
 /*
+ * Joins n rows of fp32 dw partials with the same level-by-level pairwise tree
+ * the backward uses: out[width] = tree(in[0], ..., in[n-1]), in row order.
+ * A backward call's dw is the root of that tree over its 32-row leaves, so
+ * when a batch is split across data-parallel ranks in order and every rank
+ * holds the same power-of-two number of leaves, folding the ranks' dw in rank
+ * order gives exactly (bitwise) the dw of one call over the whole batch.
+ * in: [n][width] fp32 device, read; out: [width] fp32 device, written; no
+ * workspace.  1 <= n <= 256, else RN_E_ARG; out must not overlap in.
+ */
+rn_status rn_fold_rows(int64_t n, int32_t width, const float* in, float* out,
+                       rn_stream stream);
+
+/*
  * Gated RMSNorm backward that allocates nothing: the same computation,
  * arguments and results as gated_norm_bwd, but the dw-partial scratch is a
  * fixed 8 MiB block of static device memory inside this library instead of a

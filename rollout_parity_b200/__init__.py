@@ -13,6 +13,7 @@ from .ops import (  # noqa: F401
     norm_bwd_workspace_bytes,
     norm_fwd,
     rn_describe,
+    rn_fold_rows,
     rn_test_set_geometry,
     rn_test_set_validate_only,
     workspace,

@@ -47,6 +47,7 @@ SIGNATURES = {
                                c_vp, c_vp, c_vp, c_sz, c_vp]),
     "gated_norm_bwd_static_ws": (c_i32, [c_i64, c_i32, c_f32, c_i32, c_vp, c_vp, c_vp, c_vp,
                                          c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "rn_fold_rows": (c_i32, [c_i64, c_i32, c_vp, c_vp, c_vp]),
     "rn_describe": (ctypes.c_char_p, [c_i32, c_i32]),
     "rn_bwd_launches": (c_i32, [c_i64, c_i32, c_i32]),
     "rn_status_string": (ctypes.c_char_p, [c_i32]),

@@ -87,7 +87,6 @@ struct Fmt<RN_F32> {
   }
 };
 
-__device__ __forceinline__ uint4 ld_stream(const uint4* p) { return __ldcs(p); }
 __device__ __forceinline__ void st_stream(uint4* p, const uint4& v) { __stcs(p, v); }
 
 // ---------------------------------------------------------------------------
@@ -244,24 +243,6 @@ struct BwdArgs {
   float* part;      // [groups][H] fp32 group partials (or dw when one group)
 };
 
-template <int T>
-__host__ __device__ constexpr int fwd_block() { return T <= 32 ? 256 : T; }
-template <int T, int K>
-__host__ __device__ constexpr int fwd_min_blocks() { return T <= 16 ? 3 : 1; }
-template <int T>
-__host__ __device__ constexpr int fwd_rows_per_team() { return T <= 32 ? 2 : 1; }
-template <int T>
-__host__ __device__ constexpr int bwd_max_block() { return T <= 32 ? 8 * T : (T <= 128 ? 256 : T); }
-// enough resident CTAs that one wave holds every 32-row leaf of a ~256K-row
-// batch at width 128 (1024 CTAs of 128 threads on 148 SMs)
-template <int T, int K>
-__host__ __device__ constexpr int bwd_min_blocks() {
-  return K != 1 ? 1 : (T <= 16 ? 112 / T : (T == 32 ? 3 : 1));
-}
-// sub-warp teams read w from shared memory (saves registers for occupancy)
-template <int T>
-__host__ __device__ constexpr bool bwd_w_in_smem() { return T <= 32; }
-
 // Loads this thread's gain base: w (gated) or 1 + w (zero-centred).
 template <int VE, int K, int T, bool GATED>
 __device__ __forceinline__ void load_gain(const float* __restrict__ w, int nv, int t,
@@ -277,17 +258,6 @@ __device__ __forceinline__ void load_gain(const float* __restrict__ w, int nv, i
 #pragma unroll
       for (int e = 0; e < 4; ++e) g[k][q * 4 + e] = GATED ? a[e] : __fadd_rn(1.0f, a[e]);
     }
-  }
-}
-
-// A thread's K vectors of one row; `p` points at the row's vector t.
-template <int T, int K, bool EXACT>
-__device__ __forceinline__ void load_row(uint4 (&r)[K], const uint4* __restrict__ p, int nv,
-                                         int t, bool act) {
-#pragma unroll
-  for (int k = 0; k < K; ++k) {
-    const bool ok = act && (EXACT || k * T + t < nv);
-    r[k] = ok ? ld_stream(p + k * T) : make_uint4(0, 0, 0, 0);
   }
 }
 
@@ -363,235 +333,14 @@ __device__ __forceinline__ void join_leaves(const float (&acc)[K][VE], int NT, i
   }
 }
 
-template <int DT, int T, int K, bool GATED, bool EXACT>
-__global__ void __launch_bounds__(fwd_block<T>(), fwd_min_blocks<T, K>())
-k_fwd(const FwdArgs a) {
-  using F = Fmt<DT>;
-  constexpr int VE = F::VE;
-  constexpr int U = fwd_rows_per_team<T>();
-  constexpr int NT = fwd_block<T>() / T;           // teams per CTA
-  constexpr int W = T > 32 ? T / 32 : 1;
-  __shared__ float red[T > 32 ? 2 * NT * U * W : 1];
-  const int team = threadIdx.x / T, t = threadIdx.x % T;
-  const int nv = a.nv;
-  const unsigned mask = 0xffffffffu;   // the forward block is always >= 256 threads
-  int phase = 0;
-  griddep_trigger();   // the next kernel may be scheduled
-  griddep_wait();      // the previous kernel's writes are complete and visible
-
-  float gw[K][VE];
-  load_gain<VE, K, T, GATED>(a.w, nv, t, gw);
-
-  const int64_t step = int64_t(gridDim.x) * NT * U;
-  for (int64_t base = int64_t(blockIdx.x) * NT * U; base < a.rows; base += step) {
-    uint4 xr[U][K], zr[U][K];
-    bool act[U];
-    int64_t off[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t row = base + int64_t(u) * NT + team;
-      act[u] = row < a.rows;
-      off[u] = row * nv + t;
-      load_row<T, K, EXACT>(xr[u], a.x + off[u], nv, t, act[u]);
-      if constexpr (GATED) load_row<T, K, EXACT>(zr[u], a.z + off[u], nv, t, act[u]);
-    }
-    float ss[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) ss[u] = thread_sumsq<DT, T, K, EXACT>(xr[u], nv, t);
-    team_sum<T, U>(ss, red, phase, team, NT, mask);
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const float r = rsqrtf(__fadd_rn(mean_of(ss[u], a.H, a.inv_h, a.h_pow2), a.eps));
-#pragma unroll
-      for (int k = 0; k < K; ++k) {
-        if (act[u] && (EXACT || k * T + t < nv)) {
-          float f[VE], yv[VE];
-          F::unpack(xr[u][k], f);
-          if constexpr (GATED) {
-            float zf[VE];
-            F::unpack(zr[u][k], zf);
-#pragma unroll
-            for (int e = 0; e < VE; ++e) {
-              const float act_z = __fmul_rn(zf[e], sigmoid_f(zf[e]));
-              yv[e] = __fmul_rn(__fmul_rn(__fmul_rn(f[e], r), gw[k][e]), act_z);
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < VE; ++e) yv[e] = __fmul_rn(__fmul_rn(f[e], r), gw[k][e]);
-          }
-          st_stream(a.y + off[u] + k * T, F::pack(yv));
-        }
-      }
-      if (act[u] && t == 0 && a.rstd != nullptr) a.rstd[base + int64_t(u) * NT + team] = r;
-    }
-  }
-}
-
-template <int DT, int T, int K, bool GATED, bool EXACT>
-__global__ void __launch_bounds__(bwd_max_block<T>(), bwd_min_blocks<T, K>())
-k_bwd(const BwdArgs a) {
-  using F = Fmt<DT>;
-  constexpr int VE = F::VE;
-  constexpr int W = T > 32 ? T / 32 : 1;
-  constexpr bool WS = bwd_w_in_smem<T>();
-  // dynamic shared memory: [H] gain (WS), [2][NT][W] reduction scratch (T > 32),
-  // then [NT][H] leaf partials (NT > 1)
-  extern __shared__ float dsm[];
-  const int NT = blockDim.x / T;   // leaves per CTA (power of two)
-  float* gsm = dsm;
-  float* red = dsm + (WS ? a.H : 0);
-  float* leafbuf = red + (T > 32 ? 2 * NT * W : 0);
-  const int team = threadIdx.x / T, t = threadIdx.x % T;
-  const int nv = a.nv;
-  const unsigned mask = blockDim.x >= 32 ? 0xffffffffu : ((1u << blockDim.x) - 1u);
-  const bool have_rstd = a.rstd != nullptr;
-  int phase = 0;
-  griddep_trigger();   // the next kernel (the dw fold) may be scheduled
-  griddep_wait();      // the previous kernel's writes are complete and visible
-
-  float gw_r[WS ? 1 : K][WS ? 1 : VE];
-  if constexpr (WS) {
-    for (int c = threadIdx.x; c < a.H; c += blockDim.x)
-      gsm[c] = GATED ? __ldg(a.w + c) : __fadd_rn(1.0f, __ldg(a.w + c));
-    __syncthreads();
-  } else {
-    load_gain<VE, K, T, GATED>(a.w, nv, t, gw_r);
-  }
-  // this thread's gain for vector k: from registers, or from shared memory
-  auto gain = [&](int k, float (&g)[VE]) {
-    if constexpr (WS) {
-      const float4* p = reinterpret_cast<const float4*>(gsm) + (k * T + t) * (VE / 4);
-#pragma unroll
-      for (int q = 0; q < VE / 4; ++q) {
-        const float4 f = p[q];
-        g[4 * q] = f.x; g[4 * q + 1] = f.y; g[4 * q + 2] = f.z; g[4 * q + 3] = f.w;
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < VE; ++e) g[e] = gw_r[WS ? 0 : k][WS ? 0 : e];
-    }
-  };
-
-  // one row: fetch (issued a row ahead of its use)
-  auto fetch = [&](int64_t row, bool act, uint4 (&x)[K], uint4 (&z)[K], uint4 (&d)[K],
-                   float& r) {
-    const int64_t off = row * nv + t;
-    load_row<T, K, EXACT>(x, a.x + off, nv, t, act);
-    load_row<T, K, EXACT>(d, a.dy + off, nv, t, act);
-    if constexpr (GATED) load_row<T, K, EXACT>(z, a.z + off, nv, t, act);
-    r = (act && have_rstd) ? __ldcs(a.rstd + row) : 0.0f;
-  };
-
-  float acc[K][VE];
-
-  // one row: dot, dx, dz, and the leaf's dw fold (called in ascending row order)
-  auto process = [&](int64_t row, bool act, const uint4 (&x)[K], const uint4 (&z)[K],
-                     const uint4 (&d)[K], float rs) {
-    if (!have_rstd) {   // uniform branch: recompute exactly as the forward does
-      float ss[1] = {thread_sumsq<DT, T, K, EXACT>(x, nv, t)};
-      team_sum<T, 1>(ss, red, phase, team, NT, mask);
-      rs = rsqrtf(__fadd_rn(mean_of(ss[0], a.H, a.inv_h, a.h_pow2), a.eps));
-    }
-    // pass 1: dot = sum_j (g_j * dy_j) * xh_j, xh = x*rstd, g = 1+w or w*silu(z)
-    float sg[K][GATED ? VE : 1];
-    float dp[K];   // per-vector dot partials, joined by the pairwise tree
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      dp[k] = -0.0f;
-      float xf[VE], df[VE], zf[VE], gk[VE];
-      F::unpack(x[k], xf);
-      F::unpack(d[k], df);
-      if constexpr (GATED) F::unpack(z[k], zf);
-      gain(k, gk);
-#pragma unroll
-      for (int e = 0; e < VE; ++e) {
-        const float xh = __fmul_rn(xf[e], rs);
-        float g;
-        if constexpr (GATED) {
-          sg[k][e] = sigmoid_f(zf[e]);
-          g = __fmul_rn(gk[e], __fmul_rn(zf[e], sg[k][e]));      // w * silu(z)
-        } else {
-          g = gk[e];                                             // 1 + w
-        }
-        if (EXACT || k * T + t < nv) dp[k] = __fmaf_rn(__fmul_rn(g, df[e]), xh, dp[k]);
-      }
-    }
-    float dot[1] = {pairwise_tree<K>(dp)};
-    team_sum<T, 1>(dot, red, phase, team, NT, mask);
-    const float m = mean_of(dot[0], a.H, a.inv_h, a.h_pow2);
-    // pass 2
-    const int64_t off = row * nv + t;
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      if (act && (EXACT || k * T + t < nv)) {
-        float xf[VE], df[VE], zf[VE], dxv[VE], dzv[VE], gk[VE];
-        F::unpack(x[k], xf);
-        F::unpack(d[k], df);
-        if constexpr (GATED) F::unpack(z[k], zf);
-        gain(k, gk);
-#pragma unroll
-        for (int e = 0; e < VE; ++e) {
-          const float xh = __fmul_rn(xf[e], rs);                  // same bits as pass 1
-          const float q = __fmul_rn(df[e], xh);                   // dy * xh
-          if constexpr (GATED) {
-            const float s = sg[k][e];
-            const float silu = __fmul_rn(zf[e], s);
-            const float gd = __fmul_rn(__fmul_rn(gk[e], silu), df[e]);
-            dxv[e] = __fmul_rn(rs, __fmaf_rn(-xh, m, gd));       // rstd*(g*dy - xh*m)
-            const float d1 = __fmaf_rn(zf[e], __fsub_rn(1.0f, s), 1.0f);
-            dzv[e] = __fmul_rn(__fmul_rn(__fmul_rn(q, gk[e]), s), d1);
-            acc[k][e] = __fadd_rn(acc[k][e], __fmul_rn(q, silu));
-          } else {
-            const float gd = __fmul_rn(gk[e], df[e]);
-            dxv[e] = __fmul_rn(rs, __fmaf_rn(-xh, m, gd));
-            acc[k][e] = __fadd_rn(acc[k][e], q);
-          }
-        }
-        st_stream(a.dx + off + k * T, F::pack(dxv));
-        if constexpr (GATED) st_stream(a.dz + off + k * T, F::pack(dzv));
-      }
-    }
-  };
-
-  const int64_t n_leaves = (a.rows + kLeafRows - 1) / kLeafRows;
-  const int64_t n_groups = (n_leaves + NT - 1) / NT;
-  for (int64_t grp = blockIdx.x; grp < n_groups; grp += gridDim.x) {
-    const int64_t r0 = (grp * NT + team) * kLeafRows;
-#pragma unroll
-    for (int k = 0; k < K; ++k)
-#pragma unroll
-      for (int e = 0; e < VE; ++e) acc[k][e] = -0.0f;
-
-    uint4 ax[K], az[K], ad[K], bx[K], bz[K], bd[K];
-    float ar, br;
-    fetch(r0, r0 < a.rows, ax, az, ad, ar);
-    for (int i = 0; i < kLeafRows; i += 2) {
-      const int64_t row = r0 + i;
-      fetch(row + 1, row + 1 < a.rows, bx, bz, bd, br);
-      process(row, row < a.rows, ax, az, ad, ar);
-      fetch(row + 2, i + 2 < kLeafRows && row + 2 < a.rows, ax, az, ad, ar);
-      process(row + 1, row + 1 < a.rows, bx, bz, bd, br);
-    }
-
-    // join the CTA's leaves (aligned power-of-two group) with the pairwise tree
-    const int64_t rem = n_leaves - grp * NT;
-    join_leaves<VE, K, T, EXACT>(acc, NT, rem < NT ? int(rem) : NT, team, t, nv, a.H, leafbuf,
-                                 a.part + grp * a.H);
-  }
-}
-
 // ---------------------------------------------------------------------------
-// Backward for sub-warp teams (T <= 8, K <= 4: widths up to 256 bf16 / 128
-// fp32).  Same arithmetic and order as k_bwd; the difference is the data
-// path: each thread stages its own x, dy (z) vectors and rstd through shared
-// memory with cp.async, kBwdStages - 1 rows ahead of the row it computes, so
-// no registers hold prefetched rows and pass 2 keeps xh, g*dy and s from
-// pass 1 instead of recomputing them.  Every thread reads back only what it
-// copied itself (cp.async.wait_group makes its own copies visible to it), so
-// the pipeline needs no barrier.
+// Data path of both kernels: every thread stages its own 16-byte vectors of a
+// row (and the row's rstd) into shared memory with cp.async, S-1 rows ahead of
+// the row it computes, and reads back only what it copied itself
+// (cp.async.wait_group makes a thread's own copies visible to it), so the
+// pipeline needs no barrier; multi-warp teams (T > 32) meet at one
+// __syncthreads per row reduction, all teams of a CTA in lockstep.
 // ---------------------------------------------------------------------------
-constexpr int kBwdStages = 3;
-
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa), "l"(gmem) : "memory");
@@ -606,39 +355,211 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// enough resident CTAs for one wave of 1024 (262144 rows of 128: 8192 leaves,
-// 8 per CTA) on 148 SMs, within the register file
+// Where a thread's gain (w or 1 + w) comes from: shared memory (thread-major)
+// for sub-warp teams, registers when K*VE <= 16, else global memory (L1).
+enum GainSrc { kGainSmem = 0, kGainRegs = 1, kGainGlobal = 2 };
+template <int T, int K, int VE>
+__host__ __device__ constexpr int gain_src() {
+  return T <= 16 ? kGainSmem : (K * VE <= 16 ? kGainRegs : kGainGlobal);
+}
+
+template <int VE, int K, int T, bool GATED, int SRC>
+struct Gain {
+  float r[SRC == kGainRegs ? K : 1][SRC == kGainRegs ? VE : 1];
+  const float* smem;
+  const float* w;
+  int nv, t;
+  // must be called by every thread of the CTA (it may stage into shared memory)
+  __device__ __forceinline__ void init(const float* __restrict__ w_, int nv_, int t_, float* gsm) {
+    w = w_; nv = nv_; t = t_; smem = gsm;
+    if constexpr (SRC == kGainRegs) load_gain<VE, K, T, GATED>(w_, nv_, t_, r);
+    if constexpr (SRC == kGainSmem) {
+      stage_gain<VE, K, T, GATED>(w_, nv_, gsm);
+      __syncthreads();
+    }
+  }
+  __device__ __forceinline__ void get(int k, float (&g)[VE]) const {
+    if constexpr (SRC == kGainRegs) {
+#pragma unroll
+      for (int e = 0; e < VE; ++e) g[e] = r[SRC == kGainRegs ? k : 0][SRC == kGainRegs ? e : 0];
+    } else if constexpr (SRC == kGainSmem) {
+      read_gain<VE, K, T>(smem, k, t, g);
+    } else {
+      const int v = k * T + t;
+#pragma unroll
+      for (int q = 0; q < VE / 4; ++q) {
+        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (v < nv) f = __ldg(reinterpret_cast<const float4*>(w) + v * (VE / 4) + q);
+        const float a[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) g[q * 4 + e] = GATED ? a[e] : __fadd_rn(1.0f, a[e]);
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Forward: persistent.  The grid is one wave of CTAs; team j of CTA c walks
+// rows (c + i*grid)*NT + j.  Per row: sum of squares, the team reduction,
+// rstd, the epilogue, y and rstd stores.
+// ---------------------------------------------------------------------------
 template <int T, int K>
-__host__ __device__ constexpr int bwds_min_blocks() { return T <= 4 ? 7 : (K <= 2 ? 7 : 4); }
+__host__ __device__ constexpr int fwd_block() {
+  return T <= 16 ? (K <= 2 ? 128 : 64) : (T == 32 ? 128 : T);
+}
+template <int T, int K>
+__host__ __device__ constexpr int fwd_min_blocks() { return T <= 16 ? (K <= 2 ? 4 : 8) : 1; }
+template <int T>
+__host__ __device__ constexpr int fwd_stages() { return T <= 32 ? 3 : (T <= 512 ? 2 : 1); }
 
 template <int DT, int T, int K, bool GATED, bool EXACT>
-__global__ void __launch_bounds__(8 * T, bwds_min_blocks<T, K>())
-k_bwd_s(const BwdArgs a) {
+__global__ void __launch_bounds__(fwd_block<T, K>(), fwd_min_blocks<T, K>())
+k_fwd(const FwdArgs a) {
   using F = Fmt<DT>;
   constexpr int VE = F::VE;
-  constexpr int S = kBwdStages;
+  constexpr int S = fwd_stages<T>();
+  constexpr int NTEN = GATED ? 2 : 1;   // staged tensors: x (, z)
+  constexpr int B = fwd_block<T, K>();
+  constexpr int NT = B / T;
+  constexpr int W = T > 32 ? T / 32 : 1;
+  constexpr int GS = gain_src<T, K, VE>();
+  // dynamic shared memory: reduction scratch [2][NT][W] (T > 32) |
+  // gain [K*T*VE] (sub-warp teams) | stages [S][NTEN][K][B] uint4
+  extern __shared__ float dsm[];
+  float* red = dsm;
+  float* gsm = red + (T > 32 ? 2 * NT * W : 0);
+  uint4* stg = reinterpret_cast<uint4*>(gsm + (GS == kGainSmem ? K * T * VE : 0));
+  const int tid = threadIdx.x, team = tid / T, t = tid % T;
+  const int nv = a.nv;
+  const unsigned mask = 0xffffffffu;   // blocks are whole warps
+  int phase = 0;
+
+  griddep_trigger();   // the next kernel may be scheduled
+  griddep_wait();      // the previous kernel's writes are complete and visible
+  Gain<VE, K, T, GATED, GS> gain;
+  gain.init(a.w, nv, t, gsm);
+
+  auto slot = [&](int sl, int ten, int k) -> uint4* {
+    return stg + ((sl * NTEN + ten) * K + k) * B + tid;
+  };
+  const int64_t nblk = (a.rows + NT - 1) / NT;
+  const int64_t iters = nblk > blockIdx.x ? (nblk - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  auto row_of = [&](int64_t i) { return (int64_t(blockIdx.x) + i * gridDim.x) * NT + team; };
+  auto issue = [&](int64_t i, int sl) {
+    if (i < iters) {
+      const int64_t row = row_of(i);
+      if (row < a.rows) {
+        const int64_t off = row * nv + t;
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+          if (EXACT || k * T + t < nv) {
+            cp_async16(slot(sl, 0, k), a.x + off + k * T);
+            if constexpr (GATED) cp_async16(slot(sl, 1, k), a.z + off + k * T);
+          }
+        }
+      }
+    }
+    cp_async_commit();
+  };
+
+#pragma unroll
+  for (int i = 0; i < S - 1; ++i) issue(i, i);
+  int sl = 0;
+  for (int64_t i = 0; i < iters; ++i) {
+    {
+      int sa = sl + S - 1;
+      if (sa >= S) sa -= S;
+      issue(i + S - 1, sa);
+    }
+    cp_async_wait<S - 1>();
+    uint4 xr[K], zr[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      xr[k] = *slot(sl, 0, k);
+      if constexpr (GATED) zr[k] = *slot(sl, 1, k);
+    }
+    const int64_t row = row_of(i);
+    const bool act = row < a.rows;
+    float ss[1] = {thread_sumsq<DT, T, K, EXACT>(xr, nv, t)};
+    team_sum<T, 1>(ss, red, phase, team, NT, mask);
+    const float r = rsqrtf(__fadd_rn(mean_of(ss[0], a.H, a.inv_h, a.h_pow2), a.eps));
+    const int64_t off = row * nv + t;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      if (act && (EXACT || k * T + t < nv)) {
+        float f[VE], yv[VE], gk[VE];
+        F::unpack(xr[k], f);
+        gain.get(k, gk);
+        if constexpr (GATED) {
+          float zf[VE];
+          F::unpack(zr[k], zf);
+#pragma unroll
+          for (int e = 0; e < VE; ++e) {
+            const float act_z = __fmul_rn(zf[e], sigmoid_f(zf[e]));
+            yv[e] = __fmul_rn(__fmul_rn(__fmul_rn(f[e], r), gk[e]), act_z);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < VE; ++e) yv[e] = __fmul_rn(__fmul_rn(f[e], r), gk[e]);
+        }
+        st_stream(a.y + off + k * T, F::pack(yv));
+      }
+    }
+    if (act && t == 0 && a.rstd != nullptr) a.rstd[row] = r;
+    if (++sl == S) sl = 0;
+  }
+  cp_async_wait<0>();
+}
+
+// ---------------------------------------------------------------------------
+// Backward: one team per 32-row leaf, rows in ascending order.  x, dy (z) and
+// rstd are staged S-1 rows ahead; pass 1 keeps xh, g*dy and s in registers for
+// pass 2 (dx, dz stores and the leaf's dw fold).  The CTA's leaves (an aligned
+// power-of-two group) are joined by the pairwise tree; one partial per CTA.
+// ---------------------------------------------------------------------------
+template <int T>
+__host__ __device__ constexpr int bwd_max_block() { return T <= 32 ? 8 * T : (T <= 128 ? 256 : T); }
+// at width 128 (T = 4): enough resident CTAs for one wave of 1024 (262144 rows:
+// 8192 leaves, 8 per CTA) on 148 SMs, within the register file; at width 2048
+// (T = 128, two leaves per 256-thread CTA) two CTAs per SM
+template <int T, int K>
+__host__ __device__ constexpr int bwd_min_blocks() {
+  return T <= 4 ? 7 : (T == 8 ? (K <= 2 ? 7 : 4) : ((T == 32 || T == 128) && K <= 2 ? 2 : 1));
+}
+template <int T>
+__host__ __device__ constexpr int bwd_stages() { return T <= 16 ? 3 : (T <= 512 ? 2 : 1); }
+
+template <int DT, int T, int K, bool GATED, bool EXACT>
+__global__ void __launch_bounds__(bwd_max_block<T>(), bwd_min_blocks<T, K>())
+k_bwd(const BwdArgs a) {
+  using F = Fmt<DT>;
+  constexpr int VE = F::VE;
+  constexpr int S = bwd_stages<T>();
   constexpr int NTEN = GATED ? 3 : 2;   // staged tensors: x, dy (, z)
-  // dynamic shared memory: gain [K*T*VE] | stages [S][NTEN][K][blockDim] uint4 |
-  // leaf partials [NT][H] | rstd stages [S][blockDim]
+  constexpr int W = T > 32 ? T / 32 : 1;
+  constexpr int GS = gain_src<T, K, VE>();
+  // dynamic shared memory: reduction scratch [2][NT][W] (T > 32) |
+  // gain [K*T*VE] (sub-warp teams) | stages [S][NTEN][K][blockDim] uint4 |
+  // leaf partials [NT][H] (NT > 1) | rstd stages [S][blockDim]
   extern __shared__ float dsm[];
   const int bd = blockDim.x;
   const int NT = bd / T;
   const int tid = threadIdx.x;
-  float* gsm = dsm;
-  uint4* stg = reinterpret_cast<uint4*>(dsm + K * T * VE);
+  float* red = dsm;
+  float* gsm = red + (T > 32 ? 2 * NT * W : 0);
+  uint4* stg = reinterpret_cast<uint4*>(gsm + (GS == kGainSmem ? K * T * VE : 0));
   float* leafbuf = reinterpret_cast<float*>(stg + S * NTEN * K * bd);
   float* rsm = leafbuf + (NT > 1 ? NT * a.H : 0);
   const int team = tid / T, t = tid % T;
   const int nv = a.nv;
   const unsigned mask = bd >= 32 ? 0xffffffffu : ((1u << bd) - 1u);
   const bool have_rstd = a.rstd != nullptr;
-  int phase = 0;   // unused: T <= 32 reduces with shuffles only
+  int phase = 0;
 
   griddep_trigger();   // the next kernel (the dw fold) may be scheduled
   griddep_wait();      // the previous kernel's writes are complete and visible
-  stage_gain<VE, K, T, GATED>(a.w, nv, gsm);
-  __syncthreads();
-  auto gain = [&](int k, float (&g)[VE]) { read_gain<VE, K, T>(gsm, k, t, g); };
+  Gain<VE, K, T, GATED, GS> gain;
+  gain.init(a.w, nv, t, gsm);
   auto slot = [&](int sl, int ten, int k) -> uint4* { return stg + ((sl * NTEN + ten) * K + k) * bd + tid; };
 
   // stage row `row` (if act) into slot sl, then close the copy group
@@ -693,7 +614,7 @@ k_bwd_s(const BwdArgs a) {
         rs = rsm[sl * bd + tid];
       } else {   // uniform branch: recompute exactly as the forward does
         float ss[1] = {thread_sumsq<DT, T, K, EXACT>(xr, nv, t)};
-        team_sum<T, 1>(ss, nullptr, phase, team, NT, mask);
+        team_sum<T, 1>(ss, red, phase, team, NT, mask);
         rs = rsqrtf(__fadd_rn(mean_of(ss[0], a.H, a.inv_h, a.h_pow2), a.eps));
       }
       // pass 1: keep xh, g*dy and s for pass 2
@@ -706,7 +627,7 @@ k_bwd_s(const BwdArgs a) {
         F::unpack(xr[k], xf);
         F::unpack(dr[k], df);
         if constexpr (GATED) F::unpack(zr[k], zf);
-        gain(k, gk);
+        gain.get(k, gk);
 #pragma unroll
         for (int e = 0; e < VE; ++e) {
           xh[k][e] = __fmul_rn(xf[e], rs);
@@ -722,7 +643,7 @@ k_bwd_s(const BwdArgs a) {
         }
       }
       float dot[1] = {pairwise_tree<K>(dp)};
-      team_sum<T, 1>(dot, nullptr, phase, team, NT, mask);
+      team_sum<T, 1>(dot, red, phase, team, NT, mask);
       const float m = mean_of(dot[0], a.H, a.inv_h, a.h_pow2);
       // pass 2: dx, dz, and the leaf's dw fold (rows in ascending order)
       const int64_t off = row * nv + t;
@@ -733,7 +654,7 @@ k_bwd_s(const BwdArgs a) {
           F::unpack(dr[k], df);
           if constexpr (GATED) {
             F::unpack(zr[k], zf);
-            gain(k, gk);
+            gain.get(k, gk);
           }
 #pragma unroll
           for (int e = 0; e < VE; ++e) {
@@ -760,111 +681,6 @@ k_bwd_s(const BwdArgs a) {
     join_leaves<VE, K, T, EXACT>(acc, NT, rem < NT ? int(rem) : NT, team, t, nv, a.H, leafbuf,
                                  a.part + grp * a.H);
   }
-}
-
-// ---------------------------------------------------------------------------
-// Forward for sub-warp teams (T <= 8), persistent: the grid is one wave of
-// CTAs and each team walks rows (blockIdx.x + i*gridDim.x)*NT + team, staging
-// x (and z) through shared memory with cp.async kFwdStages - 1 rows ahead.
-// Per row the arithmetic is k_fwd's, in the same order.
-// ---------------------------------------------------------------------------
-constexpr int kFwdStages = 3;
-template <int K>
-__host__ __device__ constexpr int fwds_block() { return K <= 2 ? 128 : 64; }
-
-template <int DT, int T, int K, bool GATED, bool EXACT>
-__global__ void __launch_bounds__(fwds_block<K>(), K <= 2 ? 4 : 8)
-k_fwd_s(const FwdArgs a) {
-  constexpr int kFwdsBlock = fwds_block<K>();
-  using F = Fmt<DT>;
-  constexpr int VE = F::VE;
-  constexpr int S = kFwdStages;
-  constexpr int NTEN = GATED ? 2 : 1;   // staged tensors: x (, z)
-  constexpr int NT = kFwdsBlock / T;
-  // dynamic shared memory: gain [K*T*VE] (thread-major) | stages [S][NTEN][K][block] uint4
-  extern __shared__ float dsm[];
-  float* gsm = dsm;
-  uint4* stg = reinterpret_cast<uint4*>(dsm + K * T * VE);
-  const int tid = threadIdx.x, team = tid / T, t = tid % T;
-  const int nv = a.nv;
-  const unsigned mask = 0xffffffffu;
-  int phase = 0;   // unused: sub-warp teams reduce with shuffles only
-
-  griddep_trigger();   // the next kernel may be scheduled
-  griddep_wait();      // the previous kernel's writes are complete and visible
-  stage_gain<VE, K, T, GATED>(a.w, nv, gsm);
-  __syncthreads();
-
-  auto slot = [&](int sl, int ten, int k) -> uint4* {
-    return stg + ((sl * NTEN + ten) * K + k) * kFwdsBlock + tid;
-  };
-  const int64_t nblk = (a.rows + NT - 1) / NT;
-  const int64_t iters = nblk > blockIdx.x ? (nblk - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
-  auto row_of = [&](int64_t i) { return (int64_t(blockIdx.x) + i * gridDim.x) * NT + team; };
-  auto issue = [&](int64_t i, int sl) {
-    if (i < iters) {
-      const int64_t row = row_of(i);
-      if (row < a.rows) {
-        const int64_t off = row * nv + t;
-#pragma unroll
-        for (int k = 0; k < K; ++k) {
-          if (EXACT || k * T + t < nv) {
-            cp_async16(slot(sl, 0, k), a.x + off + k * T);
-            if constexpr (GATED) cp_async16(slot(sl, 1, k), a.z + off + k * T);
-          }
-        }
-      }
-    }
-    cp_async_commit();
-  };
-
-#pragma unroll
-  for (int i = 0; i < S - 1; ++i) issue(i, i);
-  int sl = 0;
-  for (int64_t i = 0; i < iters; ++i) {
-    {
-      int sa = sl + S - 1;
-      if (sa >= S) sa -= S;
-      issue(i + S - 1, sa);
-    }
-    cp_async_wait<S - 1>();
-    uint4 xr[K], zr[K];
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      xr[k] = *slot(sl, 0, k);
-      if constexpr (GATED) zr[k] = *slot(sl, 1, k);
-    }
-    const int64_t row = row_of(i);
-    const bool act = row < a.rows;
-    float ss[1] = {thread_sumsq<DT, T, K, EXACT>(xr, nv, t)};
-    team_sum<T, 1>(ss, nullptr, phase, team, NT, mask);
-    const float r = rsqrtf(__fadd_rn(mean_of(ss[0], a.H, a.inv_h, a.h_pow2), a.eps));
-    const int64_t off = row * nv + t;
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      if (act && (EXACT || k * T + t < nv)) {
-        float f[VE], yv[VE], gk[VE];
-        F::unpack(xr[k], f);
-        read_gain<VE, K, T>(gsm, k, t, gk);
-        if constexpr (GATED) {
-          float zf[VE];
-          F::unpack(zr[k], zf);
-#pragma unroll
-          for (int e = 0; e < VE; ++e) {
-            const float act_z = __fmul_rn(zf[e], sigmoid_f(zf[e]));
-            yv[e] = __fmul_rn(__fmul_rn(__fmul_rn(f[e], r), gk[e]), act_z);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < VE; ++e) yv[e] = __fmul_rn(__fmul_rn(f[e], r), gk[e]);
-        }
-        st_stream(a.y + off + k * T, F::pack(yv));
-      }
-    }
-    if (act && t == 0 && a.rstd != nullptr) a.rstd[row] = r;
-    if (++sl == S) sl = 0;
-  }
-  cp_async_wait<0>();
 }
 
 // One fold pass: out[b] = pairwise tree of in[b*S, min(n, (b+1)*S)), S = kFoldRG * B.
@@ -982,39 +798,51 @@ bool pick_sched(int32_t width, rn_dtype dt, Sched* s) {
   return true;
 }
 
+// host copies of the kernels' launch shapes (the same formulas)
 int bwd_max_block_rt(int T) { return T <= 32 ? 8 * T : (T <= 128 ? 256 : T); }
-int fwd_block_rt(int T) { return T <= 32 ? 256 : T; }
-int fwd_rows_per_cta_rt(int T) { return T <= 32 ? (256 / T) * 2 : 1; }
+int fwd_block_rt(int T, int K) { return T <= 16 ? (K <= 2 ? 128 : 64) : (T == 32 ? 128 : T); }
+int fwd_stages_rt(int T) { return T <= 32 ? 3 : (T <= 512 ? 2 : 1); }
+int bwd_stages_rt(int T) { return T <= 16 ? 3 : (T <= 512 ? 2 : 1); }
+constexpr size_t kSmemCap = 96 * 1024;   // leaves per CTA shrink until the backward fits
 
 std::atomic<int> g_max_ctas{0}, g_leaves_per_cta{0}, g_fold_rows{0}, g_validate_only{0};
 thread_local int t_last_cuda = 0;
 thread_local char t_describe[512];
 
 
-bool bwd_pipelined(const Sched& s) { return s.T <= 16; }
-
-size_t bwd_smem_bytes(const Sched& s, int lpc, int width, bool gated) {
+// Dynamic shared memory of k_bwd: reduction scratch, sub-warp gain, staged
+// rows, leaf partials, staged rstd (the kernel's layout).
+size_t bwd_smem_bytes(const Sched& s, int lpc, int width, bool gated, rn_dtype dt) {
+  const size_t VE = dt == RN_BF16 ? 8 : 4;
+  const size_t bd = size_t(lpc) * s.T;
+  const size_t W = s.T > 32 ? s.T / 32 : 1;
+  const size_t red = s.T > 32 ? 2 * size_t(lpc) * W * sizeof(float) : 0;
+  const size_t gain = s.T <= 16 ? size_t(s.K) * s.T * VE * sizeof(float) : 0;
+  const size_t stages = size_t(bwd_stages_rt(s.T)) * (gated ? 3 : 2) * s.K * bd * 16;
   const size_t leaves = lpc > 1 ? size_t(lpc) * width * sizeof(float) : 0;
-  if (bwd_pipelined(s)) {   // k_bwd_s: gain, staged rows, leaf partials, staged rstd
-    const size_t bd = size_t(lpc) * s.T;
-    // gain: K*T*VE floats (VE <= 8)
-    return size_t(s.K) * s.T * 8 * sizeof(float) + size_t(kBwdStages) * (gated ? 3 : 2) * s.K * bd * 16 +
-           leaves + size_t(kBwdStages) * bd * sizeof(float);
-  }
-  const int W = s.T > 32 ? s.T / 32 : 1;
-  size_t f = (s.T <= 32 ? size_t(width) : 0) + (s.T > 32 ? size_t(2) * lpc * W : 0);
-  return f * sizeof(float) + leaves;
+  return red + gain + stages + leaves + size_t(bwd_stages_rt(s.T)) * bd * sizeof(float);
 }
 
-// (sized for the gated op's staging, so both ops use the same geometry)
-int leaves_per_cta(const Sched& s, int width) {
+// Dynamic shared memory of k_fwd (the kernel's layout).
+size_t fwd_smem_bytes(const Sched& s, bool gated, rn_dtype dt) {
+  const size_t VE = dt == RN_BF16 ? 8 : 4;
+  const size_t B = fwd_block_rt(s.T, s.K), NT = B / s.T;
+  const size_t W = s.T > 32 ? s.T / 32 : 1;
+  const size_t red = s.T > 32 ? 2 * NT * W * sizeof(float) : 0;
+  const size_t gain = s.T <= 16 ? size_t(s.K) * s.T * VE * sizeof(float) : 0;
+  return red + gain + size_t(fwd_stages_rt(s.T)) * (gated ? 2 : 1) * s.K * B * 16;
+}
+
+// Leaves one backward CTA folds (a power of two); sized for the gated op's
+// staging so that both ops use the same geometry.
+int leaves_per_cta(const Sched& s, int width, rn_dtype dt) {
   const int maxb = bwd_max_block_rt(s.T);
   int lpc = maxb / s.T;                                   // default: fill the block
-  if (s.T > 32 && width > 2048) lpc = 1;                  // keep leaf staging <= 16 KB
+  if (s.T > 32 && width > 2048) lpc = 1;
   const int req = g_leaves_per_cta.load();
   if (req > 0) lpc = req < lpc ? req : lpc;
   if (lpc > 8) lpc = 8;
-  while (lpc > 1 && bwd_smem_bytes(s, lpc, width, true) > 48 * 1024) lpc /= 2;
+  while (lpc > 1 && bwd_smem_bytes(s, lpc, width, true, dt) > kSmemCap) lpc /= 2;
   return lpc;
 }
 
@@ -1077,12 +905,10 @@ rn_status launch_status() {
 }
 
 // ---- dispatch over the (T, K) pairs pick_sched can return -----------------
-#define RN_TK_LIST(X) \
-  X(32, 2) X(32, 3) X(32, 4) X(128, 2) X(128, 3) X(128, 4) X(512, 2) X(512, 3) X(512, 4) \
+#define RN_TK_LIST(X)                                                                          \
+  X(1, 1) X(1, 2) X(1, 3) X(1, 4) X(2, 3) X(2, 4) X(4, 3) X(4, 4) X(8, 3) X(8, 4)              \
+  X(32, 2) X(32, 3) X(32, 4) X(128, 2) X(128, 3) X(128, 4) X(512, 2) X(512, 3) X(512, 4)      \
   X(1024, 3) X(1024, 4)
-// the sub-warp teams, which use the pipelined kernels k_fwd_s and k_bwd_s
-#define RN_TK_SMALL(X) \
-  X(1, 1) X(1, 2) X(1, 3) X(1, 4) X(2, 3) X(2, 4) X(4, 3) X(4, 4) X(8, 3) X(8, 4)
 
 int sm_count() {
   static std::atomic<int> cached[64];
@@ -1099,16 +925,25 @@ int sm_count() {
   return n;
 }
 
-// Resident CTAs per SM of a kernel (cached per instantiation and smem size).
+// Lets `kernel` use `smem` bytes of dynamic shared memory (the default limit is
+// 48 KB) and returns how many of its CTAs fit on one SM.  `done` and `per_sm`
+// cache the answer of the first call for this kernel and size class.
 template <typename Kern>
-int blocks_per_sm(Kern kernel, int block, size_t smem) {
-  int nb = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, block, smem) != cudaSuccess ||
-      nb <= 0) {
-    (void)cudaGetLastError();
-    nb = 1;
+int prepare_kernel(Kern kernel, int block, size_t smem, std::atomic<size_t>& done,
+                   std::atomic<int>& per_sm) {
+  if (smem > done.load()) {
+    if (smem > 48 * 1024)
+      (void)cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, block, smem) != cudaSuccess ||
+        nb <= 0) {
+      (void)cudaGetLastError();
+      nb = 1;
+    }
+    per_sm.store(nb);
+    done.store(smem);
   }
-  return nb;
+  return per_sm.load();
 }
 
 // Launches `kern` with programmatic stream serialization: it may be scheduled
@@ -1134,81 +969,52 @@ rn_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
   return launch_status();
 }
 
+// The forward is persistent: one wave of CTAs (as many as fit on every SM).
 template <int DT, int T, int K, bool GATED, bool EXACT>
-rn_status launch_fwd_s(const FwdArgs& a, cudaStream_t st) {
-  constexpr int NTEN = GATED ? 2 : 1;
-  constexpr int kFwdsBlock = fwds_block<K>();
-  const size_t smem = size_t(K) * T * (DT == RN_BF16 ? 8 : 4) * sizeof(float) +
-                      size_t(kFwdStages) * NTEN * K * kFwdsBlock * 16;
+rn_status launch_fwd_tk(const Sched& s, const FwdArgs& a, cudaStream_t st) {
+  constexpr int B = fwd_block<T, K>();
+  const size_t smem = fwd_smem_bytes(s, GATED, rn_dtype(DT));
+  static std::atomic<size_t> done{0};
   static std::atomic<int> per_sm{0};
-  int nb = per_sm.load();
-  if (nb <= 0) {
-    nb = blocks_per_sm(k_fwd_s<DT, T, K, GATED, EXACT>, kFwdsBlock, smem);
-    per_sm.store(nb);
-  }
-  const int64_t nblk = (a.rows + kFwdsBlock / T - 1) / (kFwdsBlock / T);
+  const int nb = prepare_kernel(k_fwd<DT, T, K, GATED, EXACT>, B, smem, done, per_sm);
+  const int64_t nblk = (a.rows + B / T - 1) / (B / T);
   const int64_t wave = int64_t(nb) * sm_count();
   const int grid = grid_cap(nblk < wave ? nblk : wave);
-  return launch_pdl(k_fwd_s<DT, T, K, GATED, EXACT>, dim3(grid), dim3(kFwdsBlock), smem, st, a);
+  return launch_pdl(k_fwd<DT, T, K, GATED, EXACT>, dim3(grid), dim3(B), smem, st, a);
 }
 
 template <int DT, bool GATED>
 rn_status launch_fwd(const Sched& s, const FwdArgs& a, cudaStream_t st) {
-  if (s.T <= 16) {
-    const bool ex = a.nv == s.T * s.K;
-#define RN_FWDS_CASE(T_, K_)                                                    \
-    if (s.T == T_ && s.K == K_)                                                 \
-      return ex ? launch_fwd_s<DT, T_, K_, GATED, true>(a, st)                  \
-                : launch_fwd_s<DT, T_, K_, GATED, false>(a, st);
-    RN_TK_SMALL(RN_FWDS_CASE)
-#undef RN_FWDS_CASE
-    return RN_E_WIDTH;
-  }
-  const int64_t per_cta = fwd_rows_per_cta_rt(s.T);
-  const int grid = grid_cap((a.rows + per_cta - 1) / per_cta);
-  const int block = fwd_block_rt(s.T);
-  const bool exact = a.nv == s.T * s.K;
+  const bool ex = a.nv == s.T * s.K;
 #define RN_FWD_CASE(T_, K_)                                                     \
-  if constexpr (T_ > 16) {                                                      \
-    if (s.T == T_ && s.K == K_) {                                               \
-      if (exact)                                                                \
-        return launch_pdl(k_fwd<DT, T_, K_, GATED, true>, dim3(grid), dim3(block), 0, st, a);  \
-      else                                                                      \
-        return launch_pdl(k_fwd<DT, T_, K_, GATED, false>, dim3(grid), dim3(block), 0, st, a); \
-    }                                                                           \
-  }
+  if (s.T == T_ && s.K == K_)                                                   \
+    return ex ? launch_fwd_tk<DT, T_, K_, GATED, true>(s, a, st)                \
+              : launch_fwd_tk<DT, T_, K_, GATED, false>(s, a, st);
   RN_TK_LIST(RN_FWD_CASE)
 #undef RN_FWD_CASE
   return RN_E_WIDTH;
 }
 
+// The backward runs one CTA per group of leaves (grid-stride if capped).
+template <int DT, int T, int K, bool GATED, bool EXACT>
+rn_status launch_bwd_tk(const Sched& s, int lpc, const BwdArgs& a, int64_t groups,
+                        cudaStream_t st) {
+  const int block = lpc * T;
+  const size_t smem = bwd_smem_bytes(s, lpc, a.H, GATED, rn_dtype(DT));
+  static std::atomic<size_t> done{0};
+  static std::atomic<int> per_sm{0};
+  (void)prepare_kernel(k_bwd<DT, T, K, GATED, EXACT>, block, smem, done, per_sm);
+  return launch_pdl(k_bwd<DT, T, K, GATED, EXACT>, dim3(grid_cap(groups)), dim3(block), smem,
+                    st, a);
+}
+
 template <int DT, bool GATED>
 rn_status launch_bwd(const Sched& s, int lpc, const BwdArgs& a, int64_t groups, cudaStream_t st) {
-  const int grid = grid_cap(groups);
-  const int block = lpc * s.T;
-  const size_t smem = bwd_smem_bytes(s, lpc, a.H, GATED);
-  const bool exact = a.nv == s.T * s.K;
-  if (bwd_pipelined(s)) {
-#define RN_BWDS_CASE(T_, K_)                                                    \
-    if (s.T == T_ && s.K == K_) {                                               \
-      if (exact)                                                                \
-        return launch_pdl(k_bwd_s<DT, T_, K_, GATED, true>, dim3(grid), dim3(block), smem, st, a); \
-      else                                                                      \
-        return launch_pdl(k_bwd_s<DT, T_, K_, GATED, false>, dim3(grid), dim3(block), smem, st, a); \
-    }
-    RN_TK_SMALL(RN_BWDS_CASE)
-#undef RN_BWDS_CASE
-    return RN_E_WIDTH;
-  }
+  const bool ex = a.nv == s.T * s.K;
 #define RN_BWD_CASE(T_, K_)                                                     \
-  if constexpr (T_ > 16) {                                                      \
-    if (s.T == T_ && s.K == K_) {                                               \
-      if (exact)                                                                \
-        return launch_pdl(k_bwd<DT, T_, K_, GATED, true>, dim3(grid), dim3(block), smem, st, a); \
-      else                                                                      \
-        return launch_pdl(k_bwd<DT, T_, K_, GATED, false>, dim3(grid), dim3(block), smem, st, a); \
-    }                                                                           \
-  }
+  if (s.T == T_ && s.K == K_)                                                   \
+    return ex ? launch_bwd_tk<DT, T_, K_, GATED, true>(s, lpc, a, groups, st)   \
+              : launch_bwd_tk<DT, T_, K_, GATED, false>(s, lpc, a, groups, st);
   RN_TK_LIST(RN_BWD_CASE)
 #undef RN_BWD_CASE
   return RN_E_WIDTH;
@@ -1317,7 +1123,7 @@ rn_status bwd_entry(int64_t rows, int32_t width, float eps, rn_dtype dt, const v
   }
   Sched s;
   pick_sched(width, dt, &s);
-  const int lpc = leaves_per_cta(s, width);
+  const int lpc = leaves_per_cta(s, width, dt);
   const int64_t leaves = n_leaves_of(rows);
   const int64_t groups = (leaves + lpc - 1) / lpc;
   float* region_a = static_cast<float*>(ws);
@@ -1400,11 +1206,27 @@ rn_status gated_norm_bwd(int64_t rows, int32_t width, float eps, rn_dtype dt, co
                          stream);
 }
 
+rn_status rn_fold_rows(int64_t n, int32_t width, const float* in, float* out, rn_stream stream) {
+  if (n < 1 || n > 256) return RN_E_ARG;
+  if (!width_ok(width)) return RN_E_WIDTH;
+  if (!in || !out) return RN_E_ARG;
+  if (!aligned16(in) || !aligned16(out)) return RN_E_ALIGN;
+  const Range rin[] = {{in, size_t(n) * width * sizeof(float)}};
+  const Range rout[] = {{out, size_t(width) * sizeof(float)}};
+  const rn_status e = check_ranges(rin, 1, rout, 1);
+  if (e != RN_OK || g_validate_only.load()) return e;
+  int S = 8;
+  while (S < n) S <<= 1;   // one pass: a CTA folds all n rows of its columns
+  const int gy = (width / 4 + 31) / 32;
+  return launch_fold(S / kFoldRG, dim3(1, gy), static_cast<cudaStream_t>(stream), in, n, width,
+                     out);
+}
+
 const char* rn_describe(int32_t width, rn_dtype dt) {
   Sched s;
   if (!pick_sched(width, dt, &s)) return "unsupported";
   const int VE = dt == RN_BF16 ? 8 : 4;
-  const int lpc = leaves_per_cta(s, width);
+  const int lpc = leaves_per_cta(s, width, dt);
   std::snprintf(t_describe, sizeof t_describe,
                 "backend=cuda-sm100a lib=librn kernels=k_fwd,k_bwd,k_fold dtype=%s width=%d "
                 "acc=fp32 team_threads=%d vectors_per_thread=%d elems_per_vector=%d "
@@ -1419,7 +1241,7 @@ const char* rn_describe(int32_t width, rn_dtype dt) {
 int32_t rn_bwd_launches(int64_t rows, int32_t width, rn_dtype dt) {
   Sched s;
   if (rows <= 0 || rows > kMaxRows || !pick_sched(width, dt, &s)) return 0;
-  const int lpc = leaves_per_cta(s, width);
+  const int lpc = leaves_per_cta(s, width, dt);
   const int64_t groups = (n_leaves_of(rows) + lpc - 1) / lpc;
   return 1 + fold_passes(groups);
 }

@@ -164,6 +164,22 @@ def gated_norm_bwd(x: torch.Tensor, z: torch.Tensor, w: torch.Tensor, dy: torch.
     return dx, dz, dw
 
 
+def rn_fold_rows(partials: torch.Tensor, *, out: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """Joins the rows of a [n, width] fp32 CUDA tensor of dw partials with the
+    backward's pairwise tree; returns the [width] result."""
+    if partials.dim() != 2 or partials.dtype != torch.float32 or not partials.is_cuda \
+            or not partials.is_contiguous():
+        raise ValueError("partials must be a contiguous fp32 CUDA tensor [n, width]")
+    n, width = int(partials.shape[0]), int(partials.shape[1])
+    out = torch.empty(width, dtype=torch.float32, device=partials.device) if out is None else \
+        _vec("out", out, width, partials.device)
+    with torch.cuda.device(partials.device):
+        check("rn_fold_rows", load().rn_fold_rows(n, width, _ptr(partials), _ptr(out),
+                                                  _stream(partials, stream)))
+    return out
+
+
 def rn_describe(width: int, dtype=torch.bfloat16) -> str:
     dt = _DT[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
     return load().rn_describe(width, dt).decode()

@@ -244,6 +244,18 @@ def test_bwd_launch_count(lib):
         lib.rn_test_set_geometry(0, 0, 0)
 
 
+def test_fold_rows_checks(lib):
+    with validate_only(lib):
+        assert lib.rn_fold_rows(8, 128, P(X), P(Y), None) == Status.OK
+        assert lib.rn_fold_rows(256, 128, P(X), P(Y), None) == Status.OK
+        assert lib.rn_fold_rows(0, 128, P(X), P(Y), None) == Status.E_ARG
+        assert lib.rn_fold_rows(257, 128, P(X), P(Y), None) == Status.E_ARG
+        assert lib.rn_fold_rows(8, 12, P(X), P(Y), None) == Status.E_WIDTH
+        assert lib.rn_fold_rows(8, 128, P(X, 4), P(Y), None) == Status.E_ALIGN
+        assert lib.rn_fold_rows(8, 128, P(X), P(X, 7 * 512), None) == Status.E_ARG   # overlap
+        assert lib.rn_fold_rows(8, 128, 0, P(Y), None) == Status.E_ARG
+
+
 def test_status_strings(lib):
     for s in Status:
         assert lib.rn_status_string(int(s))
