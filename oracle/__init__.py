@@ -4,12 +4,15 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline and
 reference legs may import this package.  The library never does.
 """
 from .rmsnorm import (  # noqa: F401
+    ACTS,
     dx_cancellation_scale,
     dz_cancellation_scale,
     gated_norm_bwd,
     gated_norm_fwd,
     norm_bwd,
     norm_fwd,
+    rmsnorm_bwd,
+    rmsnorm_fwd,
     rstd,
     sigmoid,
     silu,

@@ -36,14 +36,32 @@ ungated dx with the gain (w + offset) replaced by (w + offset) * act(z)):
     dw_j = sum_r dy_rj * xh_rj                     (zero-centred)
          = sum_r dy_rj * xh_rj * silu(z_rj)        (gated)
 
+The general form ([PR468] Summary, the displayed formula and the
+"Activation" bullet: a weight offset and a gate activation, silu or sigmoid;
+[PR468] "Changes to existing code, in detail", "Signed zero" bullet: the offset
+is added only when it is nonzero, so a -0.0 weight keeps its sign):
+
+    u_j  = w_j + offset   (offset != 0)   or   w_j   (offset == 0)
+    y_j  = xh_j * u_j * a(z_j),  a = 1 (no gate), silu(z), or s(z)
+    g_j  = u_j * a(z_j);  dx as above;  dz_j = dy_j * xh_j * u_j * a'(z_j)
+    dw_j = sum_r dy_rj * xh_rj * a(z_rj)
+    a'(z) = s(z) * (1 + z * (1 - s(z)))  (silu)   or   s(z) * (1 - s(z))  (sigmoid)
+
+The zero-centred and gated operators above are (offset 1, no gate) and
+(offset 0, silu).
+
 Parity pins (``tests/oracle_pins.py``, run by ``tests/test_oracle_pins.py``,
 with planted mistakes in ``tests/test_oracle_mutations.py``):
   rstd/forward : constant-row closed form, RMS(xh) == 1 at eps = 0, scale
-                 invariance at eps = 0, w = 0 reduces y to xh, an exact rational
-                 worked example (tests/golden/), sigmoid at ln(k) points.
+                 invariance at eps = 0, w = 0 reduces y to xh, exact rational
+                 worked examples (in tests/oracle_pins.py), sigmoid at ln(k)
+                 points.
   backward     : central finite differences of L (dx, dz, dw), the scale
                  identity sum_j x_j dx_j = rho * S * eps / (ms + eps), and a
                  brute-force double loop for dw.
+  general form : a rational worked example (sigmoid gate, offset 1), finite
+                 differences for every activation x offset {0, 1, 1/2}, the
+                 signed-zero rule, and reduction to the two operators above.
 Every public function below is pinned; none is "parity unpinned".
 """
 from __future__ import annotations
@@ -168,3 +186,50 @@ def dz_cancellation_scale(x, z, w, dy, eps: float) -> np.ndarray:
     s = sigmoid(z)
     lead = np.abs(dy * x * rho[:, None] * w[None, :] * s)
     return lead * np.maximum(1.0, np.abs(z * (1.0 - s)))
+
+
+# ---------------------------------------------------------------------------
+# The general operator: weight offset and gate activation as parameters.
+# ---------------------------------------------------------------------------
+ACTS = ("none", "silu", "sigmoid")
+
+
+def _gain(w, weight_offset):
+    w = np.asarray(w, dtype=np.float64)
+    return w + weight_offset if weight_offset != 0 else w
+
+
+def _act(z, act):
+    """(a(z), a'(z)) for the gate; (1, 0) when there is none."""
+    if act == "none":
+        return 1.0, 0.0
+    s = sigmoid(z)
+    if act == "silu":
+        return z * s, s * (1.0 + z * (1.0 - s))
+    if act == "sigmoid":
+        return s, s * (1.0 - s)
+    raise ValueError(f"unknown activation {act!r}")
+
+
+def rmsnorm_fwd(x, w, eps: float, weight_offset: float = 1.0, z=None, act: str = "none"):
+    """y = x * rho * u * a(z) with u = w + offset (offset added only when
+    nonzero).  Returns (y, rho)."""
+    x = _rows(x)
+    rho = rstd(x, eps)
+    u = _gain(w, weight_offset)
+    a, _ = _act(None if z is None else _rows(z), act)
+    return x * rho[:, None] * u[None, :] * a, rho
+
+
+def rmsnorm_bwd(x, w, dy, eps: float, weight_offset: float = 1.0, z=None, act: str = "none"):
+    """Returns (dx, dz, dw); dz is None without a gate."""
+    x, dy = _rows(x), _rows(dy)
+    rho = rstd(x, eps)
+    xh = x * rho[:, None]
+    u = _gain(w, weight_offset)[None, :]
+    a, da = _act(None if z is None else _rows(z), act)
+    g = u * a
+    dx = _dx(x, np.broadcast_to(g, x.shape), dy, rho)
+    dz = None if act == "none" else dy * xh * u * da
+    dw = np.sum(dy * xh * a, axis=0)
+    return dx, dz, dw

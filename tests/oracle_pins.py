@@ -268,6 +268,100 @@ def pin_rows_independent(orc):
         _close(b, dz[s], rtol=0, atol=0, what="dz row")
 
 
+# --------------------------------------------------------------------------
+# the general operator: weight offset and gate activation
+# --------------------------------------------------------------------------
+def pin_worked_example_sigmoid_offset(orc):
+    """Sigmoid gate with offset 1, H=4, x=[1,2,2,4], eps=0 (rho=2/5,
+    xh=[2,4,4,8]/5), L = ln 3, z = [L, -L, 0, L]: a = s(z) = [3/4, 1/4, 1/2, 3/4],
+    a' = s(1-s) = [3/16, 3/16, 1/4, 3/16].  w = [0, 1/2, -1, 1] -> u = w+1 =
+    [1, 3/2, 0, 2];  y = xh*u*a = [3/10, 3/10, 0, 12/5].
+    dy = [1, -1, 2, 1/2]: g = u*a = [3/4, 3/8, 0, 3/2]; g*dy*xh = [3/10, -3/10,
+    0, 6/5], sum = 6/5, m = 3/10; xh*m = [3, 6, 6, 12]/25;
+    g*dy - xh*m = [63/100, -123/200, -6/25, 27/100];
+    dx = [63/250, -123/500, -12/125, 27/250];
+    dz = dy*xh*u*a' = [3/40, -9/40, 0, 3/10];  dw = dy*xh*a = [3/10, -1/5, 4/5, 3/5]."""
+    L = L3
+    x = [[1.0, 2.0, 2.0, 4.0]]
+    z = [[L, -L, 0.0, L]]
+    w = [0.0, 0.5, -1.0, 1.0]
+    dy = [[1.0, -1.0, 2.0, 0.5]]
+    y, rho = orc.rmsnorm_fwd(x, w, 0.0, weight_offset=1.0, z=z, act="sigmoid")
+    _close(rho, [0.4], what="rho")
+    _close(y, [[0.3, 0.3, 0.0, 2.4]], what="y")
+    dx, dz, dw = orc.rmsnorm_bwd(x, w, dy, 0.0, weight_offset=1.0, z=z, act="sigmoid")
+    _close(dx, [[63 / 250, -123 / 500, -12 / 125, 27 / 250]], what="dx")
+    _close(dz, [[3 / 40, -9 / 40, 0.0, 0.3]], what="dz")
+    _close(dw, [0.3, -0.2, 0.8, 0.6], what="dw")
+
+
+def pin_general_special_cases(orc):
+    """Offset 1 without a gate is the zero-centred operator; offset 0 with the
+    silu gate is the gated operator (both pinned above by worked examples)."""
+    rng = np.random.default_rng(19)
+    x = rng.normal(size=(3, 8)); z = rng.normal(size=(3, 8))
+    w = rng.normal(size=8); dy = rng.normal(size=(3, 8))
+    _close(orc.rmsnorm_fwd(x, w, 1e-6)[0], orc.norm_fwd(x, w, 1e-6)[0], what="plain y")
+    dx, dz, dw = orc.rmsnorm_bwd(x, w, dy, 1e-6)
+    assert dz is None
+    dx0, dw0 = orc.norm_bwd(x, w, dy, 1e-6)
+    _close(dx, dx0, what="plain dx"); _close(dw, dw0, what="plain dw")
+    _close(orc.rmsnorm_fwd(x, w, 1e-6, 0.0, z, "silu")[0], orc.gated_norm_fwd(x, z, w, 1e-6)[0],
+           what="gated y")
+    for got, want, n in zip(orc.rmsnorm_bwd(x, w, dy, 1e-6, 0.0, z, "silu"),
+                            orc.gated_norm_bwd(x, z, w, dy, 1e-6), ("dx", "dz", "dw")):
+        _close(got, want, what="gated " + n)
+
+
+def pin_general_finite_differences(orc):
+    """dx, dz, dw of every (activation, offset) equal the numerical gradient of
+    L = sum(y * dy)."""
+    rng = np.random.default_rng(20)
+    R, H, eps = 2, 6, 1e-2
+    x = rng.normal(size=(R, H)); z = rng.normal(size=(R, H)) * 2.0
+    w = rng.normal(size=H); dy = rng.normal(size=(R, H))
+    for act in ("none", "silu", "sigmoid"):
+        for off in (0.0, 1.0, 0.5):
+            zz = None if act == "none" else z
+
+            def L(x_, z_, w_):
+                return float(np.sum(orc.rmsnorm_fwd(x_, w_, eps, off, z_, act)[0] * dy))
+
+            dx, dz, dw = orc.rmsnorm_bwd(x, w, dy, eps, off, zz, act)
+            tag = f"{act} offset {off}"
+            _close(dx, _fd(lambda a: L(a, zz, w), x), rtol=1e-7, atol=1e-8, what=tag + " dx")
+            _close(dw, _fd(lambda a: L(x, zz, a), w), rtol=1e-7, atol=1e-8, what=tag + " dw")
+            if act != "none":
+                _close(dz, _fd(lambda a: L(x, a, w), z), rtol=1e-7, atol=1e-8, what=tag + " dz")
+
+
+def pin_signed_zero_weight(orc):
+    """The offset is added only when it is nonzero, so with offset 0 a -0.0
+    weight stays -0.0 and flips the sign of the zero it multiplies into (y and
+    dz); w + 0.0 would have made it +0.0.  With offset 1, -0.0 becomes 1."""
+    x = [[1.0, 2.0, -3.0, 4.0]]
+    z = [[0.5, -1.0, 2.0, 1.5]]
+    w = [-0.0, 0.0, -0.0, 2.0]
+    dy = [[1.0, 1.0, -1.0, 1.0]]
+    for act in ("none", "silu", "sigmoid"):
+        zz = None if act == "none" else z
+        y, _ = orc.rmsnorm_fwd(x, w, 0.0, 0.0, zz, act)
+        a = np.ones(4) if act == "none" else (orc.sigmoid(np.array(z[0])) if act == "sigmoid"
+                                             else orc.silu(np.array(z[0])))
+        pos = np.array(x[0]) * a > 0
+        assert y[0, 0] == 0 and bool(np.signbit(y[0, 0])) == bool(pos[0]), (act, y)
+        assert y[0, 1] == 0 and bool(np.signbit(y[0, 1])) != bool(pos[1]), (act, y)
+        assert y[0, 2] == 0 and bool(np.signbit(y[0, 2])) == bool(pos[2]), (act, y)
+        if act != "none":
+            _, dz, _ = orc.rmsnorm_bwd(x, w, dy, 0.0, 0.0, zz, act)
+            # dz = dy*xh*w*a'(z) with a' > 0 at these z: sign of dy*x flipped by -0.0
+            sdx = np.array(dy[0]) * np.array(x[0]) > 0
+            assert dz[0, 0] == 0 and bool(np.signbit(dz[0, 0])) == bool(sdx[0]), (act, dz)
+            assert dz[0, 2] == 0 and bool(np.signbit(dz[0, 2])) == bool(sdx[2]), (act, dz)
+        y1, _ = orc.rmsnorm_fwd(x, w, 0.0, 1.0, zz, act)
+        assert y1[0, 0] != 0 and y1[0, 2] != 0, (act, y1)
+
+
 ALL_PINS = [
     pin_worked_example_norm,
     pin_worked_example_eps,
@@ -281,6 +375,10 @@ ALL_PINS = [
     pin_finite_differences,
     pin_dw_brute_force,
     pin_rows_independent,
+    pin_worked_example_sigmoid_offset,
+    pin_general_special_cases,
+    pin_general_finite_differences,
+    pin_signed_zero_weight,
 ]
 
 

@@ -162,6 +162,54 @@ def m_norm_dw_wrong_axis(o):
     o.norm_bwd = norm_bwd
 
 
+def m_general_offset_always_added(o):
+    o._gain = lambda w, off: np.asarray(w, dtype=np.float64) + off
+
+
+def m_general_offset_never_added(o):
+    o._gain = lambda w, off: np.asarray(w, dtype=np.float64)
+
+
+def m_general_sigmoid_takes_silu_derivative(o):
+    real = o._act
+
+    def _act(z, act):
+        a, da = real(z, act)
+        if act == "sigmoid":
+            s = o.sigmoid(z)
+            da = s * (1.0 + z * (1.0 - s))
+        return a, da
+    o._act = _act
+
+
+def m_general_sigmoid_gate_is_silu(o):
+    real = o._act
+    o._act = lambda z, act: real(z, "silu" if act == "sigmoid" else act)
+
+
+def m_general_dz_without_offset(o):
+    real = o.rmsnorm_bwd
+
+    def rmsnorm_bwd(x, w, dy, eps, weight_offset=1.0, z=None, act="none"):
+        dx, dz, dw = real(x, w, dy, eps, weight_offset, z, act)
+        if dz is not None and weight_offset != 0:
+            u = o._gain(w, weight_offset)
+            dz = dz / u[None, :] * np.asarray(w, dtype=np.float64)[None, :]
+        return dx, dz, dw
+    o.rmsnorm_bwd = rmsnorm_bwd
+
+
+def m_general_dw_drops_gate(o):
+    real = o.rmsnorm_bwd
+
+    def rmsnorm_bwd(x, w, dy, eps, weight_offset=1.0, z=None, act="none"):
+        dx, dz, _ = real(x, w, dy, eps, weight_offset, z, act)
+        x = np.asarray(x, dtype=np.float64)
+        xh = x * o.rstd(x, eps)[:, None]
+        return dx, dz, np.sum(np.asarray(dy, dtype=np.float64) * xh, axis=0)
+    o.rmsnorm_bwd = rmsnorm_bwd
+
+
 MUTANTS = [m for name, m in sorted(globals().items()) if name.startswith("m_")]
 
 
