@@ -3,9 +3,12 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = gated_norm_fwd + gated_norm_bwd (the backward kernel and its dw
-fold) over one batch of 262144 rows (8192 tokens x 32 heads) x 128, bf16, with
-1% of channels scaled x50 in x, z and dy (seeded synthetic data).  Prints one
+One step = rmsnorm_fwd + rmsnorm_bwd (the backward kernel and its dw fold)
+with the workload's gate activation and weight offset; by default the gated
+operator (silu, offset 0: the kernels gated_norm_fwd / gated_norm_bwd run) over
+one batch of 262144 rows (8192 tokens x 32 heads) x 128, bf16, with 1% of
+channels scaled x50 in x, z and dy (seeded synthetic data).  --workload picks
+another configuration or a variant (sigmoid gate, fp16, offset).  Prints one
 JSON line on rank 0.
 
 value     = algorithmic HBM bytes of all steps on all ranks / max-over-ranks time
@@ -60,7 +63,7 @@ def parse():
     ap.add_argument("--no-invariance", action="store_true")
     ap.add_argument("--buffer-sets", type=int, default=SETS,
                     help="rotating input sets (fewer only for profiler captures)")
-    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(workloads.CONFIGS),
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(workloads.ALL),
                     help="which synthetic workload one step runs (default: the headline)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every call from Python instead of replaying a CUDA graph")
@@ -86,22 +89,39 @@ def peaks():
 
 
 def src_sha():
+    """Digest of the kernel sources (csrc/*.cu, *.cuh) and the C header."""
     h = hashlib.sha1()
-    for f in ("rollout_parity_b200/csrc/rn.cu", "include/rn.h"):
-        h.update(open(os.path.join(ROOT, f), "rb").read())
+    csrc = os.path.join(ROOT, "rollout_parity_b200", "csrc")
+    files = sorted(f for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
+    for f in [os.path.join(csrc, f) for f in files] + [os.path.join(ROOT, "include", "rn.h")]:
+        h.update(open(f, "rb").read())
     return h.hexdigest()[:12]
 
 
-def profiled_traffic():
-    """DRAM bytes per backward call from the committed ncu summary, if it was
-    taken on the current kernel source; else None."""
+def op_name(wl):
+    if wl.act == "none":
+        return ("zero-centred RMSNorm fwd+bwd" if wl.weight_offset == 1.0 else
+                f"RMSNorm (weight offset {wl.weight_offset:g}) fwd+bwd")
+    if wl.act == "silu" and wl.weight_offset == 0.0:
+        return "gated RMSNorm fwd+bwd"
+    return f"gated RMSNorm ({wl.act} gate, weight offset {wl.weight_offset:g}) fwd+bwd"
+
+
+def esize_of(wl):
+    return 4 if wl.dtype == "f32" else 2
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per backward call of this workload from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
     want = src_sha()
     for ln in open(p):
         kv = dict(t.split("=", 1) for t in ln.split() if "=" in t)
-        if kv.get("unit") == "gated_norm_bwd" and kv.get("source_sha1") == want:
+        if (kv.get("workload") == workload and kv.get("unit") == "bwd_call"
+                and kv.get("source_sha1") == want):
             return int(kv["dram_bytes_per_call"])
     return None
 
@@ -188,6 +208,7 @@ def dist_setup(n):
 def run_ours(a):
     import rollout_parity_b200 as rn
     from rollout_parity_b200._lib import DType, check
+    from rollout_parity_b200.ops import act_code
 
     rank, local, world, dist, dt_mod = dist_setup(a.gpus)
     torch.cuda.set_device(local)
@@ -198,45 +219,42 @@ def run_ours(a):
     lib = rn.load()
 
     nsets = max(1, a.buffer_sets)
-    make = workloads.CONFIGS[a.workload]
+    make = workloads.ALL[a.workload]
     host = [make(seed=1000 * rank + s) for s in range(nsets)]
-    R, H, eps = host[0].rows, host[0].width, host[0].eps
-    gated = host[0].gated
-    dtc = int(DType.BF16 if host[0].dtype == "bf16" else DType.F32)
-    esize = 2 if host[0].dtype == "bf16" else 4
+    wl0 = host[0]
+    R, H, eps = wl0.rows, wl0.width, wl0.eps
+    gated = wl0.gated
+    dtc = int({"bf16": DType.BF16, "f16": DType.F16, "f32": DType.F32}[wl0.dtype])
+    actc, woff = int(act_code(wl0.act)), wl0.weight_offset
+    esize = esize_of(wl0)
     fwd_b, bwd_b = bytes_model(R, H, esize=esize, gated=gated)
     step_b = fwd_b + bwd_b
     nws = lib.norm_bwd_workspace_bytes(R, H)
     sets = []
     for wl in host:
         d = wl.to(dev)
-        sets.append(dict(x=d.x, z=d.z if gated else d.x, w=d.w, dy=d.dy, y=torch.empty_like(d.x),
+        sets.append(dict(x=d.x, z=d.z, w=d.w, dy=d.dy, y=torch.empty_like(d.x),
                          rstd=torch.empty(R, dtype=torch.float32, device=dev),
-                         dx=torch.empty_like(d.x), dz=torch.empty_like(d.x),
+                         dx=torch.empty_like(d.x), dz=torch.empty_like(d.x) if gated else None,
                          dw=torch.empty(H, dtype=torch.float32, device=dev),
                          ws=torch.empty(nws, dtype=torch.uint8, device=dev)))
-    P = [{k: v.data_ptr() for k, v in s.items()} for s in sets]
+    P = [{k: (None if v is None else v.data_ptr()) for k, v in s.items()} for s in sets]
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
 
     def fwd(p, stp=sp):
-        if gated:
-            return lib.gated_norm_fwd(R, H, eps, dtc, p["x"], p["z"], p["w"], p["y"], p["rstd"],
-                                      stp)
-        return lib.norm_fwd(R, H, eps, dtc, p["x"], p["w"], p["y"], p["rstd"], stp)
+        return lib.rmsnorm_fwd(R, H, eps, woff, actc, dtc, p["x"], p["z"], p["w"], p["y"],
+                               p["rstd"], stp)
 
     def bwd(p, stp=sp):
-        if gated:
-            return lib.gated_norm_bwd(R, H, eps, dtc, p["x"], p["z"], p["w"], p["dy"], p["rstd"],
-                                      p["dx"], p["dz"], p["dw"], p["ws"], nws, stp)
-        return lib.norm_bwd(R, H, eps, dtc, p["x"], p["w"], p["dy"], p["rstd"], p["dx"], p["dw"],
-                            p["ws"], nws, stp)
+        return lib.rmsnorm_bwd(R, H, eps, woff, actc, dtc, p["x"], p["z"], p["w"], p["dy"],
+                               p["rstd"], p["dx"], p["dz"], p["dw"], p["ws"], nws, stp)
 
     for p in P:                       # every set gets its rstd before any backward
-        check("gated_norm_fwd", fwd(p))
+        check("rmsnorm_fwd", fwd(p))
     for k in range(a.warmup):
-        check("gated_norm_fwd", fwd(P[k % nsets]))
-        check("gated_norm_bwd", bwd(P[(k + 2) % nsets]))
+        check("rmsnorm_fwd", fwd(P[k % nsets]))
+        check("rmsnorm_bwd", bwd(P[(k + 2) % nsets]))
     torch.cuda.synchronize()
 
     K = a.steps
@@ -305,8 +323,8 @@ def run_ours(a):
                 exchange(sets[(k + 2) % nsets]["dw"])
             e[2].record(stream)
             if s1 or s2:
-                check("gated_norm_fwd", s1)
-                check("gated_norm_bwd", s2)
+                check("rmsnorm_fwd", s1)
+                check("rmsnorm_bwd", s2)
     t_end.record(stream)
     torch.cuda.synchronize()
     clocks.mark("t1")
@@ -328,7 +346,7 @@ def run_ours(a):
     value = world * step_b * K / (ms / 1e3) / 1e9
     launches = K * (1 + lib.rn_bwd_launches(R, H, dtc))
 
-    inv = invariance_checks(rn, sets[0], R, H, eps, gated) \
+    inv = invariance_checks(rn, sets[0], R, H, eps, wl0) \
         if rank == 0 and not a.no_invariance else None
     e2e = run_e2e(rn, host[0], dev, a.e2e_steps, step_b, world, dist) if a.e2e_steps > 0 \
         else None
@@ -341,18 +359,20 @@ def run_ours(a):
         bwd_mean = float(np.mean(bwd_ms))
         fwd_mean = float(np.mean(fwd_ms))
         achieved = bwd_b / (bwd_mean / 1e3) / 1e9
-        traffic = profiled_traffic()
+        traffic = profiled_traffic(a.workload)
         desc = {WORKLOAD: {"layout": "8192 tokens x 32 heads, row = token*32 + head",
                            "outliers": "1% of channels x50 in x, z, dy"}}.get(a.workload, {})
-        opname = "gated RMSNorm fwd+bwd" if gated else "zero-centred RMSNorm fwd+bwd"
-        iod = host[0].dtype
+        opname = op_name(wl0)
+        iod = wl0.dtype
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": a.warmup, "ms_per_step": round(ms_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": iod,
             "data": "synthetic (seeded; no dataset or checkpoint)",
             "config": {"workload": a.workload, "op": opname, "rows": R, "width": H, **desc,
-                       "eps": eps, "io_dtype": f"{iod} x/z/dy/y/dx/dz, fp32 w/rstd/dw",
+                       "activation": wl0.act, "weight_offset": woff,
+                       "eps": eps, "io_dtype": (f"{iod} x/z/dy/y/dx/dz" if gated else
+                                                f"{iod} x/dy/y/dx") + ", fp32 w/rstd/dw",
                        "accumulate": "fp32",
                        "bytes_per_step": step_b,
                        "parallelism": (f"data parallel x{world}: rows split across ranks, dw "
@@ -374,8 +394,7 @@ def run_ours(a):
             "bwd_gbs": round(achieved, 1),
             "invariance": inv,
             "roofline": {"bound": "hbm",
-                         "kernel": ("gated_norm_bwd" if gated else "norm_bwd") +
-                                   " call (k_bwd + k_fold passes)",
+                         "kernel": "rmsnorm_bwd call (k_bwd + k_fold passes)",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_source": src,
                          "traffic": traffic, "algorithmic_bytes": bwd_b},
@@ -388,26 +407,25 @@ def run_ours(a):
         dist.destroy_process_group()
 
 
-def invariance_checks(rn, s, R, H, eps, gated=True):
+def invariance_checks(rn, s, R, H, eps, wl):
     """Bitwise: rows inside the full batch vs the same rows as their own batch,
     and dw across repeats and launch geometries."""
-    def fb(x, z, dy):
-        if gated:
-            y, r = rn.gated_norm_fwd(x, z, s["w"], eps)
-            dx, dz, dw = rn.gated_norm_bwd(x, z, s["w"], dy, r, eps)
-            return [y, r, dx, dz], dw
-        y, r = rn.norm_fwd(x, s["w"], eps)
-        dx, dw = rn.norm_bwd(x, s["w"], dy, r, eps)
-        return [y, r, dx], dw
+    gated = wl.gated
 
-    bits = lambda t: t.view(torch.int16 if t.dtype == torch.bfloat16 else torch.int32)
+    def fb(x, z, dy):
+        y, r = rn.rmsnorm_fwd(x, s["w"], eps, wl.weight_offset, z, wl.act)
+        dx, dz, dw = rn.rmsnorm_bwd(x, s["w"], dy, r, eps, wl.weight_offset, z, wl.act)
+        return ([y, r, dx, dz] if gated else [y, r, dx]), dw
+
+    bits = lambda t: t.view(torch.int32 if t.dtype == torch.float32 else torch.int16)
+    cl = lambda t, sl: None if t is None else t[sl].clone()
     full, dw = fb(s["x"], s["z"], s["dy"])
     checks, bad = 0, 0
     for st, n in ((R // 3, 1), (R // 5, 7), (R // 2 - 5, min(4099, R // 2)), (R - 33, 33)):
         if st < 0 or st + n > R:
             continue
         sl = slice(st, st + n)
-        part, _ = fb(s["x"][sl].clone(), s["z"][sl].clone(), s["dy"][sl].clone())
+        part, _ = fb(cl(s["x"], sl), cl(s["z"], sl), cl(s["dy"], sl))
         for a_, b_ in zip([t[sl] for t in full], part):
             checks += 1
             bad += int(not torch.equal(bits(a_), bits(b_)))
@@ -449,12 +467,10 @@ def run_e2e(rn, wl, dev, steps, step_b, world, dist):
             z.copy_(hz, non_blocking=True)
         dy.copy_(hdy, non_blocking=True)
         w.copy_(hw, non_blocking=True)
-        if gated:
-            rn.gated_norm_fwd(x, z, w, eps, y=y, rstd=rstd)
-            rn.gated_norm_bwd(x, z, w, dy, rstd, eps, dx=dx, dz=dz, dw=dw, ws=ws)
-        else:
-            rn.norm_fwd(x, w, eps, y=y, rstd=rstd)
-            rn.norm_bwd(x, w, dy, rstd, eps, dx=dx, dw=dw, ws=ws)
+        zz = z if gated else None
+        rn.rmsnorm_fwd(x, w, eps, wl.weight_offset, zz, wl.act, y=y, rstd=rstd)
+        rn.rmsnorm_bwd(x, w, dy, rstd, eps, wl.weight_offset, zz, wl.act, dx=dx,
+                       dz=dz if gated else None, dw=dw, ws=ws)
         oy.copy_(y, non_blocking=True)
         ors.copy_(rstd, non_blocking=True)
         odx.copy_(dx, non_blocking=True)
@@ -481,19 +497,15 @@ def run_e2e(rn, wl, dev, steps, step_b, world, dist):
     return {"value": round(world * step_b * steps / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 4),
-            "api": "rollout_parity_b200." + ("gated_norm_fwd/bwd" if gated else "norm_fwd/bwd")}
+            "api": "rollout_parity_b200.rmsnorm_fwd/rmsnorm_bwd"}
 
 
 # ---------------------------------------------------------------------------
 # the fp64 oracle on the host cores
 # ---------------------------------------------------------------------------
-def _oracle_step(orc, x, z, w, dy, eps):
-    if z is None:
-        orc.norm_fwd(x, w, eps)
-        orc.norm_bwd(x, w, dy, eps)
-        return
-    orc.gated_norm_fwd(x, z, w, eps)
-    orc.gated_norm_bwd(x, z, w, dy, eps)
+def _oracle_step(orc, wl, x, z, w, dy):
+    orc.rmsnorm_fwd(x, w, wl.eps, wl.weight_offset, z, wl.act)
+    orc.rmsnorm_bwd(x, w, dy, wl.eps, wl.weight_offset, z, wl.act)
 
 
 def cpu_baseline(wl, fwd_b, bwd_b, min_s=10.0, max_s=30.0):
@@ -504,12 +516,12 @@ def cpu_baseline(wl, fwd_b, bwd_b, min_s=10.0, max_s=30.0):
         n = max(32, (1 << 26) // wl.width)
         x, dy = x[:n], dy[:n]
         z = None if z is None else z[:n]
-        fwd_b, bwd_b = bytes_model(n, wl.width, 2 if wl.dtype == "bf16" else 4, wl.gated)
+        fwd_b, bwd_b = bytes_model(n, wl.width, esize_of(wl), wl.gated)
     else:
         n = wl.rows
     reps, t0 = 0, time.perf_counter()
     while True:
-        _oracle_step(oracle, x, z, w, dy, wl.eps)
+        _oracle_step(oracle, wl, x, z, w, dy)
         reps += 1
         el = time.perf_counter() - t0
         if el >= min_s or el * (reps + 1) / reps > max_s:
@@ -526,27 +538,27 @@ def run_reference(a):
     if rank != 0:
         return
     import oracle
-    wl = workloads.CONFIGS[a.workload]()
+    wl = workloads.ALL[a.workload]()
     R, H, eps = wl.rows, wl.width, wl.eps
     f = workloads.as_f64
     fz = (lambda t: None) if not wl.gated else f
     # size the per-step row sample so the whole run stays near a minute of CPU
     probe = min(R, max(32, 4096 * 128 // H))
     t0 = time.perf_counter()
-    _oracle_step(oracle, f(wl.x[:probe]), fz(wl.z[:probe] if wl.gated else None), f(wl.w),
-                 f(wl.dy[:probe]), eps)
+    _oracle_step(oracle, wl, f(wl.x[:probe]), fz(wl.z[:probe] if wl.gated else None), f(wl.w),
+                 f(wl.dy[:probe]))
     per_row = (time.perf_counter() - t0) / probe
     n = int(60.0 / per_row / max(1, a.steps + a.warmup))
     n = max(32, min(R, n // 32 * 32))
     x, w, dy = f(wl.x[:n]), f(wl.w), f(wl.dy[:n])
     z = f(wl.z[:n]) if wl.gated else None
     for _ in range(a.warmup):
-        _oracle_step(oracle, x, z, w, dy, eps)
+        _oracle_step(oracle, wl, x, z, w, dy)
     t0 = time.perf_counter()
     for _ in range(a.steps):
-        _oracle_step(oracle, x, z, w, dy, eps)
+        _oracle_step(oracle, wl, x, z, w, dy)
     el = time.perf_counter() - t0
-    fwd_b, bwd_b = bytes_model(n, H, 2 if wl.dtype == "bf16" else 4, wl.gated)
+    fwd_b, bwd_b = bytes_model(n, H, esize_of(wl), wl.gated)
     value = (fwd_b + bwd_b) * a.steps / el / 1e9
     sample = (f"fp64 numpy oracle fwd+bwd on rows [0, {n}) of the {R}-row workload per step "
               f"(single thread)")
@@ -557,7 +569,7 @@ def run_reference(a):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded; no dataset or checkpoint)",
         "config": {"workload": a.workload,
-                   "op": "gated RMSNorm fwd+bwd" if wl.gated else "zero-centred RMSNorm fwd+bwd",
+                   "op": op_name(wl),
                    "rows": R, "width": H, "sample_rows_per_step": n},
         "rows_per_s": round(n * a.steps / el, 1),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",

@@ -12,8 +12,21 @@
  *   gated:         y_j = x_j * rstd * w_j * silu(z_j)   (weight offset 0,
  *                  norm before gate, one group per row, silu = z * sigmoid(z))
  *
- * and the backward (the "Backward" bullet of the same section, and the
- * calculus of the forward), with g_j = 1 + w_j or w_j * silu(z_j):
+ * and, in general (the displayed formula and the "Activation" bullet of the
+ * same section), with a weight offset and a gate activation a:
+ *
+ *   y_j = x_j * rstd * u_j * a(z_j),  u_j = w_j + offset,  a = silu or sigmoid
+ *
+ * where the offset is added only when it is nonzero, so with offset 0 a -0.0
+ * weight keeps its sign (the "Signed zero" bullet of that page's "Changes to
+ * existing code, in detail").  The zero-centred operator is offset 1 with no
+ * gate, the gated one offset 0 with silu; rmsnorm_fwd / rmsnorm_bwd take both
+ * as arguments.
+ *
+ * The backward (the "Backward" bullet of the same section, and the calculus
+ * of the forward), with g_j = 1 + w_j or w_j * silu(z_j) (in general
+ * g_j = u_j * a(z_j), dz_j = dy_j * x_j * rstd * u_j * a'(z_j) and
+ * dw_j sums dy_j * x_j * rstd * a(z_j)):
  *
  *   m     = mean_j(g_j * dy_j * x_j * rstd)
  *   dx_j  = rstd * (g_j * dy_j - x_j * rstd * m)
@@ -38,7 +51,7 @@
  * Data layout and ownership
  * -------------------------
  * x, z, dy, y, dx, dz: row-major contiguous [rows, width] of dtype `dt`
- *   (RN_BF16 or RN_F32); y, dx, dz take the dtype of x.
+ *   (RN_BF16, RN_F16 or RN_F32); y, dx, dz take the dtype of x.
  * w: fp32 [width].  rstd: fp32 [rows].  dw: fp32 [width].
  * All pointers are DEVICE pointers on the device that is current when the
  * call is made, and `stream` is a cudaStream_t of that device (NULL = the
@@ -50,10 +63,11 @@
  * ------
  * Every argument is checked before anything is enqueued.  A failed check
  * returns its status and enqueues nothing:
- *   RN_E_ARG       rows < 0 or > 2^36, eps negative or not finite, a required
- *                  pointer is NULL, or an output overlaps an input or another
- *                  output;
- *   RN_E_DTYPE     dt is not RN_BF16 or RN_F32;
+ *   RN_E_ARG       rows < 0 or > 2^36, eps negative or not finite, the
+ *                  weight offset not finite, an unknown activation, a
+ *                  required pointer is NULL (or z / dz given without a
+ *                  gate), or an output overlaps an input or another output;
+ *   RN_E_DTYPE     dt is not RN_BF16, RN_F16 or RN_F32;
  *   RN_E_WIDTH     width is not a multiple of 8 in [8, 16384];
  *   RN_E_ALIGN     a tensor pointer is not 16-byte aligned (rstd: 4 bytes);
  *   RN_E_WORKSPACE the backward's workspace is NULL or smaller than
@@ -84,14 +98,51 @@ typedef enum {
 
 typedef enum {
     RN_F32 = 0,
-    RN_BF16 = 1
+    RN_BF16 = 1,
+    RN_F16 = 2
 } rn_dtype;
+
+/* Gate activation a(z) (PR #468 Summary, "Activation" bullet; "swish" is
+ * another name for silu).  RN_ACT_NONE: the ungated operator, no z. */
+typedef enum {
+    RN_ACT_NONE = 0,
+    RN_ACT_SILU = 1,       /* a(z) = z * s(z),  s(z) = 1 / (1 + exp(-z)) */
+    RN_ACT_SIGMOID = 2     /* a(z) = s(z) */
+} rn_act;
 
 /* A cudaStream_t, passed as a plain pointer so this header needs no CUDA. */
 typedef void* rn_stream;
 
 /*
+ * General forward (PR #468 Summary, the displayed formula):
+ *   y[r, j] = x[r, j] * rstd[r] * u[j] * a(z[r, j]),
+ *   u[j] = w[j] + weight_offset when weight_offset != 0, else w[j] itself.
+ * act selects a; with RN_ACT_NONE the factor a(z) is absent and z must be
+ * NULL.  x, z: [rows, width] dt, read.  w: [width] fp32, read.
+ * y: [rows, width] dt, written.  rstd: [rows] fp32, written, or NULL.
+ * rstd depends on x, eps and width only: bitwise the same for every
+ * activation and offset.
+ */
+rn_status rmsnorm_fwd(int64_t rows, int32_t width, float eps, float weight_offset,
+                      rn_act act, rn_dtype dt, const void* x, const void* z,
+                      const float* w, void* y, float* rstd, rn_stream stream);
+
+/*
+ * General backward, the gradient of sum(y * dy) for rmsnorm_fwd's y:
+ *   g = u * a(z),  m = mean_j(g_j * dy_j * xh_j),  xh = x * rstd,
+ *   dx = rstd * (g * dy - xh * m),  dz = dy * xh * u * a'(z),
+ *   dw[j] = sum over rows of dy * xh * a(z)   (the offset is a constant).
+ * With RN_ACT_NONE, z and dz must be NULL.  Arguments otherwise as
+ * gated_norm_bwd (workspace: norm_bwd_workspace_bytes).
+ */
+rn_status rmsnorm_bwd(int64_t rows, int32_t width, float eps, float weight_offset,
+                      rn_act act, rn_dtype dt, const void* x, const void* z,
+                      const float* w, const void* dy, const float* rstd, void* dx,
+                      void* dz, float* dw, void* ws, size_t ws_bytes, rn_stream stream);
+
+/*
  * Zero-centred RMSNorm forward (PR #468 Summary, with weight offset 1):
+ * rmsnorm_fwd with weight_offset = 1 and RN_ACT_NONE.
  *   y[r, j] = x[r, j] * rstd[r] * (1 + w[j]).
  * x: [rows, width] dt, read.  w: [width] fp32, read.  y: [rows, width] dt,
  * written.  rstd: [rows] fp32, written, or NULL to skip it.
@@ -102,6 +153,7 @@ rn_status norm_fwd(int64_t rows, int32_t width, float eps, rn_dtype dt,
 
 /*
  * Gated RMSNorm forward (PR #468 Summary, weight offset 0, act = silu):
+ * rmsnorm_fwd with weight_offset = 0 and RN_ACT_SILU.
  *   y[r, j] = x[r, j] * rstd[r] * w[j] * silu(z[r, j]).
  * The offset is never added, so a -0.0 weight keeps its sign.  rstd is
  * bitwise identical to norm_fwd's for the same x (same reduction).

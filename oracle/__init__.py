@@ -12,6 +12,8 @@ from .rmsnorm import (  # noqa: F401
     norm_bwd,
     norm_fwd,
     rmsnorm_bwd,
+    rmsnorm_dx_scale,
+    rmsnorm_dz_scale,
     rmsnorm_fwd,
     rstd,
     sigmoid,

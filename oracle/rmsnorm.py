@@ -233,3 +233,30 @@ def rmsnorm_bwd(x, w, dy, eps: float, weight_offset: float = 1.0, z=None, act: s
     dz = None if act == "none" else dy * xh * u * da
     dw = np.sum(dy * xh * a, axis=0)
     return dx, dz, dw
+
+
+def rmsnorm_dx_scale(x, w, dy, eps: float, weight_offset: float = 1.0, z=None,
+                     act: str = "none") -> np.ndarray:
+    """dx_cancellation_scale for the general operator (g = u * a(z))."""
+    x, dy = _rows(x), _rows(dy)
+    rho = rstd(x, eps)
+    xh = x * rho[:, None]
+    a, _ = _act(None if z is None else _rows(z), act)
+    g = np.broadcast_to(_gain(w, weight_offset)[None, :] * a, x.shape)
+    m_abs = np.sum(np.abs(g * dy * xh), axis=1) / x.shape[1]
+    return np.maximum(np.abs(rho[:, None] * g * dy), np.abs(rho[:, None] * xh * m_abs[:, None]))
+
+
+def rmsnorm_dz_scale(x, w, dy, eps: float, weight_offset: float, z, act: str) -> np.ndarray:
+    """Largest term inside dz = dy*xh*u*s*c(z), c = 1 + z(1-s) (silu) or 1 - s
+    (sigmoid): |dy*xh*u*s| times max(1, |z(1-s)|) for silu and 1 for the
+    sigmoid, whose 1 - s is a difference of terms no larger than 1."""
+    x, z, dy = _rows(x), _rows(z), _rows(dy)
+    rho = rstd(x, eps)
+    s = sigmoid(z)
+    lead = np.abs(dy * x * rho[:, None] * _gain(w, weight_offset)[None, :] * s)
+    if act == "silu":
+        return lead * np.maximum(1.0, np.abs(z * (1.0 - s)))
+    if act == "sigmoid":
+        return lead
+    raise ValueError(f"no dz without a gate (act {act!r})")

@@ -5,8 +5,9 @@ declared in include/rn.h).  This package is its thin binding: ``ops`` has one
 function per C entry point with the same name; ``autograd`` wraps them as
 torch.autograd Functions; ``workloads`` draws seeded synthetic inputs.
 """
-from ._lib import LIB_PATH, DType, RNError, Status, load  # noqa: F401
+from ._lib import LIB_PATH, Act, DType, RNError, Status, load  # noqa: F401
 from .ops import (  # noqa: F401
+    act_code,
     gated_norm_bwd,
     gated_norm_fwd,
     norm_bwd,
@@ -16,5 +17,7 @@ from .ops import (  # noqa: F401
     rn_fold_rows,
     rn_test_set_geometry,
     rn_test_set_validate_only,
+    rmsnorm_bwd,
+    rmsnorm_fwd,
     workspace,
 )

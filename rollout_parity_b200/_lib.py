@@ -26,6 +26,13 @@ class Status(enum.IntEnum):
 class DType(enum.IntEnum):
     F32 = 0
     BF16 = 1
+    F16 = 2
+
+
+class Act(enum.IntEnum):
+    NONE = 0
+    SILU = 1
+    SIGMOID = 2
 
 
 class RNError(RuntimeError):
@@ -38,6 +45,10 @@ class RNError(RuntimeError):
 
 # name -> (restype, argtypes); the same set include/rn.h declares
 SIGNATURES = {
+    "rmsnorm_fwd": (c_i32, [c_i64, c_i32, c_f32, c_f32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp,
+                            c_vp, c_vp]),
+    "rmsnorm_bwd": (c_i32, [c_i64, c_i32, c_f32, c_f32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp,
+                            c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "norm_fwd": (c_i32, [c_i64, c_i32, c_f32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "gated_norm_fwd": (c_i32, [c_i64, c_i32, c_f32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "norm_bwd_workspace_bytes": (c_sz, [c_i64, c_i32]),

@@ -1,0 +1,182 @@
+// Internal declarations shared by librn's translation units: the host part
+// (rn.cu: checks, schedule, dw fold, C ABI) and the row-kernel units
+// (rows_{fwd,bwd}_{bf16,f16,f32}.cu, one per direction and element format, so
+// that they compile in parallel).  Not part of the public interface.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "rn.h"
+
+namespace rn_detail {
+
+constexpr int kLeafRows = 32;       // rows folded in ascending order into one dw leaf
+constexpr int kFoldRG = 8;          // row groups (warps) per fold CTA
+constexpr int64_t kMaxRows = int64_t(1) << 36;
+constexpr int kMaxGrid = 1 << 20;
+
+// Gate activation a(z) (PR #468 Summary, "Activation" bullet); kActNone is
+// the ungated operator.  The values are those of rn_act.
+enum Act { kActNone = RN_ACT_NONE, kActSilu = RN_ACT_SILU, kActSigmoid = RN_ACT_SIGMOID };
+
+// A row of width H is owned by a team of T threads, each holding K 16-byte
+// vectors (vector v = k*T + t).  (T, K) depends on (H, dtype) only.
+struct Sched {
+  int T = 0, K = 0;
+};
+
+struct FwdArgs {
+  int64_t rows;
+  int H, nv;
+  float eps, inv_h;
+  int h_pow2;
+  float woff;       // weight offset; added to w only when nonzero
+  const uint4* x;
+  const uint4* z;
+  const float* w;
+  uint4* y;
+  float* rstd;
+};
+
+struct BwdArgs {
+  int64_t rows;
+  int H, nv;
+  float eps, inv_h;
+  int h_pow2;
+  float woff;
+  const uint4* x;
+  const uint4* z;
+  const float* w;
+  const uint4* dy;
+  const float* rstd;
+  uint4* dx;
+  uint4* dz;
+  float* part;      // [groups][H] fp32 group partials (or dw when one group)
+};
+
+// ---- launch shapes (one formula, used by the kernels' launch bounds and the
+// host's shared-memory sizing) -------------------------------------------------
+__host__ __device__ constexpr int fwd_block_of(int T, int K) {
+  return T <= 16 ? (K <= 2 ? 128 : 64) : (T == 32 ? 128 : T);
+}
+__host__ __device__ constexpr int fwd_min_blocks_of(int T, int K) {
+  return T <= 16 ? (K <= 2 ? 4 : 8) : 1;
+}
+__host__ __device__ constexpr int fwd_stages_of(int T) { return T <= 32 ? 3 : (T <= 512 ? 2 : 1); }
+__host__ __device__ constexpr int bwd_max_block_of(int T) {
+  return T <= 32 ? 8 * T : (T <= 128 ? 256 : T);
+}
+// at width 128 (T = 4): enough resident CTAs for one wave of 1024 (262144 rows:
+// 8192 leaves, 8 per CTA) on 148 SMs, within the register file; at width 2048
+// (T = 128, two leaves per 256-thread CTA) two CTAs per SM
+__host__ __device__ constexpr int bwd_min_blocks_of(int T, int K) {
+  return T <= 4 ? 7 : (T == 8 ? (K <= 2 ? 7 : 4) : ((T == 32 || T == 128) && K <= 2 ? 2 : 1));
+}
+__host__ __device__ constexpr int bwd_stages_of(int T) { return T <= 16 ? 3 : (T <= 512 ? 2 : 1); }
+
+// Where a thread's gain (w, or w + offset) comes from: shared memory
+// (thread-major) for sub-warp teams, registers when K*VE <= 16, else global
+// memory through L1.
+enum GainSrc { kGainSmem = 0, kGainRegs = 1, kGainGlobal = 2 };
+__host__ __device__ constexpr int gain_src_of(int T, int K, int VE) {
+  return T <= 16 ? kGainSmem : (K * VE <= 16 ? kGainRegs : kGainGlobal);
+}
+
+inline int vec_elems(rn_dtype dt) { return dt == RN_F32 ? 4 : 8; }
+inline size_t elem_bytes(rn_dtype dt) { return dt == RN_F32 ? 4 : 2; }
+
+// ---- host helpers defined in rn.cu -------------------------------------------
+int sm_count();
+int grid_cap(int64_t want);
+rn_status launch_status();   // RN_OK, or RN_E_CUDA with the error recorded
+// dynamic shared memory of k_fwd / k_bwd (their layouts)
+size_t fwd_smem_bytes(const Sched& s, bool gated, rn_dtype dt);
+size_t bwd_smem_bytes(const Sched& s, int lpc, int width, bool gated, rn_dtype dt);
+
+// ---- row kernels, one instantiation per element format (rows_*.cu) ------------
+template <int DT>
+rn_status launch_fwd(int act, const Sched& s, const FwdArgs& a, cudaStream_t st);
+template <int DT>
+rn_status launch_bwd(int act, const Sched& s, int lpc, const BwdArgs& a, int64_t groups,
+                     cudaStream_t st);
+
+// Lets `kernel` use `smem` bytes of dynamic shared memory (the default limit is
+// 48 KB) and returns how many of its CTAs fit on one SM.  `done` and `per_sm`
+// cache the answer of the first call for this kernel and size class.
+template <typename Kern>
+int prepare_kernel(Kern kernel, int block, size_t smem, std::atomic<size_t>& done,
+                   std::atomic<int>& per_sm) {
+  if (smem > done.load()) {
+    if (smem > 48 * 1024)
+      (void)cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, block, smem) != cudaSuccess ||
+        nb <= 0) {
+      (void)cudaGetLastError();
+      nb = 1;
+    }
+    per_sm.store(nb);
+    done.store(smem);
+  }
+  return per_sm.load();
+}
+
+// Launches `kern` with programmatic stream serialization: it may be scheduled
+// while the kernel before it in the stream finishes, and waits for it
+// (griddepcontrol.wait) before touching global memory.  If the launch with
+// the attribute is refused it is retried as an ordinary launch.
+template <typename... KArgs, typename... Args>
+rn_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, args...) == cudaSuccess) return launch_status();
+  (void)cudaGetLastError();
+  kern<<<grid, block, smem, st>>>(args...);
+  return launch_status();
+}
+
+// ---- device helpers used by every unit -------------------------------------
+__device__ __forceinline__ float4 add4(const float4& a, const float4& b) {
+  return make_float4(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y), __fadd_rn(a.z, b.z),
+                     __fadd_rn(a.w, b.w));
+}
+
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before its predecessor ends; griddep_wait() blocks
+// until the predecessor grid has completed and its writes are visible (it
+// returns at once for a normal launch).  griddep_trigger() lets the next such
+// kernel be scheduled.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void griddep_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
+// 1/d for d in [1, 2]: the hardware approximation (rcp.approx, within 1 ulp)
+// refined by Newton-Raphson steps written as fused multiply-adds, e = 1 - d*y,
+// y' = y + y*e (Markstein, "Computation of elementary functions on the IBM
+// RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990).  The domain
+// needs no special cases (no zero, infinity, NaN or subnormal).  A GPU test
+// compares it with IEEE division for every float in [1, 2].
+template <int STEPS>
+__device__ __forceinline__ float rcp_1to2(float d) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(d));
+#pragma unroll
+  for (int i = 0; i < STEPS; ++i) y = __fmaf_rn(y, __fmaf_rn(-d, y, 1.0f), y);
+  return y;
+}
+constexpr int kRcpSteps = 1;   // one step is already IEEE-exact on [1, 2]
+
+}  // namespace rn_detail

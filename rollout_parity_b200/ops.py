@@ -13,15 +13,29 @@ from typing import Optional, Tuple
 
 import torch
 
-from ._lib import DType, check, load
+from ._lib import Act, DType, check, load
 
-_DT = {torch.bfloat16: DType.BF16, torch.float32: DType.F32}
+_DT = {torch.bfloat16: DType.BF16, torch.float16: DType.F16, torch.float32: DType.F32}
+# gate activation names; "swish" is another name for silu
+_ACT = {None: Act.NONE, "none": Act.NONE, "silu": Act.SILU, "swish": Act.SILU,
+        "sigmoid": Act.SIGMOID}
 
 
 def _dt(x: torch.Tensor) -> DType:
     if x.dtype not in _DT:
-        raise TypeError(f"x dtype {x.dtype} not supported (bf16 or fp32)")
+        raise TypeError(f"x dtype {x.dtype} not supported (bf16, fp16 or fp32)")
     return _DT[x.dtype]
+
+
+def act_code(act) -> Act:
+    """The C enum for an activation name (None/"none", "silu"/"swish",
+    "sigmoid") or an Act value."""
+    if isinstance(act, Act):
+        return act
+    key = act.lower() if isinstance(act, str) else act
+    if key not in _ACT:
+        raise ValueError(f"unknown activation {act!r} (none, silu, swish or sigmoid)")
+    return _ACT[key]
 
 
 def _mat(name: str, t: Optional[torch.Tensor], like: torch.Tensor) -> torch.Tensor:
@@ -73,6 +87,33 @@ def workspace(rows: int, width: int, device) -> torch.Tensor:
     return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
 
 
+def rmsnorm_fwd(x: torch.Tensor, w: torch.Tensor, eps: float = 1e-6, weight_offset: float = 1.0,
+                z: Optional[torch.Tensor] = None, act=None, *,
+                y: Optional[torch.Tensor] = None, rstd: Optional[torch.Tensor] = None,
+                want_rstd: bool = True, stream=None):
+    """General forward y = x * rstd * (w + weight_offset) * act(z) (the offset
+    is added only when nonzero; act None means no gate and no z).  Returns
+    (y, rstd)."""
+    rows, width = _rows_width(x)
+    a = act_code(act)
+    if a == Act.NONE:
+        if z is not None:
+            raise ValueError("z given without a gate activation")
+    else:
+        _mat("z", z, x)
+    _vec("w", w, width, x.device)
+    y = torch.empty_like(x) if y is None else _mat("y", y, x)
+    if rstd is None and want_rstd:
+        rstd = torch.empty(rows, dtype=torch.float32, device=x.device)
+    if rstd is not None:
+        _vec("rstd", rstd, rows, x.device)
+    with torch.cuda.device(x.device):
+        check("rmsnorm_fwd",
+              load().rmsnorm_fwd(rows, width, eps, weight_offset, int(a), _dt(x), _ptr(x), _ptr(z),
+                                 _ptr(w), _ptr(y), _ptr(rstd), _stream(x, stream)))
+    return y, rstd
+
+
 def norm_fwd(x: torch.Tensor, w: torch.Tensor, eps: float = 1e-6, *,
              y: Optional[torch.Tensor] = None, rstd: Optional[torch.Tensor] = None,
              want_rstd: bool = True, stream=None):
@@ -116,6 +157,38 @@ def _ws(rows, width, device, ws):
     if ws.device != device or not ws.is_contiguous():
         raise ValueError("ws must be a contiguous buffer on the tensors' device")
     return ws, ws.numel() * ws.element_size()
+
+
+def rmsnorm_bwd(x: torch.Tensor, w: torch.Tensor, dy: torch.Tensor,
+                rstd: Optional[torch.Tensor] = None, eps: float = 1e-6, weight_offset: float = 1.0,
+                z: Optional[torch.Tensor] = None, act=None, *,
+                dx: Optional[torch.Tensor] = None, dz: Optional[torch.Tensor] = None,
+                dw: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                stream=None):
+    """General backward.  Returns (dx, dz, dw); dz is None without a gate.
+    rstd=None recomputes it."""
+    rows, width = _rows_width(x)
+    a = act_code(act)
+    if a == Act.NONE:
+        if z is not None or dz is not None:
+            raise ValueError("z or dz given without a gate activation")
+    else:
+        _mat("z", z, x)
+        dz = torch.empty_like(x) if dz is None else _mat("dz", dz, x)
+    _vec("w", w, width, x.device)
+    _mat("dy", dy, x)
+    if rstd is not None:
+        _vec("rstd", rstd, rows, x.device)
+    dx = torch.empty_like(x) if dx is None else _mat("dx", dx, x)
+    dw = torch.empty(width, dtype=torch.float32, device=x.device) if dw is None else \
+        _vec("dw", dw, width, x.device)
+    ws, nws = _ws(rows, width, x.device, ws)
+    with torch.cuda.device(x.device):
+        check("rmsnorm_bwd",
+              load().rmsnorm_bwd(rows, width, eps, weight_offset, int(a), _dt(x), _ptr(x), _ptr(z),
+                                 _ptr(w), _ptr(dy), _ptr(rstd), _ptr(dx), _ptr(dz), _ptr(dw),
+                                 _ptr(ws), nws, _stream(x, stream)))
+    return dx, dz, dw
 
 
 def norm_bwd(x: torch.Tensor, w: torch.Tensor, dy: torch.Tensor,

@@ -29,7 +29,10 @@ from typing import List, Optional
 import numpy as np
 import torch
 
-DTYPES = {"bf16": torch.bfloat16, "f32": torch.float32}
+DTYPES = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}
+# the operator's (activation, weight offset) by op name; "general" takes both
+# from the caller
+OP_DEFAULTS = {"norm": ("none", 1.0), "gated": ("silu", 0.0)}
 
 # child-stream ids of SeedSequence(seed).spawn(...)
 _X, _Z, _DY, _W, _OUTLIER, _PACK = range(6)
@@ -40,21 +43,31 @@ class Workload:
     """One batch of synthetic inputs (host tensors, stored dtype)."""
 
     name: str
-    op: str                     # "norm" (zero-centred) or "gated"
+    op: str                     # "norm" (zero-centred), "gated" or "general"
     rows: int
     width: int
-    dtype: str                  # "bf16" or "f32"
+    dtype: str                  # "bf16", "f16" or "f32"
     eps: float
     x: torch.Tensor             # [rows, width], stored dtype, CPU
-    z: Optional[torch.Tensor]   # gated only
+    z: Optional[torch.Tensor]   # present when there is a gate
     dy: torch.Tensor            # upstream gradient, stored dtype
     w: torch.Tensor             # [width] fp32
     seq_lens: Optional[List[int]] = None
     outlier_channels: Optional[List[int]] = None
+    act: Optional[str] = None   # gate activation: "none", "silu" or "sigmoid"
+    weight_offset: Optional[float] = None   # added to w when nonzero
+
+    def __post_init__(self):
+        # "norm" and "gated" fix both; "general" must name them
+        if self.op in OP_DEFAULTS:
+            act, off = OP_DEFAULTS[self.op]
+            self.act = act if self.act is None else self.act
+            self.weight_offset = off if self.weight_offset is None else self.weight_offset
+        assert self.act in ("none", "silu", "sigmoid") and self.weight_offset is not None
 
     @property
     def gated(self) -> bool:
-        return self.op == "gated"
+        return self.act != "none"
 
     def to(self, device) -> "Workload":
         f = lambda t: None if t is None else t.to(device)
@@ -76,12 +89,19 @@ def _store(a: np.ndarray, dtype: str) -> torch.Tensor:
 def make(op: str, rows: int, width: int, dtype: str = "bf16", *, seed: int = 0,
          eps: float = 1e-6, w_mean: float = 1.0, w_std: float = 0.1,
          outlier_frac: float = 0.0, outlier_scale: float = 50.0,
-         outlier_round: str = "nearest", name: str = "") -> Workload:
-    """Draw one workload.  ``op`` is "norm" or "gated"."""
-    assert op in ("norm", "gated") and dtype in DTYPES
+         outlier_round: str = "nearest", name: str = "", act: Optional[str] = None,
+         weight_offset: Optional[float] = None) -> Workload:
+    """Draw one workload.  ``op`` is "norm" (no gate, offset 1), "gated" (silu,
+    offset 0) or "general" (``act`` and ``weight_offset`` given)."""
+    assert op in ("norm", "gated", "general") and dtype in DTYPES
+    if op == "general":
+        assert act in ("none", "silu", "sigmoid") and weight_offset is not None
+    else:
+        assert act is None and weight_offset is None
+        act, weight_offset = OP_DEFAULTS[op]
     rx, rz, rdy, rw, ro, _ = _streams(seed)
     x = _normal(rx, (rows, width))
-    z = _normal(rz, (rows, width)) if op == "gated" else None
+    z = _normal(rz, (rows, width)) if act != "none" else None
     dy = _normal(rdy, (rows, width))
     w = (np.float32(w_mean) + np.float32(w_std) * _normal(rw, (width,))).astype(np.float32)
     chans = None
@@ -96,7 +116,8 @@ def make(op: str, rows: int, width: int, dtype: str = "bf16", *, seed: int = 0,
     return Workload(name=name or f"{op}_{rows}x{width}_{dtype}", op=op, rows=rows,
                     width=width, dtype=dtype, eps=eps, x=_store(x, dtype),
                     z=None if z is None else _store(z, dtype), dy=_store(dy, dtype),
-                    w=torch.from_numpy(w), outlier_channels=chans)
+                    w=torch.from_numpy(w), outlier_channels=chans, act=act,
+                    weight_offset=float(weight_offset))
 
 
 def ragged_lengths(total_rows: int, max_len: int, seed: int = 0) -> List[int]:
@@ -156,8 +177,45 @@ CONFIGS = {
 SWEEP_8192 = (1, 7, 128, 4096, 32768)
 
 
+# Variants of the operator (PR #468 Summary: activation silu or sigmoid, weight
+# offset 0 or 1, fp32/fp16/bf16, H in {128, 2048, 5120}) at benchmark sizes.
+def cfg_sigmoid_heads(seed: int = 0) -> Workload:
+    """The 262144 x 128 bf16 head layout with outliers, sigmoid gate, offset 0."""
+    return make("general", 262144, 128, "bf16", seed=seed, outlier_frac=0.01,
+                outlier_scale=50.0, act="sigmoid", weight_offset=0.0,
+                name="sigmoid_262144x128_bf16_outliers")
+
+
+def cfg_f16_heads(seed: int = 0) -> Workload:
+    """The 262144 x 128 head layout with outliers in fp16, silu gate, offset 0."""
+    return make("general", 262144, 128, "f16", seed=seed, outlier_frac=0.01,
+                outlier_scale=50.0, act="silu", weight_offset=0.0,
+                name="silu_262144x128_f16_outliers")
+
+
+def cfg_norm_5120(seed: int = 0) -> Workload:
+    """Zero-centred (offset 1, no gate), 16384 x 5120 bf16, w ~ N(0, 0.1)."""
+    return make("general", 16384, 5120, "bf16", seed=seed, w_mean=0.0, w_std=0.1,
+                act="none", weight_offset=1.0, name="norm_16384x5120_bf16")
+
+
+def cfg_sigmoid_f32_2048(seed: int = 0) -> Workload:
+    """Sigmoid gate with offset 1, 16384 x 2048 fp32, w ~ N(0, 0.1)."""
+    return make("general", 16384, 2048, "f32", seed=seed, w_mean=0.0, w_std=0.1,
+                act="sigmoid", weight_offset=1.0, name="sigmoid_off1_16384x2048_f32")
+
+
+VARIANTS = {
+    "sigmoid_262144x128_bf16_outliers": cfg_sigmoid_heads,
+    "silu_262144x128_f16_outliers": cfg_f16_heads,
+    "norm_16384x5120_bf16": cfg_norm_5120,
+    "sigmoid_off1_16384x2048_f32": cfg_sigmoid_f32_2048,
+}
+ALL = {**CONFIGS, **VARIANTS}
+
+
 def as_f64(t: Optional[torch.Tensor]) -> Optional[np.ndarray]:
-    """Widen stored values to fp64 exactly (bf16 and fp32 embed in fp64)."""
+    """Widen stored values to fp64 exactly (bf16, fp16 and fp32 embed in fp64)."""
     if t is None:
         return None
     return t.detach().to("cpu").to(torch.float64).numpy()

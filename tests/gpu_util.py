@@ -12,9 +12,21 @@ from rollout_parity_b200 import workloads
 f64 = workloads.as_f64
 
 
+def is_general(wl) -> bool:
+    """True for op "general": its activation and offset are given explicitly,
+    so it runs through rmsnorm_fwd / rmsnorm_bwd."""
+    return wl.op == "general"
+
+
 def run(rn, wl, rstd_in_bwd=True):
-    """Forward then backward through the C ABI; returns a dict of outputs."""
-    if wl.gated:
+    """Forward then backward through the C ABI; returns a dict of outputs.
+    op "norm" / "gated" use their own entry points, op "general" rmsnorm_fwd /
+    rmsnorm_bwd."""
+    if is_general(wl):
+        y, rstd = rn.rmsnorm_fwd(wl.x, wl.w, wl.eps, wl.weight_offset, wl.z, wl.act)
+        dx, dz, dw = rn.rmsnorm_bwd(wl.x, wl.w, wl.dy, rstd if rstd_in_bwd else None, wl.eps,
+                                    wl.weight_offset, wl.z, wl.act)
+    elif wl.gated:
         y, rstd = rn.gated_norm_fwd(wl.x, wl.z, wl.w, wl.eps)
         dx, dz, dw = rn.gated_norm_bwd(wl.x, wl.z, wl.w, wl.dy, rstd if rstd_in_bwd else None,
                                        wl.eps)
@@ -31,7 +43,14 @@ def oracle_rows(wl, idx=None):
     sel = (lambda t: f64(t)) if idx is None else (lambda t: f64(t[idx]))
     x, dy = sel(wl.x), sel(wl.dy)
     w = f64(wl.w)
-    if wl.gated:
+    if is_general(wl):
+        z = None if wl.z is None else sel(wl.z)
+        o, a = wl.weight_offset, wl.act
+        y, r = oracle.rmsnorm_fwd(x, w, wl.eps, o, z, a)
+        dx, dz, _ = oracle.rmsnorm_bwd(x, w, dy, wl.eps, o, z, a)
+        sdx = oracle.rmsnorm_dx_scale(x, w, dy, wl.eps, o, z, a)
+        sdz = None if z is None else oracle.rmsnorm_dz_scale(x, w, dy, wl.eps, o, z, a)
+    elif wl.gated:
         z = sel(wl.z)
         y, r = oracle.gated_norm_fwd(x, z, w, wl.eps)
         dx, dz, _ = oracle.gated_norm_bwd(x, z, w, dy, wl.eps)
@@ -52,7 +71,10 @@ def oracle_dw(wl, chunk=4096):
     for s in range(0, wl.rows, chunk):
         e = min(wl.rows, s + chunk)
         x, dy = f64(wl.x[s:e]), f64(wl.dy[s:e])
-        if wl.gated:
+        if is_general(wl):
+            z = None if wl.z is None else f64(wl.z[s:e])
+            _, _, dw = oracle.rmsnorm_bwd(x, w, dy, wl.eps, wl.weight_offset, z, wl.act)
+        elif wl.gated:
             _, _, dw = oracle.gated_norm_bwd(x, f64(wl.z[s:e]), w, dy, wl.eps)
         else:
             _, dw = oracle.norm_bwd(x, w, dy, wl.eps)

@@ -1,9 +1,9 @@
-"""Comparison helpers for the parity tests: exact fp64 -> bf16 rounding, bf16 ulp,
-and the tolerance rules.  No norm arithmetic lives here.
+"""Comparison helpers for the parity tests: exact fp64 -> bf16 / fp16 rounding,
+their ulps, and the tolerance rules.  No norm arithmetic lives here.
 
 Tolerances (the operators' contract asks for fp32 accumulation and bf16 outputs;
 the bar is 2 bf16 ulp per bf16 element and relative L2 <= 1e-4 for fp32 tensors):
-  * bf16 y:        |gpu - ref| <= 2 ulp_bf16(|ref|)
+  * bf16 y:        |gpu - ref| <= 2 ulp_bf16(|ref|)   (fp16: the same in fp16 ulps)
   * bf16 dx, dz:   |gpu - ref| <= 2 ulp_bf16(|ref|) + 2**-16 * T
     where T is the size of the largest term that cancels in that element
     (the oracle's cancellation scale; for dx's mean term it is built from the
@@ -17,55 +17,74 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-BF16_MIN_EXP = -133          # bf16 subnormal spacing is 2**-133
-BF16_MAX = float.fromhex("0x1.fep127")
+# 16-bit formats: (significant bits, exponent of the subnormal spacing, largest finite)
+BF16 = (8, -133, float.fromhex("0x1.fep127"))
+F16 = (11, -24, 65504.0)
+BF16_MIN_EXP = BF16[1]       # bf16 subnormal spacing is 2**-133
+BF16_MAX = BF16[2]
 
 
-def bf16_round(a) -> np.ndarray:
-    """Round fp64 values to the nearest bf16 value, ties to even, in one step
-    (no intermediate fp32 rounding).  Returns fp64 holding bf16 values."""
+def round16(a, fmt) -> np.ndarray:
+    """Round fp64 values to the nearest value of the 16-bit format ``fmt``
+    (BF16 or F16), ties to even, in one step (no intermediate fp32 rounding);
+    past the largest finite value, to infinity.  Returns fp64."""
+    p, min_exp, vmax = fmt
     a = np.asarray(a, dtype=np.float64)
     out = np.zeros_like(a)
     nz = (a != 0) & np.isfinite(a)
     _, e = np.frexp(a[nz])                       # a = m * 2**e, 0.5 <= |m| < 1
-    step_exp = np.maximum(e - 8, BF16_MIN_EXP)   # 8 significant bits
-    step = np.ldexp(1.0, step_exp)
+    step = np.ldexp(1.0, np.maximum(e - p, min_exp))
     q = np.rint(a[nz] / step) * step             # exact scaling; rint is ties-to-even
-    q = np.where(np.abs(q) > BF16_MAX, np.copysign(np.inf, q), q)
+    q = np.where(np.abs(q) > vmax, np.copysign(np.inf, q), q)
     out[nz] = q
     out[~np.isfinite(a)] = a[~np.isfinite(a)]
     out[a == 0] = a[a == 0]
     return out
 
 
-def bf16_ulp(a) -> np.ndarray:
-    """Spacing of bf16 values at |a| (the subnormal spacing below 2**-126)."""
+def ulp16(a, fmt) -> np.ndarray:
+    """Spacing of the 16-bit format's values at |a| (the subnormal spacing at
+    the bottom)."""
+    p, min_exp, _ = fmt
     a = np.abs(np.asarray(a, dtype=np.float64))
     _, e = np.frexp(np.where(a == 0, 1e-300, a))
-    return np.ldexp(1.0, np.maximum(e - 8, BF16_MIN_EXP))
+    return np.ldexp(1.0, np.maximum(e - p, min_exp))
+
+
+def bf16_round(a) -> np.ndarray:
+    return round16(a, BF16)
+
+
+def bf16_ulp(a) -> np.ndarray:
+    return ulp16(a, BF16)
+
+
+FMT_OF = {torch.bfloat16: BF16, torch.float16: F16}
 
 
 def to64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").to(torch.float64).numpy()
 
 
-def check_bf16(got: torch.Tensor, ref: np.ndarray, scale=None, what="", ulps=2.0,
-               floor=2.0 ** -16) -> dict:
-    """Assert the bf16 tolerance; return pass statistics."""
+def check_16(got: torch.Tensor, ref: np.ndarray, scale=None, what="", ulps=2.0,
+             floor=2.0 ** -16) -> dict:
+    """Assert the 16-bit (bf16 or fp16) tolerance; return pass statistics."""
+    fmt = FMT_OF[got.dtype]
+    ulp = lambda v: ulp16(v, fmt)
     g = to64(got)
     ref = np.asarray(ref, dtype=np.float64)
     assert g.shape == ref.shape, (what, g.shape, ref.shape)
     assert np.all(np.isfinite(g)), f"{what}: non-finite output"
     err = np.abs(g - ref)
-    lim_plain = ulps * bf16_ulp(ref)
+    lim_plain = ulps * ulp(ref)
     lim = lim_plain if scale is None else lim_plain + floor * np.asarray(scale)
     bad = err > lim
     stats = {
         "n": int(g.size),
-        "max_err_ulps": float(np.max(err / bf16_ulp(ref))) if g.size else 0.0,
+        "max_err_ulps": float(np.max(err / ulp(ref))) if g.size else 0.0,
         "plain_2ulp_pass_frac": float(np.mean(err <= lim_plain)) if g.size else 1.0,
         "floor_hits": int(np.sum((err > lim_plain) & ~bad)),
-        "correctly_rounded_frac": float(np.mean(g == bf16_round(ref))) if g.size else 1.0,
+        "correctly_rounded_frac": float(np.mean(g == round16(ref, fmt))) if g.size else 1.0,
     }
     if np.any(bad):
         i = np.unravel_index(np.argmax(err - lim), err.shape)
@@ -90,6 +109,6 @@ def check_f32(got: torch.Tensor, ref: np.ndarray, what="", rel_l2=1e-4) -> dict:
 
 
 def check_out(got: torch.Tensor, ref: np.ndarray, scale=None, what="") -> dict:
-    if got.dtype == torch.bfloat16:
-        return check_bf16(got, ref, scale=scale, what=what)
+    if got.dtype in FMT_OF:
+        return check_16(got, ref, scale=scale, what=what)
     return check_f32(got, ref, what=what)

@@ -11,7 +11,7 @@ import pytest
 
 import rollout_parity_b200 as rn
 from rollout_parity_b200 import build as rn_build
-from rollout_parity_b200._lib import SIGNATURES, DType, Status
+from rollout_parity_b200._lib import SIGNATURES, Act, DType, Status
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "rn.h")
@@ -165,7 +165,8 @@ GBWD_CASES = [
     ("rows 0 only needs dw", dict(rows=0, x=0, z=0, dy=0, dx=0, dz=0, ws=0, rstd=0), Status.OK),
     ("rows 0 still needs dw", dict(rows=0, dw=0), Status.E_ARG),
     ("width", dict(width=20), Status.E_WIDTH),
-    ("dtype", dict(dt=2), Status.E_DTYPE),
+    ("dtype", dict(dt=7), Status.E_DTYPE),
+    ("fp16", dict(dt=DType.F16), Status.OK),
 ]
 
 
@@ -191,6 +192,68 @@ def test_norm_bwd_checks(lib, name, kw, want):
         assert bwd(lib, **kw) == want
 
 
+def rfwd(lib, rows=R, width=H, eps=1e-6, woff=1.0, act=Act.SIGMOID, dt=DType.BF16, **kw):
+    ptr = dict(x=P(X), z=P(Z), w=P(W), y=P(Y), rstd=P(RS))
+    ptr.update(kw)
+    return lib.rmsnorm_fwd(rows, width, eps, woff, act, dt, ptr["x"], ptr["z"], ptr["w"],
+                           ptr["y"], ptr["rstd"], None)
+
+
+def rbwd(lib, rows=R, width=H, eps=1e-6, woff=1.0, act=Act.SIGMOID, dt=DType.BF16, **kw):
+    ptr = dict(x=P(X), z=P(Z), w=P(W), dy=P(DY), rstd=P(RS), dx=P(DX), dz=P(DZ), dw=P(DW),
+               ws=P(WS))
+    ptr.update(kw)
+    nws = lib.norm_bwd_workspace_bytes(rows, width)
+    return lib.rmsnorm_bwd(rows, width, eps, woff, act, dt, ptr["x"], ptr["z"], ptr["w"],
+                           ptr["dy"], ptr["rstd"], ptr["dx"], ptr["dz"], ptr["dw"], ptr["ws"],
+                           nws, None)
+
+
+GENERAL_CASES = [
+    ("sigmoid offset 1", {}, Status.OK),
+    ("silu offset 0", dict(act=Act.SILU, woff=0.0), Status.OK),
+    ("offset -0.0", dict(woff=-0.0), Status.OK),
+    ("offset 2.5", dict(woff=2.5), Status.OK),
+    ("fp16", dict(dt=DType.F16), Status.OK),
+    ("fp32", dict(dt=DType.F32), Status.OK),
+    ("no gate, z NULL", dict(act=Act.NONE, z=0, dz=0), Status.OK),
+    ("no gate but z given", dict(act=Act.NONE, dz=0), Status.E_ARG),
+    ("gate without z", dict(z=0), Status.E_ARG),
+    ("activation 3", dict(act=3), Status.E_ARG),
+    ("activation -1", dict(act=-1), Status.E_ARG),
+    ("offset nan", dict(woff=float("nan")), Status.E_ARG),
+    ("offset inf", dict(woff=float("inf")), Status.E_ARG),
+    ("dtype 3", dict(dt=3), Status.E_DTYPE),
+    ("y aliases z", dict(y=P(Z), dx=P(Z)), Status.E_ARG),
+    ("rows 0", dict(rows=0, x=0, z=0, y=0, dy=0, dx=0, dz=0, ws=0, rstd=0), Status.OK),
+]
+
+
+@pytest.mark.parametrize("name,kw,want", GENERAL_CASES, ids=[c[0] for c in GENERAL_CASES])
+def test_general_entry_checks(lib, name, kw, want):
+    fk = {k: v for k, v in kw.items() if k in ("rows", "width", "eps", "woff", "act", "dt", "x",
+                                               "z", "w", "y", "rstd")}
+    bk = {k: v for k, v in kw.items() if k not in ("y",)}
+    with validate_only(lib):
+        assert rfwd(lib, **fk) == want
+        if name != "no gate but z given" or "dz" in kw:
+            assert rbwd(lib, **bk) == want
+
+
+def test_general_backward_rejects_dz_without_gate(lib):
+    with validate_only(lib):
+        assert rbwd(lib, act=Act.NONE, z=0) == Status.E_ARG          # dz given
+        assert rbwd(lib, act=Act.NONE, z=0, dz=0) == Status.OK
+
+
+def test_binding_activation_names():
+    assert rn.act_code(None) == Act.NONE and rn.act_code("none") == Act.NONE
+    assert rn.act_code("silu") == Act.SILU and rn.act_code("swish") == Act.SILU
+    assert rn.act_code("SiLU") == Act.SILU and rn.act_code("sigmoid") == Act.SIGMOID
+    with pytest.raises(ValueError):
+        rn.act_code("gelu")
+
+
 @pytest.mark.parametrize("rows", [1, 31, 32, 33, 256, 257, 4096, 262144, 1 << 30])
 @pytest.mark.parametrize("width", [8, 128, 2048, 8192, 16384])
 def test_workspace_bytes(lib, rows, width):
@@ -207,7 +270,8 @@ def test_workspace_bytes_invalid(lib):
 @pytest.mark.parametrize("width,dt,team", [(128, DType.BF16, 4), (128, DType.F32, 8),
                                            (8, DType.BF16, 1), (2048, DType.BF16, 128),
                                            (8192, DType.BF16, 512), (5120, DType.BF16, 512),
-                                           (16384, DType.F32, 1024)])
+                                           (16384, DType.F32, 1024), (128, DType.F16, 4),
+                                           (5120, DType.F16, 512), (2048, DType.F16, 128)])
 def test_describe(lib, width, dt, team):
     d = lib.rn_describe(width, dt).decode()
     assert f"team_threads={team} " in d

@@ -9,6 +9,8 @@ every row, a batch-size sweep; and its prefix-slice and dweight batch tests in
 "Summary") are the model; the sub-batch sweep visits every start position
 (the review finding on the stride at sub-batch size 1).
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -25,13 +27,12 @@ ROW_KEYS = ("y", "rstd", "dx", "dz")
 def sub(wl, s, e):
     """The rows [s, e) as a workload of their own (fresh contiguous copies)."""
     c = lambda t: None if t is None else t[s:e].clone()
-    return workloads.Workload(name=wl.name, op=wl.op, rows=e - s, width=wl.width,
-                              dtype=wl.dtype, eps=wl.eps, x=c(wl.x), z=c(wl.z), dy=c(wl.dy),
-                              w=wl.w)
+    return dataclasses.replace(wl, rows=e - s, x=c(wl.x), z=c(wl.z), dy=c(wl.dy),
+                               seq_lens=None)
 
 
 def bits(t):
-    return t.view(torch.int16 if t.dtype == torch.bfloat16 else torch.int32)
+    return t.view(torch.int32 if t.dtype == torch.float32 else torch.int16)
 
 
 def assert_rows_equal(full, part, s, e, what=""):

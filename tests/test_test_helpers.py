@@ -4,7 +4,7 @@ import pytest
 import torch
 
 import fold_model as fm
-from numerics import bf16_round, bf16_ulp
+from numerics import F16, bf16_round, bf16_ulp, round16, ulp16
 
 
 def test_bf16_round_matches_torch_on_fp32_values():
@@ -97,3 +97,21 @@ def test_dw_tree_leaf_is_left_fold():
     c2[0] = big; c2[1] = 1.0; c2[32] = 1.0
     # leaf0 = big+1 -> big (ties to even), leaf1 = 1; big + 1 -> big
     assert fm.dw_tree(c2)[0] == big
+
+
+def test_f16_round_matches_torch_on_fp32_values():
+    rng = np.random.default_rng(3)
+    a = np.concatenate([rng.standard_normal(20000).astype(np.float32) * s
+                        for s in (1e-7, 1e-5, 1e-2, 1.0, 300.0, 6e4)])
+    want = torch.from_numpy(a).to(torch.float16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(round16(a.astype(np.float64), F16), want)
+
+
+def test_f16_ulp_and_range():
+    assert ulp16(1.0, F16) == 2.0 ** -10
+    assert ulp16(0.0, F16) == 2.0 ** -24 and ulp16(1e-7, F16) == 2.0 ** -24
+    assert round16(65504.0, F16) == 65504.0
+    assert round16(65519.0, F16) == 65504.0
+    assert np.isinf(round16(65520.0, F16))            # the tie rounds to even: 2**16
+    assert round16(2.0 ** -25, F16) == 0.0            # tie between 0 and 2**-24 -> even (0)
+    assert round16(3 * 2.0 ** -25, F16) == 2.0 ** -23
