@@ -415,6 +415,18 @@ size_t bwd_smem_bytes(const Sched& s, int lpc, int width, bool gated, rn_dtype d
   return red + gain + stages + leaves + size_t(bwd_stages_of(s.T)) * bd * sizeof(float);
 }
 
+// Dynamic shared memory of k_bwd_stripe: gain, staged rows, staged rstd, the
+// transpose buffer (the kernel's layout).
+size_t bwd_stripe_smem_bytes(const Sched& s, int width, bool gated, rn_dtype dt) {
+  const size_t VE = size_t(vec_elems(dt));
+  const size_t S = size_t(bwd_stages_of(s.T));
+  const size_t gain = size_t(s.K) * s.T * VE * sizeof(float);
+  const size_t stages = S * (gated ? 3 : 2) * s.K * 32 * 16;
+  const size_t rstd = S * 32 * sizeof(float);
+  const size_t tbuf = size_t(32 / s.T) * size_t(width + 4) * sizeof(float);
+  return gain + stages + rstd + tbuf;
+}
+
 // Dynamic shared memory of k_fwd (the kernel's layout).
 size_t fwd_smem_bytes(const Sched& s, bool gated, rn_dtype dt) {
   const size_t VE = size_t(vec_elems(dt));
@@ -493,13 +505,15 @@ const char* rn_describe(int32_t width, rn_dtype dt) {
   Sched s;
   if (!pick_sched(width, dt, &s)) return "unsupported";
   const int lpc = leaves_per_cta(s, width, dt);
+  const bool stripe = stripe_shape(s.T, s.K, vec_elems(dt), width / vec_elems(dt) == s.T * s.K);
   std::snprintf(t_describe, sizeof t_describe,
-                "backend=cuda-sm100a lib=librn kernels=k_fwd,k_bwd,k_fold dtype=%s width=%d "
+                "backend=cuda-sm100a lib=librn kernels=k_fwd,%s,k_fold dtype=%s width=%d "
                 "acc=fp32 team_threads=%d vectors_per_thread=%d elems_per_vector=%d "
                 "thread_order=ascending-fma-from-neg0 lane_join=xor-butterfly(%d..1) "
                 "warp_join=%s dw_tree=leaf32-ascending-fold+level-pairwise "
                 "leaves_per_cta=%d fast_math=off atomics=none",
-                dtype_name(dt), width, s.T, s.K, vec_elems(dt), (s.T < 32 ? s.T : 32) / 2,
+                stripe ? "k_bwd_stripe" : "k_bwd", dtype_name(dt), width, s.T, s.K, vec_elems(dt),
+                (s.T < 32 ? s.T : 32) / 2,
                 s.T > 32 ? "smem-pairwise" : "none", lpc);
   return t_describe;
 }

@@ -85,6 +85,12 @@ __host__ __device__ constexpr int gain_src_of(int T, int K, int VE) {
   return T <= 16 ? kGainSmem : (K * VE <= 16 ? kGainRegs : kGainGlobal);
 }
 
+// Narrow rows that the backward runs with k_bwd_stripe: teams of at most 8
+// threads, every vector slot used, H a multiple of 128.
+__host__ __device__ constexpr bool stripe_shape(int T, int K, int VE, bool exact) {
+  return exact && T <= 8 && (T * K * VE) % 128 == 0;
+}
+
 inline int vec_elems(rn_dtype dt) { return dt == RN_F32 ? 4 : 8; }
 inline size_t elem_bytes(rn_dtype dt) { return dt == RN_F32 ? 4 : 2; }
 
@@ -95,6 +101,7 @@ rn_status launch_status();   // RN_OK, or RN_E_CUDA with the error recorded
 // dynamic shared memory of k_fwd / k_bwd (their layouts)
 size_t fwd_smem_bytes(const Sched& s, bool gated, rn_dtype dt);
 size_t bwd_smem_bytes(const Sched& s, int lpc, int width, bool gated, rn_dtype dt);
+size_t bwd_stripe_smem_bytes(const Sched& s, int width, bool gated, rn_dtype dt);
 
 // ---- row kernels, one instantiation per element format (rows_*.cu) ------------
 template <int DT>
@@ -162,6 +169,43 @@ __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wa
 __device__ __forceinline__ void griddep_trigger() {
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 }
+
+// The level-by-level pairwise tree (node 2i + node 2i+1 at each level, an odd
+// last node carried up) over up to B = 2^LB items that arrive in order, kept
+// as a binary counter: slot k holds a pending perfect subtree of 2^k items.
+// push(i, v) adds item i; finish(n) returns the root over the n items pushed
+// (n <= B): the pending subtrees joined smallest (rightmost) first, which is
+// where the level-by-level tree puts them.  V is float4 or float.
+__device__ __forceinline__ float tree_add(float a, float b) { return __fadd_rn(a, b); }
+__device__ __forceinline__ float4 tree_add(const float4& a, const float4& b) { return add4(a, b); }
+template <int LB, typename V>
+struct TreeCounter {
+  V slot[LB + 1];
+  __device__ __forceinline__ void push(int i, V cur) {
+#pragma unroll
+    for (int k = 0; k <= LB; ++k) {
+      if ((i >> k) & 1) {
+        cur = tree_add(slot[k], cur);
+      } else {
+        slot[k] = cur;
+        break;
+      }
+    }
+  }
+  __device__ __forceinline__ V finish(int n) const {
+    if (n == (1 << LB)) return slot[LB];
+    V res = slot[0];
+    bool have = false;
+#pragma unroll
+    for (int k = 0; k < LB; ++k) {
+      if ((n >> k) & 1) {
+        res = have ? tree_add(slot[k], res) : slot[k];
+        have = true;
+      }
+    }
+    return res;
+  }
+};
 
 // 1/d for d in [1, 2]: the hardware approximation (rcp.approx, within 1 ulp)
 // refined by Newton-Raphson steps written as fused multiply-adds, e = 1 - d*y,

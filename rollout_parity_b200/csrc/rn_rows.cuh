@@ -517,6 +517,88 @@ k_fwd(const FwdArgs a) {
   cp_async_wait<0>();
 }
 
+// One row of the backward for this thread's K vectors: rstd (staged, or
+// recomputed exactly as the forward does), pass 1 (xh, g*dy, s and the
+// per-vector dot partials), the team's dot product, pass 2 (dx and dz
+// stores).  d receives the row's dw contributions dy*xh*a(z) of this thread's
+// elements (meaningful only when act).  For T > 32 every team of the CTA must
+// call it in lockstep.
+//   g = u * a(z);  m = mean(g * dy * xh);  dx = rstd * (g*dy - xh*m)
+//   dz = dy * xh * u * a'(z)
+template <int DT, int T, int K, int ACT, bool EXACT, typename G>
+__device__ __forceinline__ void bwd_row(const BwdArgs& a, const G& gain, const uint4 (&xr)[K],
+                                        const uint4 (&dr)[K], const uint4 (&zr)[K],
+                                        float rs_staged, bool have_rstd, int64_t row, bool act,
+                                        int t, float* red, int& phase, int team, int NT,
+                                        unsigned mask, float2 (&d)[K][Fmt<DT>::VE / 2]) {
+  using F = Fmt<DT>;
+  constexpr bool GATED = ACT != kActNone;
+  constexpr int VE = F::VE;
+  const int nv = a.nv;
+  float rs = rs_staged;
+  if (!have_rstd) {   // uniform branch
+    float ss[1] = {thread_sumsq<DT, T, K, EXACT>(xr, nv, t)};
+    team_sum<T, 1>(ss, red, phase, team, NT, mask);
+    rs = rsqrtf(__fadd_rn(mean_of(ss[0], a.H, a.inv_h, a.h_pow2), a.eps));
+  }
+  // pass 1: keep xh, g*dy and s for pass 2 (element pairs)
+  const float2 rs2 = bc2(rs);
+  float2 xh[K][VE / 2], gd[K][VE / 2], sg[K][GATED ? VE / 2 : 1];
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    float2 xf[VE / 2], df[VE / 2], zf[VE / 2], gk[VE / 2];
+    F::unpack2(xr[k], xf);
+    F::unpack2(dr[k], df);
+    if constexpr (GATED) F::unpack2(zr[k], zf);
+    gain.get2(k, gk);
+#pragma unroll
+    for (int q = 0; q < VE / 2; ++q) {
+      xh[k][q] = mul2(xf[q], rs2);
+      float2 g;
+      if constexpr (GATED) {
+        sg[k][q] = sigmoid2(zf[q]);
+        g = mul2(gk[q], gate2<ACT>(zf[q], sg[k][q]));   // u * a(z)
+      } else {
+        g = gk[q];                                      // u
+      }
+      gd[k][q] = mul2(g, df[q]);
+    }
+  }
+  float dp[K];   // per-vector dot partials, joined by the pairwise tree
+  vector_dots<VE, T, K, EXACT>(gd, xh, nv, t, dp);
+  float dot[1] = {pairwise_tree<K>(dp)};
+  team_sum<T, 1>(dot, red, phase, team, NT, mask);
+  const float2 m2 = bc2(mean_of(dot[0], a.H, a.inv_h, a.h_pow2));
+  // pass 2: dx, dz and the dw contributions
+  const int64_t off = row * nv + t;
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    if (act && (EXACT || k * T + t < nv)) {
+      float2 df[VE / 2], zf[VE / 2], dxv[VE / 2], dzv[VE / 2], gk[VE / 2];
+      F::unpack2(dr[k], df);
+      if constexpr (GATED) {
+        F::unpack2(zr[k], zf);
+        gain.get2(k, gk);
+      }
+#pragma unroll
+      for (int q = 0; q < VE / 2; ++q) {
+        dxv[q] = mul2(rs2, fma2(neg2(xh[k][q]), m2, gd[k][q]));   // rstd*(g*dy - xh*m)
+        const float2 qv = mul2(df[q], xh[k][q]);                  // dy * xh
+        if constexpr (GATED) {
+          const float2 sv = sg[k][q];
+          const float2 c = gate_slope_over_s2<ACT>(zf[q], sv);
+          dzv[q] = mul2(mul2(mul2(qv, gk[q]), sv), c);            // dy*xh*u*a'(z)
+          d[k][q] = mul2(qv, gate2<ACT>(zf[q], sv));              // dy*xh*a(z)
+        } else {
+          d[k][q] = qv;
+        }
+      }
+      st_stream(a.dx + off + k * T, F::pack2v(dxv));
+      if constexpr (GATED) st_stream(a.dz + off + k * T, F::pack2v(dzv));
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Backward: one team per 32-row leaf, rows in ascending order.  x, dy (z) and
 // rstd are staged S-1 rows ahead; pass 1 keeps xh, g*dy and s in registers for
@@ -606,68 +688,16 @@ k_bwd(const BwdArgs a) {
         dr[k] = *slot(sl, 1, k);
         if constexpr (GATED) zr[k] = *slot(sl, 2, k);
       }
-      float rs;
-      if (have_rstd) {
-        rs = rsm[sl * bd + tid];
-      } else {   // uniform branch: recompute exactly as the forward does
-        float ss[1] = {thread_sumsq<DT, T, K, EXACT>(xr, nv, t)};
-        team_sum<T, 1>(ss, red, phase, team, NT, mask);
-        rs = rsqrtf(__fadd_rn(mean_of(ss[0], a.H, a.inv_h, a.h_pow2), a.eps));
-      }
-      // pass 1: keep xh, g*dy and s for pass 2 (element pairs)
-      const float2 rs2 = bc2(rs);
-      float2 xh[K][VE / 2], gd[K][VE / 2], sg[K][GATED ? VE / 2 : 1];
+      float2 d[K][VE / 2];
+      bwd_row<DT, T, K, ACT, EXACT>(a, gain, xr, dr, zr, have_rstd ? rsm[sl * bd + tid] : 0.0f,
+                                   have_rstd, row, act, t, red, phase, team, NT, mask, d);
+      if (act) {
 #pragma unroll
-      for (int k = 0; k < K; ++k) {
-        float2 xf[VE / 2], df[VE / 2], zf[VE / 2], gk[VE / 2];
-        F::unpack2(xr[k], xf);
-        F::unpack2(dr[k], df);
-        if constexpr (GATED) F::unpack2(zr[k], zf);
-        gain.get2(k, gk);
+        for (int k = 0; k < K; ++k) {
+          if (EXACT || k * T + t < nv) {
 #pragma unroll
-        for (int q = 0; q < VE / 2; ++q) {
-          xh[k][q] = mul2(xf[q], rs2);
-          float2 g;
-          if constexpr (GATED) {
-            sg[k][q] = sigmoid2(zf[q]);
-            g = mul2(gk[q], gate2<ACT>(zf[q], sg[k][q]));   // u * a(z)
-          } else {
-            g = gk[q];                                      // u
+            for (int q = 0; q < VE / 2; ++q) acc[k][q] = add2(acc[k][q], d[k][q]);
           }
-          gd[k][q] = mul2(g, df[q]);
-        }
-      }
-      float dp[K];   // per-vector dot partials, joined by the pairwise tree
-      vector_dots<VE, T, K, EXACT>(gd, xh, nv, t, dp);
-      float dot[1] = {pairwise_tree<K>(dp)};
-      team_sum<T, 1>(dot, red, phase, team, NT, mask);
-      const float2 m2 = bc2(mean_of(dot[0], a.H, a.inv_h, a.h_pow2));
-      // pass 2: dx, dz, and the leaf's dw fold (rows in ascending order)
-      const int64_t off = row * nv + t;
-#pragma unroll
-      for (int k = 0; k < K; ++k) {
-        if (act && (EXACT || k * T + t < nv)) {
-          float2 df[VE / 2], zf[VE / 2], dxv[VE / 2], dzv[VE / 2], gk[VE / 2];
-          F::unpack2(dr[k], df);
-          if constexpr (GATED) {
-            F::unpack2(zr[k], zf);
-            gain.get2(k, gk);
-          }
-#pragma unroll
-          for (int q = 0; q < VE / 2; ++q) {
-            dxv[q] = mul2(rs2, fma2(neg2(xh[k][q]), m2, gd[k][q]));   // rstd*(g*dy - xh*m)
-            const float2 qv = mul2(df[q], xh[k][q]);                  // dy * xh
-            if constexpr (GATED) {
-              const float2 sv = sg[k][q];
-              const float2 c = gate_slope_over_s2<ACT>(zf[q], sv);
-              dzv[q] = mul2(mul2(mul2(qv, gk[q]), sv), c);            // dy*xh*u*a'(z)
-              acc[k][q] = add2(acc[k][q], mul2(qv, gate2<ACT>(zf[q], sv)));   // += dy*xh*a(z)
-            } else {
-              acc[k][q] = add2(acc[k][q], qv);
-            }
-          }
-          st_stream(a.dx + off + k * T, F::pack2v(dxv));
-          if constexpr (GATED) st_stream(a.dz + off + k * T, F::pack2v(dzv));
         }
       }
       if (++sl == S) sl = 0;
@@ -677,6 +707,141 @@ k_bwd(const BwdArgs a) {
     const int64_t rem = n_leaves - grp * NT;
     join_leaves<VE, K, T, EXACT>(acc, NT, rem < NT ? int(rem) : NT, team, t, nv, a.H, leafbuf,
                                  a.part + grp * a.H);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Backward for narrow rows (stripe_shape: T <= 8, every vector slot used, H a
+// multiple of 128): one warp per group of lpc leaves (an aligned power-of-two
+// block).  Per step the warp's RPS = 32/T teams take RPS consecutive rows of
+// the group, in row order, so each step reads and writes one contiguous block
+// of rows (2 KB of each tensor at H = 128, bf16); a team per leaf would touch
+// RPS places 8 KB apart per step, which HBM serves markedly slower.  The
+// step's dw contributions pass through shared memory transposed: lane l then
+// holds columns [128c + 4l, 128c + 4l + 4) of every row of the step and adds
+// them to its leaf accumulator in row order (the leaf's ascending left fold
+// from -0.0); a finished leaf partial is pushed onto a binary counter of
+// pending subtrees (the level-by-level pairwise tree), whose root is the group
+// partial.  Same bits as k_bwd.
+// ---------------------------------------------------------------------------
+template <int DT, int T, int K, int ACT>
+__global__ void __launch_bounds__(32, bwd_min_blocks_of(T, K))
+k_bwd_stripe(const BwdArgs a, int lpc) {
+  using F = Fmt<DT>;
+  constexpr bool GATED = ACT != kActNone;
+  constexpr int VE = F::VE;
+  constexpr int S = bwd_stages_of(T);
+  constexpr int NTEN = GATED ? 3 : 2;     // staged tensors: x, dy (, z)
+  constexpr int GS = gain_src_of(T, K, VE);
+  constexpr int RPS = 32 / T;             // rows per step
+  constexpr int H = T * K * VE;           // every vector slot used
+  constexpr int C4 = H / 128;             // float4 column groups a lane folds
+  constexpr int TS = H + 4;               // padded row stride of the transpose buffer
+  static_assert(stripe_shape(T, K, VE, true) && GS == kGainSmem, "narrow rows only");
+  // dynamic shared memory: gain [K*T*VE] | stages [S][NTEN][K][32] uint4 |
+  // rstd stages [S][32] | transpose buffer [RPS][TS]
+  extern __shared__ float dsm[];
+  float* gsm = dsm;
+  uint4* stg = reinterpret_cast<uint4*>(gsm + K * T * VE);
+  float* rsm = reinterpret_cast<float*>(stg + S * NTEN * K * 32);
+  float* tbuf = rsm + S * 32;
+  const int tid = threadIdx.x, team = tid / T, t = tid % T;
+  const bool have_rstd = a.rstd != nullptr;
+  int phase = 0;
+
+  griddep_trigger();   // the next kernel (the dw fold) may be scheduled
+  griddep_wait();      // the previous kernel's writes are complete and visible
+  Gain<VE, K, T, GS> gain;
+  gain.init(a.w, a.woff, a.nv, t, gsm);
+  auto slot = [&](int sl, int ten, int k) -> uint4* { return stg + ((sl * NTEN + ten) * K + k) * 32 + tid; };
+  auto issue = [&](int64_t row, bool act, int sl) {
+    if (act) {
+      const int64_t off = row * (H / VE) + t;
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        cp_async16(slot(sl, 0, k), a.x + off + k * T);
+        cp_async16(slot(sl, 1, k), a.dy + off + k * T);
+        if constexpr (GATED) cp_async16(slot(sl, 2, k), a.z + off + k * T);
+      }
+      if (have_rstd) cp_async4(rsm + sl * 32 + tid, a.rstd + row);
+    }
+    cp_async_commit();
+  };
+
+  const int64_t n_leaves = (a.rows + kLeafRows - 1) / kLeafRows;
+  const int64_t n_groups = (n_leaves + lpc - 1) / lpc;
+  float4* out4 = reinterpret_cast<float4*>(a.part);
+  for (int64_t grp = blockIdx.x; grp < n_groups; grp += gridDim.x) {
+    const int64_t base = grp * lpc * kLeafRows;
+    const int64_t left = n_leaves - grp * lpc;
+    const int nl = left < lpc ? int(left) : lpc;
+    const int nsteps = nl * T;            // T steps of RPS rows per leaf
+    float4 lacc[C4];
+    TreeCounter<3, float4> tree[C4];
+#pragma unroll
+    for (int c = 0; c < C4; ++c) lacc[c] = make_float4(-0.0f, -0.0f, -0.0f, -0.0f);
+
+#pragma unroll
+    for (int i = 0; i < S - 1; ++i) {
+      const int64_t r = base + int64_t(i) * RPS + team;
+      issue(r, i < nsteps && r < a.rows, i);
+    }
+    int sl = 0;
+    for (int st = 0; st < nsteps; ++st) {
+      const int64_t row = base + int64_t(st) * RPS + team;
+      const bool act = row < a.rows;
+      {
+        const int ahead = st + S - 1;
+        const int64_t r = base + int64_t(ahead) * RPS + team;
+        int sa = sl + S - 1;
+        if (sa >= S) sa -= S;
+        issue(r, ahead < nsteps && r < a.rows, sa);
+      }
+      cp_async_wait<S - 1>();
+      uint4 xr[K], dr[K], zr[K];
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        xr[k] = *slot(sl, 0, k);
+        dr[k] = *slot(sl, 1, k);
+        if constexpr (GATED) zr[k] = *slot(sl, 2, k);
+      }
+      float2 d[K][VE / 2];
+      bwd_row<DT, T, K, ACT, true>(a, gain, xr, dr, zr, have_rstd ? rsm[sl * 32 + tid] : 0.0f,
+                                  have_rstd, row, act, t, nullptr, phase, team, RPS, 0xffffffffu,
+                                  d);
+      // transpose the step's contributions: row `team` of the buffer
+      __syncwarp();   // the previous step's readers are done
+      if (act) {
+        float4* mine = reinterpret_cast<float4*>(tbuf + team * TS);
+#pragma unroll
+        for (int k = 0; k < K; ++k)
+#pragma unroll
+          for (int h = 0; h < VE / 4; ++h)
+            mine[(k * T + t) * (VE / 4) + h] = make_float4(d[k][2 * h].x, d[k][2 * h].y,
+                                                           d[k][2 * h + 1].x, d[k][2 * h + 1].y);
+      }
+      __syncwarp();
+      const int64_t step_row = base + int64_t(st) * RPS;
+#pragma unroll
+      for (int r = 0; r < RPS; ++r) {
+        if (step_row + r < a.rows) {   // rows past the batch contribute nothing
+          const float4* src = reinterpret_cast<const float4*>(tbuf + r * TS);
+#pragma unroll
+          for (int c = 0; c < C4; ++c) lacc[c] = add4(lacc[c], src[c * 32 + tid]);
+        }
+      }
+      if ((st + 1) % T == 0) {         // a leaf is complete
+#pragma unroll
+        for (int c = 0; c < C4; ++c) {
+          tree[c].push(st / T, lacc[c]);
+          lacc[c] = make_float4(-0.0f, -0.0f, -0.0f, -0.0f);
+        }
+      }
+      if (++sl == S) sl = 0;
+    }
+    cp_async_wait<0>();   // no copy may be in flight into slots the next group reuses
+#pragma unroll
+    for (int c = 0; c < C4; ++c) out4[grp * (H / 4) + c * 32 + tid] = tree[c].finish(nl);
   }
 }
 
@@ -702,6 +867,14 @@ rn_status launch_fwd_tk(const Sched& s, const FwdArgs& a, cudaStream_t st) {
 template <int DT, int T, int K, int ACT, bool EXACT>
 rn_status launch_bwd_tk(const Sched& s, int lpc, const BwdArgs& a, int64_t groups,
                         cudaStream_t st) {
+  if constexpr (stripe_shape(T, K, Fmt<DT>::VE, EXACT)) {
+    const size_t smem = bwd_stripe_smem_bytes(s, a.H, ACT != kActNone, rn_dtype(DT));
+    static std::atomic<size_t> done{0};
+    static std::atomic<int> per_sm{0};
+    (void)prepare_kernel(k_bwd_stripe<DT, T, K, ACT>, 32, smem, done, per_sm);
+    return launch_pdl(k_bwd_stripe<DT, T, K, ACT>, dim3(grid_cap(groups)), dim3(32), smem, st,
+                      a, lpc);
+  }
   const int block = lpc * T;
   const size_t smem = bwd_smem_bytes(s, lpc, a.H, ACT != kActNone, rn_dtype(DT));
   static std::atomic<size_t> done{0};
