@@ -75,7 +75,12 @@ __host__ __device__ constexpr int bwd_max_block_of(int T) {
 __host__ __device__ constexpr int bwd_min_blocks_of(int T, int K) {
   return T <= 4 ? 7 : (T == 8 ? (K <= 2 ? 7 : 4) : ((T == 32 || T == 128) && K <= 2 ? 2 : 1));
 }
-__host__ __device__ constexpr int bwd_stages_of(int T) { return T <= 16 ? 3 : (T <= 512 ? 2 : 1); }
+// Backward staging depth (rows in flight per team): deeper for the wide teams,
+// whose few leaves (one per 32 rows) must each keep more bytes in flight,
+// within 227 KB of shared memory per CTA at the widest rows.
+__host__ __device__ constexpr int bwd_stages_of(int T, int K) {
+  return T <= 16 ? 3 : (T <= 128 ? 4 : (T <= 512 ? (K <= 2 ? 3 : 2) : 1));
+}
 
 // Where a thread's gain (w, or w + offset) comes from: shared memory
 // (thread-major) for sub-warp teams, registers when K*VE <= 16, else global

@@ -613,7 +613,7 @@ k_bwd(const BwdArgs a) {
   using F = Fmt<DT>;
   constexpr bool GATED = ACT != kActNone;
   constexpr int VE = F::VE;
-  constexpr int S = bwd_stages_of(T);
+  constexpr int S = bwd_stages_of(T, K);
   constexpr int NTEN = GATED ? 3 : 2;   // staged tensors: x, dy (, z)
   constexpr int W = T > 32 ? T / 32 : 1;
   constexpr int GS = gain_src_of(T, K, VE);
@@ -730,7 +730,7 @@ k_bwd_stripe(const BwdArgs a, int lpc) {
   using F = Fmt<DT>;
   constexpr bool GATED = ACT != kActNone;
   constexpr int VE = F::VE;
-  constexpr int S = bwd_stages_of(T);
+  constexpr int S = bwd_stages_of(T, K);
   constexpr int NTEN = GATED ? 3 : 2;     // staged tensors: x, dy (, z)
   constexpr int GS = gain_src_of(T, K, VE);
   constexpr int RPS = 32 / T;             // rows per step
