@@ -141,27 +141,46 @@ bool pick_sched(int32_t width, rn_dtype dt, Sched* s) {
   if (nv <= 32) { s->T = pow2ceil(nv) / 4 > 1 ? pow2ceil(nv) / 4 : 1; s->K = (nv + s->T - 1) / s->T; }
   else if (nv <= 128) { s->T = 32; s->K = (nv + 31) / 32; }
   else if (nv <= 512) { s->T = 128; s->K = (nv + 127) / 128; }
-  else if (nv <= 2048) { s->T = 512; s->K = (nv + 511) / 512; }
+  else if (nv <= 2048) {
+    // exact fits first (no idle lanes): 512 x K, else 128 x K or 256 x K with
+    // K <= 5 (H = 5120 in 16-bit formats is 128 x 5), else 512 x ceil(nv/512)
+    if (nv % 512 == 0) { s->T = 512; s->K = nv / 512; }
+    else if (nv % 128 == 0 && nv / 128 <= 5) { s->T = 128; s->K = nv / 128; }
+    else if (nv % 256 == 0 && nv / 256 <= 5) { s->T = 256; s->K = nv / 256; }
+    else { s->T = 512; s->K = (nv + 511) / 512; }
+  }
   else { s->T = 1024; s->K = (nv + 1023) / 1024; }
   return true;
 }
 
 constexpr size_t kSmemCap = 96 * 1024;   // leaves per CTA shrink until the backward fits
 
-// Leaves one backward CTA folds (a power of two); sized for the gated op's
-// staging so that every activation uses the same geometry.
-int leaves_per_cta(const Sched& s, int width, rn_dtype dt) {
+int64_t n_leaves_of(int64_t rows) { return (rows + kLeafRows - 1) / kLeafRows; }
+
+// Leaves one backward CTA folds (a power of two).  k_bwd: sized for the gated
+// op's staging so that every activation uses the same geometry.  k_bwd_stripe
+// (one warp walks its leaves 32/T rows at a time): the fewest leaves per warp
+// that still fit the group count into about one wave of resident warps (8 per
+// SM), so small batches spread over many warps instead of walking 8 leaves
+// each.  The bits never depend on this choice.
+int leaves_per_cta(const Sched& s, int width, rn_dtype dt, int64_t rows) {
+  const int req = g_leaves_per_cta.load();
+  if (stripe_shape(s.T, s.K, vec_elems(dt), width / vec_elems(dt) == s.T * s.K)) {
+    if (req > 0) return req < 8 ? req : 8;
+    const int64_t slots = int64_t(8) * sm_count();
+    const int64_t leaves = n_leaves_of(rows);
+    int lpc = 1;
+    while (lpc < 8 && (leaves + lpc - 1) / lpc > slots) lpc *= 2;
+    return lpc;
+  }
   const int maxb = bwd_max_block_of(s.T);
   int lpc = maxb / s.T;                                   // default: fill the block
   if (s.T > 32 && width > 2048) lpc = 1;
-  const int req = g_leaves_per_cta.load();
   if (req > 0) lpc = req < lpc ? req : lpc;
   if (lpc > 8) lpc = 8;
   while (lpc > 1 && bwd_smem_bytes(s, lpc, width, true, dt) > kSmemCap) lpc /= 2;
   return lpc;
 }
-
-int64_t n_leaves_of(int64_t rows) { return (rows + kLeafRows - 1) / kLeafRows; }
 
 size_t ws_bytes_of(int64_t rows, int32_t width) {
   if (rows <= 0 || rows > kMaxRows || !width_ok(width)) return 0;
@@ -306,7 +325,7 @@ rn_status bwd_entry(int64_t rows, int32_t width, float eps, float woff, rn_act a
   }
   Sched s;
   pick_sched(width, dt, &s);
-  const int lpc = leaves_per_cta(s, width, dt);
+  const int lpc = leaves_per_cta(s, width, dt, rows);
   const int64_t leaves = n_leaves_of(rows);
   const int64_t groups = (leaves + lpc - 1) / lpc;
   float* region_a = static_cast<float*>(ws);
@@ -504,14 +523,14 @@ rn_status rn_fold_rows(int64_t n, int32_t width, const float* in, float* out, rn
 const char* rn_describe(int32_t width, rn_dtype dt) {
   Sched s;
   if (!pick_sched(width, dt, &s)) return "unsupported";
-  const int lpc = leaves_per_cta(s, width, dt);
+  const int lpc = leaves_per_cta(s, width, dt, 262144);
   const bool stripe = stripe_shape(s.T, s.K, vec_elems(dt), width / vec_elems(dt) == s.T * s.K);
   std::snprintf(t_describe, sizeof t_describe,
                 "backend=cuda-sm100a lib=librn kernels=k_fwd,%s,k_fold dtype=%s width=%d "
                 "acc=fp32 team_threads=%d vectors_per_thread=%d elems_per_vector=%d "
                 "thread_order=ascending-fma-from-neg0 lane_join=xor-butterfly(%d..1) "
                 "warp_join=%s dw_tree=leaf32-ascending-fold+level-pairwise "
-                "leaves_per_cta=%d fast_math=off atomics=none",
+                "leaves_per_cta(262144_rows)=%d fast_math=off atomics=none",
                 stripe ? "k_bwd_stripe" : "k_bwd", dtype_name(dt), width, s.T, s.K, vec_elems(dt),
                 (s.T < 32 ? s.T : 32) / 2,
                 s.T > 32 ? "smem-pairwise" : "none", lpc);
@@ -521,7 +540,7 @@ const char* rn_describe(int32_t width, rn_dtype dt) {
 int32_t rn_bwd_launches(int64_t rows, int32_t width, rn_dtype dt) {
   Sched s;
   if (rows <= 0 || rows > kMaxRows || !pick_sched(width, dt, &s)) return 0;
-  const int lpc = leaves_per_cta(s, width, dt);
+  const int lpc = leaves_per_cta(s, width, dt, rows);
   const int64_t groups = (n_leaves_of(rows) + lpc - 1) / lpc;
   return 1 + fold_passes(groups);
 }

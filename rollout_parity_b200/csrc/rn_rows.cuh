@@ -76,23 +76,19 @@ struct Fmt<RN_BF16> {
 template <>
 struct Fmt<RN_F16> {
   static constexpr int VE = 8;
+  __device__ static __forceinline__ float2 pair(uint32_t w) {
+    return __half22float2(*reinterpret_cast<const __half2*>(&w));   // .x = low half
+  }
   __device__ static __forceinline__ void unpack2(const uint4& u, float2 (&f)[4]) {
-    f[0] = make_float2(lo(u.x), hi(u.x)); f[1] = make_float2(lo(u.y), hi(u.y));
-    f[2] = make_float2(lo(u.z), hi(u.z)); f[3] = make_float2(lo(u.w), hi(u.w));
+    f[0] = pair(u.x); f[1] = pair(u.y); f[2] = pair(u.z); f[3] = pair(u.w);
+  }
+  __device__ static __forceinline__ uint32_t pack2(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);   // .x (low half) = a, each rounded to nearest even
+    return *reinterpret_cast<uint32_t*>(&h);
   }
   __device__ static __forceinline__ uint4 pack2v(const float2 (&f)[4]) {
     return make_uint4(pack2(f[0].x, f[0].y), pack2(f[1].x, f[1].y), pack2(f[2].x, f[2].y),
                       pack2(f[3].x, f[3].y));
-  }
-  __device__ static __forceinline__ float lo(uint32_t w) {
-    return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xffffu)));
-  }
-  __device__ static __forceinline__ float hi(uint32_t w) {
-    return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
-  }
-  __device__ static __forceinline__ uint32_t pack2(float a, float b) {
-    return uint32_t(__half_as_ushort(__float2half_rn(a))) |
-           (uint32_t(__half_as_ushort(__float2half_rn(b))) << 16);
   }
 };
 
@@ -896,7 +892,7 @@ rn_status launch_bwd_tk(const Sched& s, int lpc, const BwdArgs& a, int64_t group
   X(128, 2, false) X(128, 2, true) X(128, 3, false) X(128, 3, true)                             \
   X(128, 4, false) X(128, 4, true)                                                              \
   X(512, 2, false) X(512, 2, true) X(512, 3, false) X(512, 3, true)                             \
-  X(512, 4, false) X(512, 4, true)
+  X(512, 4, false) X(512, 4, true) X(128, 5, true) X(256, 3, true) X(256, 5, true)
 #define RN_SHAPES_32(X)                                                                         \
   X(1, 2, true) X(1, 4, true) X(2, 3, true) X(2, 4, true)                                       \
   X(4, 3, false) X(4, 3, true) X(4, 4, false) X(4, 4, true)                                     \
@@ -906,7 +902,8 @@ rn_status launch_bwd_tk(const Sched& s, int lpc, const BwdArgs& a, int64_t group
   X(128, 4, false) X(128, 4, true)                                                              \
   X(512, 2, false) X(512, 2, true) X(512, 3, false) X(512, 3, true)                             \
   X(512, 4, false) X(512, 4, true)                                                              \
-  X(1024, 3, false) X(1024, 3, true) X(1024, 4, false) X(1024, 4, true)
+  X(1024, 3, false) X(1024, 3, true) X(1024, 4, false) X(1024, 4, true)                         \
+  X(128, 5, true) X(256, 3, true) X(256, 5, true)
 
 template <int DT, int ACT>
 rn_status launch_fwd_act(const Sched& s, const FwdArgs& a, cudaStream_t st) {

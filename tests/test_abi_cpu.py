@@ -269,9 +269,11 @@ def test_workspace_bytes_invalid(lib):
 
 @pytest.mark.parametrize("width,dt,team", [(128, DType.BF16, 4), (128, DType.F32, 8),
                                            (8, DType.BF16, 1), (2048, DType.BF16, 128),
-                                           (8192, DType.BF16, 512), (5120, DType.BF16, 512),
+                                           (8192, DType.BF16, 512), (5120, DType.BF16, 128),
+                                           (6144, DType.BF16, 256), (10240, DType.BF16, 256),
+                                           (5120, DType.F32, 256), (4104, DType.BF16, 512),
                                            (16384, DType.F32, 1024), (128, DType.F16, 4),
-                                           (5120, DType.F16, 512), (2048, DType.F16, 128)])
+                                           (5120, DType.F16, 128), (2048, DType.F16, 128)])
 def test_describe(lib, width, dt, team):
     d = lib.rn_describe(width, dt).decode()
     assert f"team_threads={team} " in d
@@ -296,9 +298,14 @@ def test_geometry_knob_checks(lib):
 
 
 def test_bwd_launch_count(lib):
-    # 262144 rows of width 128: 8192 leaves, 8 per CTA -> 1024 partials -> 2 fold passes
+    # 262144 rows of width 128 (stripe kernel): 8192 leaves, 8 per warp -> 1024 partials
+    # -> 2 fold passes
     assert lib.rn_bwd_launches(262144, 128, DType.BF16) == 3
-    assert lib.rn_bwd_launches(256, 128, DType.BF16) == 1      # one CTA writes dw itself
+    # small batches spread one leaf per warp: 8 or 128 partials, one fold pass
+    assert lib.rn_bwd_launches(256, 128, DType.BF16) == 2
+    assert lib.rn_bwd_launches(4096, 128, DType.BF16) == 2
+    # width 136 (team-per-leaf kernel, 8 leaves per CTA): one CTA writes dw itself
+    assert lib.rn_bwd_launches(256, 136, DType.BF16) == 1
     assert lib.rn_bwd_launches(0, 128, DType.BF16) == 0
     assert lib.rn_bwd_launches(64, 100, DType.BF16) == 0
     try:

@@ -24,6 +24,9 @@ SMALL = [  # (op, rows, width, dtype): several tiles and a ragged tail
     ("norm", 65, 4096, "bf16"), ("gated", 65, 5120, "bf16"), ("norm", 40, 8192, "bf16"),
     ("gated", 33, 8192, "f32"), ("norm", 33, 12288, "bf16"), ("gated", 17, 16384, "bf16"),
     ("norm", 17, 16384, "f32"), ("gated", 1, 128, "bf16"), ("norm", 31, 2048, "bf16"),
+    # exact-fit wide teams: 128 x 5 (H=5120 16-bit, 2560 fp32), 256 x 3, 256 x 5
+    ("gated", 67, 6144, "bf16"), ("norm", 37, 10240, "bf16"), ("gated", 45, 2560, "f32"),
+    ("norm", 40, 3072, "f32"), ("gated", 35, 5120, "f32"), ("norm", 66, 5120, "bf16"),
 ]
 
 
