@@ -21,3 +21,4 @@ from .ops import (  # noqa: F401
     rmsnorm_fwd,
     workspace,
 )
+from . import autograd  # noqa: E402,F401
