@@ -108,6 +108,47 @@ k_fold(const float* __restrict__ in, int64_t n, int H, float* __restrict__ out) 
   }
 }
 
+// The last fold pass when at most kFold1Rows = 1024 partial rows remain: a CTA
+// of 32 warps covers 32 columns (one float per lane); warp g streams rows
+// [32g, 32g + 32) through the binary counter of pending subtrees, and the warps'
+// results (aligned blocks of 32 rows: perfect subtrees) are joined in shared
+// memory by the pairwise tree.  One launch where k_fold would need two.
+constexpr int kFold1Rows = 1024;
+__global__ void __launch_bounds__(1024)
+k_fold1(const float* __restrict__ in, int64_t n, int H, float* __restrict__ out) {
+  griddep_trigger();
+  griddep_wait();      // the partials of the previous kernel are complete and visible
+  const int lane = threadIdx.x & 31, g = threadIdx.x >> 5;
+  const int c = blockIdx.x * 32 + lane;
+  const bool col_ok = c < H;
+  const int64_t start = int64_t(g) * 32;
+  const int64_t left = n - start;
+  const int cnt = left <= 0 ? 0 : (left >= 32 ? 32 : int(left));
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = (col_ok && i < cnt) ? __ldcg(in + (start + i) * H + c) : 0.0f;
+  TreeCounter<5, float> tc;
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if (i < cnt) tc.push(i, v[i]);
+  __shared__ float sm[32][33];
+  sm[g][lane] = cnt > 0 ? tc.finish(cnt) : 0.0f;
+  __syncthreads();
+  if (g == 0 && col_ok) {
+    const int ng = int((n + 31) / 32);
+    float p[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) p[i] = sm[i][lane];
+#pragma unroll
+    for (int sft = 1; sft < 32; sft <<= 1) {
+#pragma unroll
+      for (int l = 0; l + sft < 32; l += 2 * sft)
+        if (l + sft < ng) p[l] = __fadd_rn(p[l], p[l + sft]);
+    }
+    out[c] = p[0];
+  }
+}
+
 // Test kernel: the reciprocal used by the sigmoid, for checking against IEEE
 // division over every float in [1, 2].
 __global__ void k_test_rcp(const float* __restrict__ d, float* __restrict__ out, int64_t n,
@@ -230,10 +271,16 @@ int fold_rows_default(int64_t n) {
   return int(s);
 }
 
+// With the default geometry, 257..1024 rows are folded in one k_fold1 pass
+// (k_fold would take two); up to 256 in one k_fold pass; more in passes of
+// fold_rows_default rows first.
+bool use_fold1(int64_t n) { return g_fold_rows.load() <= 0 && n > 256 && n <= kFold1Rows; }
+
 int fold_passes(int64_t n) {
   int passes = 0;
   while (n > 1) {
     int S = g_fold_rows.load();
+    if (use_fold1(n)) return passes + 1;
     if (S <= 0) S = fold_rows_default(n);
     n = (n + S - 1) / S;
     ++passes;
@@ -270,6 +317,8 @@ rn_status run_fold(float* a, float* b, int64_t n, int H, float* dw, cudaStream_t
   rn_status e = RN_OK;
   while (n > 1) {
     int S = g_fold_rows.load();
+    if (use_fold1(n))
+      return launch_pdl(k_fold1, dim3(unsigned((H + 31) / 32)), dim3(1024), 0, st, src, n, H, dw);
     if (S <= 0) S = fold_rows_default(n);
     const int B = S / kFoldRG;
     const int64_t nout = (n + S - 1) / S;
@@ -526,7 +575,7 @@ const char* rn_describe(int32_t width, rn_dtype dt) {
   const int lpc = leaves_per_cta(s, width, dt, 262144);
   const bool stripe = stripe_shape(s.T, s.K, vec_elems(dt), width / vec_elems(dt) == s.T * s.K);
   std::snprintf(t_describe, sizeof t_describe,
-                "backend=cuda-sm100a lib=librn kernels=k_fwd,%s,k_fold dtype=%s width=%d "
+                "backend=cuda-sm100a lib=librn kernels=k_fwd,%s,k_fold,k_fold1 dtype=%s width=%d "
                 "acc=fp32 team_threads=%d vectors_per_thread=%d elems_per_vector=%d "
                 "thread_order=ascending-fma-from-neg0 lane_join=xor-butterfly(%d..1) "
                 "warp_join=%s dw_tree=leaf32-ascending-fold+level-pairwise "

@@ -299,13 +299,15 @@ def test_geometry_knob_checks(lib):
 
 def test_bwd_launch_count(lib):
     # 262144 rows of width 128 (stripe kernel): 8192 leaves, 8 per warp -> 1024 partials
-    # -> 2 fold passes
-    assert lib.rn_bwd_launches(262144, 128, DType.BF16) == 3
+    # -> one fold pass of up to 1024 rows
+    assert lib.rn_bwd_launches(262144, 128, DType.BF16) == 2
     # small batches spread one leaf per warp: 8 or 128 partials, one fold pass
     assert lib.rn_bwd_launches(256, 128, DType.BF16) == 2
     assert lib.rn_bwd_launches(4096, 128, DType.BF16) == 2
     # width 136 (team-per-leaf kernel, 8 leaves per CTA): one CTA writes dw itself
     assert lib.rn_bwd_launches(256, 136, DType.BF16) == 1
+    # 2^22 rows at width 2048 (one leaf per CTA): 131072 partials -> 4096 -> 128 -> dw
+    assert lib.rn_bwd_launches(1 << 22, 2048, DType.BF16) == 1 + 3
     assert lib.rn_bwd_launches(0, 128, DType.BF16) == 0
     assert lib.rn_bwd_launches(64, 100, DType.BF16) == 0
     try:
