@@ -50,6 +50,11 @@ is added only when it is nonzero, so a -0.0 weight keeps its sign):
 The zero-centred and gated operators above are (offset 1, no gate) and
 (offset 0, silu).
 
+Row mask for dw ([PR468] "Changes to existing code, in detail": the dw entry
+point takes a mask; read as one flag per row, rows with the flag clear left out
+of dw's sum, e.g. padding):  dw_j = sum over rows r with mask_r of
+dy_rj * xh_rj * a(z_rj); dx and dz are unchanged.
+
 Parity pins (``tests/oracle_pins.py``, run by ``tests/test_oracle_pins.py``,
 with planted mistakes in ``tests/test_oracle_mutations.py``):
   rstd/forward : constant-row closed form, RMS(xh) == 1 at eps = 0, scale
@@ -62,6 +67,9 @@ with planted mistakes in ``tests/test_oracle_mutations.py``):
   general form : a rational worked example (sigmoid gate, offset 1), finite
                  differences for every activation x offset {0, 1, 1/2}, the
                  signed-zero rule, and reduction to the two operators above.
+  row mask     : all-ones equals no mask, a brute-force loop over the selected
+                 rows, masked rows holding NaN/Inf leave dw finite and dx of the
+                 other rows unchanged, dw(mask) + dw(not mask) = dw.
 Every public function below is pinned; none is "parity unpinned".
 """
 from __future__ import annotations
@@ -221,8 +229,11 @@ def rmsnorm_fwd(x, w, eps: float, weight_offset: float = 1.0, z=None, act: str =
     return x * rho[:, None] * u[None, :] * a, rho
 
 
-def rmsnorm_bwd(x, w, dy, eps: float, weight_offset: float = 1.0, z=None, act: str = "none"):
-    """Returns (dx, dz, dw); dz is None without a gate."""
+def rmsnorm_bwd(x, w, dy, eps: float, weight_offset: float = 1.0, z=None, act: str = "none",
+                row_mask=None):
+    """Returns (dx, dz, dw); dz is None without a gate.  row_mask (one value per
+    row, nonzero = the row counts) limits dw's sum to those rows; dx and dz are
+    every row's.  A row outside the mask adds nothing, whatever its values."""
     x, dy = _rows(x), _rows(dy)
     rho = rstd(x, eps)
     xh = x * rho[:, None]
@@ -231,7 +242,10 @@ def rmsnorm_bwd(x, w, dy, eps: float, weight_offset: float = 1.0, z=None, act: s
     g = u * a
     dx = _dx(x, np.broadcast_to(g, x.shape), dy, rho)
     dz = None if act == "none" else dy * xh * u * da
-    dw = np.sum(dy * xh * a, axis=0)
+    contrib = dy * xh * a * np.ones_like(x)
+    if row_mask is not None:
+        contrib = contrib[np.asarray(row_mask).astype(bool)]
+    dw = np.sum(contrib, axis=0)
     return dx, dz, dw
 
 

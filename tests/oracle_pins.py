@@ -362,6 +362,43 @@ def pin_signed_zero_weight(orc):
         assert y1[0, 0] != 0 and y1[0, 2] != 0, (act, y1)
 
 
+def pin_row_mask(orc):
+    """dw over the rows a mask selects: all-ones is no mask; a loop over the
+    selected rows using one-row forward outputs (dy * y / u is dy * xh * a(z));
+    masked rows with non-finite values change nothing else; the mask and its
+    complement add up to the whole batch; dx and dz ignore the mask."""
+    rng = np.random.default_rng(21)
+    R, H, eps = 11, 6, 1e-3
+    x = rng.normal(size=(R, H)); z = rng.normal(size=(R, H)); dy = rng.normal(size=(R, H))
+    w = rng.uniform(0.5, 1.5, size=H)
+    mask = np.array([1, 0, 1, 1, 0, 0, 1, 0, 1, 1, 0], dtype=np.uint8)
+    for act, off in (("none", 1.0), ("silu", 0.0), ("sigmoid", 1.0)):
+        zz = None if act == "none" else z
+        full = orc.rmsnorm_bwd(x, w, dy, eps, off, zz, act)
+        ones = orc.rmsnorm_bwd(x, w, dy, eps, off, zz, act, row_mask=np.ones(R, np.uint8))
+        _close(ones[2], full[2], rtol=0, atol=0, what=f"{act} all-ones mask dw")
+        dx, dz, dw = orc.rmsnorm_bwd(x, w, dy, eps, off, zz, act, row_mask=mask)
+        _close(dx, full[0], rtol=0, atol=0, what=f"{act} dx ignores the mask")
+        if dz is not None:
+            _close(dz, full[1], rtol=0, atol=0, what=f"{act} dz ignores the mask")
+        want = np.zeros(H)
+        u = w + off if off != 0 else w
+        for r in range(R):
+            if mask[r]:
+                y, _ = orc.rmsnorm_fwd(x[r:r + 1], w, eps, off, None if zz is None else z[r:r + 1], act)
+                want += dy[r] * y[0] / u
+        _close(dw, want, rtol=1e-12, atol=1e-14, what=f"{act} masked dw brute force")
+        _, _, dwc = orc.rmsnorm_bwd(x, w, dy, eps, off, zz, act, row_mask=1 - mask)
+        _close(dw + dwc, full[2], rtol=1e-12, atol=1e-14, what=f"{act} mask + complement")
+        xb = x.copy(); xb[1] = np.nan; xb[4, 2] = np.inf
+        with np.errstate(all="ignore"):
+            dxb, _, dwb = orc.rmsnorm_bwd(xb, w, dy, eps, off, zz, act, row_mask=mask)
+        assert np.all(np.isfinite(dwb)), f"{act}: masked non-finite rows leaked into dw"
+        _close(dwb, dw, rtol=0, atol=0, what=f"{act} masked non-finite rows")
+        keep = [r for r in range(R) if r not in (1, 4)]
+        _close(dxb[keep], dx[keep], rtol=0, atol=0, what=f"{act} other rows' dx")
+
+
 ALL_PINS = [
     pin_worked_example_norm,
     pin_worked_example_eps,
@@ -379,6 +416,7 @@ ALL_PINS = [
     pin_general_special_cases,
     pin_general_finite_differences,
     pin_signed_zero_weight,
+    pin_row_mask,
 ]
 
 

@@ -210,6 +210,50 @@ def m_general_dw_drops_gate(o):
     o.rmsnorm_bwd = rmsnorm_bwd
 
 
+def m_mask_ignored(o):
+    real = o.rmsnorm_bwd
+    o.rmsnorm_bwd = lambda x, w, dy, eps, weight_offset=1.0, z=None, act="none", row_mask=None: \
+        real(x, w, dy, eps, weight_offset, z, act)
+
+
+def m_mask_inverted(o):
+    real = o.rmsnorm_bwd
+
+    def rmsnorm_bwd(x, w, dy, eps, weight_offset=1.0, z=None, act="none", row_mask=None):
+        m = None if row_mask is None else 1 - np.asarray(row_mask)
+        if m is not None and not m.any():
+            m = None
+        return real(x, w, dy, eps, weight_offset, z, act, m)
+    o.rmsnorm_bwd = rmsnorm_bwd
+
+
+def m_mask_zeroes_dx(o):
+    real = o.rmsnorm_bwd
+
+    def rmsnorm_bwd(x, w, dy, eps, weight_offset=1.0, z=None, act="none", row_mask=None):
+        dx, dz, dw = real(x, w, dy, eps, weight_offset, z, act, row_mask)
+        if row_mask is not None:
+            dx = dx * np.asarray(row_mask, dtype=np.float64)[:, None]
+        return dx, dz, dw
+    o.rmsnorm_bwd = rmsnorm_bwd
+
+
+def m_mask_multiplies_contributions(o):
+    # a multiply by the mask instead of leaving rows out: NaN * 0 is NaN
+    real = o.rmsnorm_bwd
+
+    def rmsnorm_bwd(x, w, dy, eps, weight_offset=1.0, z=None, act="none", row_mask=None):
+        dx, dz, dw = real(x, w, dy, eps, weight_offset, z, act)
+        if row_mask is not None:
+            xr = np.asarray(x, dtype=np.float64)
+            rho = o.rstd(xr, eps)
+            a, _ = o._act(None if z is None else np.asarray(z, dtype=np.float64), act)
+            c = np.asarray(dy, dtype=np.float64) * xr * rho[:, None] * a
+            dw = np.sum(c * np.asarray(row_mask, dtype=np.float64)[:, None], axis=0)
+        return dx, dz, dw
+    o.rmsnorm_bwd = rmsnorm_bwd
+
+
 MUTANTS = [m for name, m in sorted(globals().items()) if name.startswith("m_")]
 
 
