@@ -5,6 +5,11 @@ reference legs may import this package.  The library never does.
 """
 from .rmsnorm import (  # noqa: F401
     ACTS,
+    FORMATS,
+    residual_add,
+    rmsnorm_add_bwd,
+    rmsnorm_add_fwd,
+    round_to_format,
     dx_cancellation_scale,
     dz_cancellation_scale,
     gated_norm_bwd,

@@ -67,6 +67,10 @@ with planted mistakes in ``tests/test_oracle_mutations.py``):
   general form : a rational worked example (sigmoid gate, offset 1), finite
                  differences for every activation x offset {0, 1, 1/2}, the
                  signed-zero rule, and reduction to the two operators above.
+  residual add : fp32 -> bf16 / fp16 rounding against torch's conversions and
+                 hand-checked ties, an exact example where the rounded sum is
+                 the worked example's row, r = 0 reduces to the plain forward,
+                 finite differences of sum(y*dy) + sum(h*dh) in x and in r.
   row mask     : all-ones equals no mask, a brute-force loop over the selected
                  rows, masked rows holding NaN/Inf leave dw finite and dx of the
                  other rows unchanged, dw(mask) + dw(not mask) = dw.
@@ -274,3 +278,61 @@ def rmsnorm_dz_scale(x, w, dy, eps: float, weight_offset: float, z, act: str) ->
     if act == "sigmoid":
         return lead
     raise ValueError(f"no dz without a gate (act {act!r})")
+
+
+# ---------------------------------------------------------------------------
+# Residual add.  [PR468] names an RMSNorm variant "with a residual" ("Notes",
+# on the strict profile's norm choice) and defines nothing more; read as the
+# usual fused form: the residual stream h = x + r is stored in the tensors'
+# format and normalised:
+#     h = fmt(x + r),   y = h * rho(h) * u * a(z)
+# The sum is formed in fp32 and rounded once to the format, the kernel's
+# precision for that rounding decision (the pages fix none).  Backward: the
+# gradient reaching h is the norm's plus dh, the gradient of the residual
+# output, and both x and r receive it:  dx = dr = dnorm(h; dy) + dh.
+# ---------------------------------------------------------------------------
+FORMATS = ("f32", "bf16", "f16", "f64")
+
+
+def round_to_format(a, fmt: str) -> np.ndarray:
+    """fp32 values rounded to nearest even in the 16-bit formats (f32 keeps
+    them; f64 means no rounding at all).  Returns fp64."""
+    if fmt == "f64":
+        return np.asarray(a, dtype=np.float64)
+    a32 = np.asarray(a, dtype=np.float32)
+    if fmt == "f32":
+        return a32.astype(np.float64)
+    if fmt == "f16":
+        return a32.astype(np.float16).astype(np.float64)   # IEEE round to nearest even
+    if fmt == "bf16":
+        # keep the top 16 bits of the fp32 encoding, rounding the dropped 16 to
+        # nearest with ties to the even kept value (finite inputs)
+        b = a32.view(np.uint32).astype(np.uint64)
+        b = (b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000
+        return b.astype(np.uint32).view(np.float32).astype(np.float64)
+    raise ValueError(f"unknown format {fmt!r}")
+
+
+def residual_add(x, r, fmt: str) -> np.ndarray:
+    """h = fmt(fp32(x) + fp32(r)); x and r hold values of the format."""
+    if fmt == "f64":
+        return _rows(x) + _rows(r)
+    s = np.asarray(x, dtype=np.float32) + np.asarray(r, dtype=np.float32)
+    return round_to_format(s, fmt).reshape(_rows(x).shape)
+
+
+def rmsnorm_add_fwd(x, r, w, eps: float, weight_offset: float = 1.0, z=None, act: str = "none",
+                    fmt: str = "bf16"):
+    """Returns (h, y, rho)."""
+    h = residual_add(x, r, fmt)
+    y, rho = rmsnorm_fwd(h, w, eps, weight_offset, z, act)
+    return h, y, rho
+
+
+def rmsnorm_add_bwd(h, w, dy, dh, eps: float, weight_offset: float = 1.0, z=None,
+                    act: str = "none", row_mask=None):
+    """Returns (dx, dz, dw); dx is the gradient of both x and r."""
+    dx, dz, dw = rmsnorm_bwd(h, w, dy, eps, weight_offset, z, act, row_mask)
+    if dh is not None:
+        dx = dx + _rows(dh)
+    return dx, dz, dw

@@ -399,6 +399,69 @@ def pin_row_mask(orc):
         _close(dxb[keep], dx[keep], rtol=0, atol=0, what=f"{act} other rows' dx")
 
 
+def pin_round_to_format(orc):
+    """fp32 -> bf16 / fp16 rounding equals torch's conversions (a library
+    routine) on random values across magnitudes, and hand-checked ties."""
+    import torch
+    rng = np.random.default_rng(22)
+    a = np.concatenate([rng.standard_normal(4000).astype(np.float32) * s
+                        for s in (1e-6, 1e-3, 1.0, 300.0, 3e4)])
+    # exact ties: a kept value plus half its last place
+    a = np.concatenate([a, np.float32([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(2 + 2.0 ** -7),
+                                       1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11])])
+    t = torch.from_numpy(a)
+    for fmt, dt in (("bf16", torch.bfloat16), ("f16", torch.float16)):
+        got = orc.round_to_format(a, fmt)
+        want = t.to(dt).double().numpy()          # fp16 overflows to inf past 65504
+        assert np.array_equal(got, want), f"{fmt} rounding differs at " \
+            f"{np.flatnonzero(got != want)[:5]}"
+    _close(orc.round_to_format(np.float32([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8]), "bf16"),
+           [1.0, 1 + 2.0 ** -6], rtol=0, atol=0, what="bf16 ties to even")
+    _close(orc.round_to_format(np.float32([1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11]), "f16"),
+           [1.0, 1 + 2.0 ** -9], rtol=0, atol=0, what="f16 ties to even")
+
+
+def pin_residual_add_example(orc):
+    """x = [1, 2, 2, 4], r = [2^-9, 0, 0, 0]: the fp32 sum 1 + 2^-9 is below half
+    a bf16 place of 1, so h is x itself and y is the first worked example's
+    ([2/5, 6/5, 0, 16/5] at w = [0, 1/2, -1, 1], offset 1, eps = 0); in fp32 the
+    sum is kept and h differs.  r = 0 reduces to the plain forward."""
+    x = [[1.0, 2.0, 2.0, 4.0]]
+    r = [[2.0 ** -9, 0.0, 0.0, 0.0]]
+    w = [0.0, 0.5, -1.0, 1.0]
+    h, y, rho = orc.rmsnorm_add_fwd(x, r, w, 0.0, 1.0, None, "none", fmt="bf16")
+    _close(h, x, rtol=0, atol=0, what="bf16 h")
+    _close(y, [[0.4, 1.2, 0.0, 3.2]], what="y from the rounded h")
+    _close(rho, [0.4], what="rho")
+    h32, _, _ = orc.rmsnorm_add_fwd(x, r, w, 0.0, 1.0, None, "none", fmt="f32")
+    _close(h32, [[1 + 2.0 ** -9, 2.0, 2.0, 4.0]], rtol=0, atol=0, what="f32 h")
+    rng = np.random.default_rng(23)
+    xs = rng.normal(size=(3, 8)); zs = rng.normal(size=(3, 8)); ws = rng.normal(size=8)
+    h0, y0, _ = orc.rmsnorm_add_fwd(xs, np.zeros_like(xs), ws, 1e-6, 0.0, zs, "silu", fmt="f64")
+    _close(h0, xs, rtol=0, atol=0, what="r = 0 keeps x")
+    _close(y0, orc.gated_norm_fwd(xs, zs, ws, 1e-6)[0], what="r = 0 is the plain forward")
+
+
+def pin_residual_finite_differences(orc):
+    """With the sum unrounded (f64), dx equals the numerical gradient of
+    L = sum(y * dy) + sum(h * dh) in x and in r (both get the same gradient)."""
+    rng = np.random.default_rng(24)
+    R, H, eps = 2, 6, 1e-2
+    x = rng.normal(size=(R, H)); r = rng.normal(size=(R, H)); z = rng.normal(size=(R, H))
+    w = rng.normal(size=H); dy = rng.normal(size=(R, H)); dh = rng.normal(size=(R, H))
+    for act, off in (("none", 1.0), ("silu", 0.0), ("sigmoid", 1.0)):
+        zz = None if act == "none" else z
+
+        def L(x_, r_):
+            h, y, _ = orc.rmsnorm_add_fwd(x_, r_, w, eps, off, zz, act, fmt="f64")
+            return float(np.sum(y * dy) + np.sum(h * dh))
+
+        h, _, _ = orc.rmsnorm_add_fwd(x, r, w, eps, off, zz, act, fmt="f64")
+        dx, _, _ = orc.rmsnorm_add_bwd(h, w, dy, dh, eps, off, zz, act)
+        _close(dx, _fd(lambda a: L(a, r), x), rtol=1e-7, atol=1e-8, what=f"{act} d/dx")
+        _close(dx, _fd(lambda a: L(x, a), r), rtol=1e-7, atol=1e-8, what=f"{act} d/dr")
+
+
 ALL_PINS = [
     pin_worked_example_norm,
     pin_worked_example_eps,
@@ -417,6 +480,9 @@ ALL_PINS = [
     pin_general_finite_differences,
     pin_signed_zero_weight,
     pin_row_mask,
+    pin_round_to_format,
+    pin_residual_add_example,
+    pin_residual_finite_differences,
 ]
 
 

@@ -254,6 +254,48 @@ def m_mask_multiplies_contributions(o):
     o.rmsnorm_bwd = rmsnorm_bwd
 
 
+def m_residual_not_rounded(o):
+    real = o.residual_add
+    o.residual_add = lambda x, r, fmt: real(x, r, "f64")
+
+
+def m_residual_dh_dropped(o):
+    real = o.rmsnorm_add_bwd
+    o.rmsnorm_add_bwd = lambda h, w, dy, dh, eps, weight_offset=1.0, z=None, act="none", \
+        row_mask=None: real(h, w, dy, None, eps, weight_offset, z, act, row_mask)
+
+
+def m_residual_norm_of_unrounded_sum(o):
+    def rmsnorm_add_fwd(x, r, w, eps, weight_offset=1.0, z=None, act="none", fmt="bf16"):
+        h = o.residual_add(x, r, fmt)
+        y, rho = o.rmsnorm_fwd(o.residual_add(x, r, "f64"), w, eps, weight_offset, z, act)
+        return h, y, rho
+    o.rmsnorm_add_fwd = rmsnorm_add_fwd
+
+
+def m_bf16_round_truncates(o):
+    real = o.round_to_format
+
+    def round_to_format(a, fmt):
+        if fmt != "bf16":
+            return real(a, fmt)
+        b = np.asarray(a, dtype=np.float32).view(np.uint32) & np.uint32(0xFFFF0000)
+        return b.view(np.float32).astype(np.float64)
+    o.round_to_format = round_to_format
+
+
+def m_bf16_round_ties_up(o):
+    real = o.round_to_format
+
+    def round_to_format(a, fmt):
+        if fmt != "bf16":
+            return real(a, fmt)
+        b = np.asarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+        b = (b + 0x8000) & 0xFFFF0000
+        return b.astype(np.uint32).view(np.float32).astype(np.float64)
+    o.round_to_format = round_to_format
+
+
 MUTANTS = [m for name, m in sorted(globals().items()) if name.startswith("m_")]
 
 
