@@ -248,7 +248,7 @@ def run_ours(a):
 
     def bwd(p, stp=sp):
         return lib.rmsnorm_bwd(R, H, eps, woff, actc, dtc, p["x"], p["z"], p["w"], p["dy"],
-                               p["rstd"], p["dx"], p["dz"], p["dw"], p["ws"], nws, stp)
+                               p["rstd"], None, p["dx"], p["dz"], p["dw"], p["ws"], nws, stp)
 
     for p in P:                       # every set gets its rstd before any backward
         check("rmsnorm_fwd", fwd(p))

@@ -132,13 +132,48 @@ rn_status rmsnorm_fwd(int64_t rows, int32_t width, float eps, float weight_offse
  *   g = u * a(z),  m = mean_j(g_j * dy_j * xh_j),  xh = x * rstd,
  *   dx = rstd * (g * dy - xh * m),  dz = dy * xh * u * a'(z),
  *   dw[j] = sum over rows of dy * xh * a(z)   (the offset is a constant).
+ * row_mask: [rows] bytes, read, or NULL.  Rows with row_mask[r] == 0 are left
+ *   out of dw (they add nothing, whatever their values -- padding may hold
+ *   anything); dx and dz are written for every row.  A left-out row stands
+ *   for the additive identity (-0.0) in dw's fixed tree, so the tree's shape
+ *   still depends on the row count only; a column no row contributes to is
+ *   -0.0.  (PR #468 Notes: the dw entry point takes a mask.)
  * With RN_ACT_NONE, z and dz must be NULL.  Arguments otherwise as
  * gated_norm_bwd (workspace: norm_bwd_workspace_bytes).
  */
 rn_status rmsnorm_bwd(int64_t rows, int32_t width, float eps, float weight_offset,
                       rn_act act, rn_dtype dt, const void* x, const void* z,
-                      const float* w, const void* dy, const float* rstd, void* dx,
-                      void* dz, float* dw, void* ws, size_t ws_bytes, rn_stream stream);
+                      const float* w, const void* dy, const float* rstd,
+                      const uint8_t* row_mask, void* dx, void* dz, float* dw,
+                      void* ws, size_t ws_bytes, rn_stream stream);
+
+/*
+ * Residual-add forward (PR #468 Notes name a norm "with a residual"; read as
+ * the usual fused form):
+ *   h[r, j] = fmt(x[r, j] + r_in[r, j])   fp32 sum, rounded once to dt, written;
+ *   y = rmsnorm_fwd of h (the stored, rounded h), rstd likewise.
+ * x, r: [rows, width] dt, read.  h, y: [rows, width] dt, written; h may be
+ * exactly x or exactly r (an in-place update of the residual stream), any
+ * other overlap is RN_E_ARG.  Other arguments as rmsnorm_fwd.
+ */
+rn_status rmsnorm_add_fwd(int64_t rows, int32_t width, float eps, float weight_offset,
+                          rn_act act, rn_dtype dt, const void* x, const void* r,
+                          const void* z, const float* w, void* h, void* y, float* rstd,
+                          rn_stream stream);
+
+/*
+ * Residual-add backward: h (from rmsnorm_add_fwd) takes x's place in
+ * rmsnorm_bwd, and the gradient reaching h is the norm's plus dh, the
+ * gradient of the residual output; x and r both receive it:
+ *   dx = fmt(dnorm(h; dy) + dh)   (fp32 sum, one rounding);  dz, dw as rmsnorm_bwd.
+ * dh: [rows, width] dt, read, or NULL (no gradient into h beyond the norm's);
+ * dx may be exactly dh.  Other arguments as rmsnorm_bwd.
+ */
+rn_status rmsnorm_add_bwd(int64_t rows, int32_t width, float eps, float weight_offset,
+                          rn_act act, rn_dtype dt, const void* h, const void* z,
+                          const float* w, const void* dy, const void* dh,
+                          const float* rstd, const uint8_t* row_mask, void* dx, void* dz,
+                          float* dw, void* ws, size_t ws_bytes, rn_stream stream);
 
 /*
  * Zero-centred RMSNorm forward (PR #468 Summary, with weight offset 1):

@@ -17,6 +17,8 @@ from .ops import (  # noqa: F401
     rn_fold_rows,
     rn_test_set_geometry,
     rn_test_set_validate_only,
+    rmsnorm_add_bwd,
+    rmsnorm_add_fwd,
     rmsnorm_bwd,
     rmsnorm_fwd,
     workspace,

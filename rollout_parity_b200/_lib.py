@@ -48,7 +48,11 @@ SIGNATURES = {
     "rmsnorm_fwd": (c_i32, [c_i64, c_i32, c_f32, c_f32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp,
                             c_vp, c_vp]),
     "rmsnorm_bwd": (c_i32, [c_i64, c_i32, c_f32, c_f32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp,
-                            c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+                            c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "rmsnorm_add_fwd": (c_i32, [c_i64, c_i32, c_f32, c_f32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp,
+                                c_vp, c_vp, c_vp, c_vp]),
+    "rmsnorm_add_bwd": (c_i32, [c_i64, c_i32, c_f32, c_f32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp,
+                                c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "norm_fwd": (c_i32, [c_i64, c_i32, c_f32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "gated_norm_fwd": (c_i32, [c_i64, c_i32, c_f32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "norm_bwd_workspace_bytes": (c_sz, [c_i64, c_i32]),

@@ -251,11 +251,17 @@ rn_status common_checks(int64_t rows, int32_t width, float eps, rn_dtype dt) {
 }
 
 // inputs: read-only ranges; outputs: written ranges.  Outputs must not overlap
-// anything else; inputs may overlap one another.
-rn_status check_ranges(const Range* in, int nin, const Range* out, int nout) {
+// anything else; inputs may overlap one another.  alias_out / alias_in name
+// one output that may be exactly the given input (same start, same size): an
+// in-place update, which the kernels allow because a thread reads each element
+// before it writes the same element and no other thread touches it.
+rn_status check_ranges(const Range* in, int nin, const Range* out, int nout, int alias_out = -1,
+                       int alias_in = -1) {
   for (int i = 0; i < nout; ++i) {
-    for (int j = 0; j < nin; ++j)
+    for (int j = 0; j < nin; ++j) {
+      if (i == alias_out && j == alias_in && out[i].p == in[j].p && out[i].n == in[j].n) continue;
       if (overlap(out[i], in[j])) return RN_E_ARG;
+    }
     for (int j = i + 1; j < nout; ++j)
       if (overlap(out[i], out[j])) return RN_E_ARG;
   }
@@ -336,10 +342,11 @@ rn_status run_fold(float* a, float* b, int64_t n, int H, float* dw, cudaStream_t
   return RN_OK;
 }
 
+// dres (residual-add backward) may be NULL; dx may be exactly dres.
 rn_status bwd_entry(int64_t rows, int32_t width, float eps, float woff, rn_act act, rn_dtype dt,
                     const void* x, const void* z, const float* w, const void* dy,
-                    const float* rstd, void* dx, void* dz, float* dw, void* ws, size_t ws_bytes,
-                    rn_stream stream) {
+                    const float* rstd, const uint8_t* mask, const void* dres, void* dx, void* dz,
+                    float* dw, void* ws, size_t ws_bytes, rn_stream stream) {
   rn_status e = common_checks(rows, width, eps, dt);
   if (e != RN_OK) return e;
   if (!act_ok(act) || !std::isfinite(woff)) return RN_E_ARG;
@@ -351,7 +358,8 @@ rn_status bwd_entry(int64_t rows, int32_t width, float eps, float woff, rn_act a
   const size_t need = ws_bytes_of(rows, width);
   if (rows > 0) {
     if (!aligned16(x) || !aligned16(dy) || !aligned16(dx) || !aligned16(w) || !aligned16(dw) ||
-        (gated && (!aligned16(z) || !aligned16(dz))) || (uintptr_t(rstd) & 3u))
+        (gated && (!aligned16(z) || !aligned16(dz))) || (uintptr_t(rstd) & 3u) ||
+        !aligned16(dres))
       return RN_E_ALIGN;
     if (!ws || ws_bytes < need) return RN_E_WORKSPACE;
     if (!aligned16(ws)) return RN_E_ALIGN;
@@ -359,10 +367,11 @@ rn_status bwd_entry(int64_t rows, int32_t width, float eps, float woff, rn_act a
     return RN_E_ALIGN;
   }
   const Range in[] = {{x, tb}, {z, tb}, {w, size_t(width) * 4},
-                      {dy, tb}, {rstd, rstd ? size_t(rows) * 4 : 0}};
+                      {dy, tb}, {rstd, rstd ? size_t(rows) * 4 : 0},
+                      {mask, mask ? size_t(rows) : 0}, {dres, tb}};
   const Range out[] = {{dx, tb}, {dz, tb}, {dw, size_t(width) * 4},
                        {ws, rows > 0 ? need : 0}};
-  e = check_ranges(in, 5, out, 4);
+  e = check_ranges(in, 7, out, 4, 0, 6);   // dx may be dres itself
   if (e != RN_OK) return e;
   if (g_validate_only.load()) return RN_OK;
 
@@ -382,35 +391,40 @@ rn_status bwd_entry(int64_t rows, int32_t width, float eps, float woff, rn_act a
   const bool pow2 = (width & (width - 1)) == 0;
   BwdArgs a{rows, width, width / vec_elems(dt), eps, 1.0f / float(width), pow2 ? 1 : 0, woff,
             static_cast<const uint4*>(x), static_cast<const uint4*>(z), w,
-            static_cast<const uint4*>(dy), rstd, static_cast<uint4*>(dx), static_cast<uint4*>(dz),
+            static_cast<const uint4*>(dy), rstd, mask, static_cast<const uint4*>(dres),
+            static_cast<uint4*>(dx), static_cast<uint4*>(dz),
             groups == 1 ? dw : region_a};
   switch (dt) {
-    case RN_BF16: e = launch_bwd<RN_BF16>(act, s, lpc, a, groups, st); break;
-    case RN_F16: e = launch_bwd<RN_F16>(act, s, lpc, a, groups, st); break;
-    default: e = launch_bwd<RN_F32>(act, s, lpc, a, groups, st); break;
+    case RN_BF16: e = launch_bwd<RN_BF16>(act, dres != nullptr, s, lpc, a, groups, st); break;
+    case RN_F16: e = launch_bwd<RN_F16>(act, dres != nullptr, s, lpc, a, groups, st); break;
+    default: e = launch_bwd<RN_F32>(act, dres != nullptr, s, lpc, a, groups, st); break;
   }
   if (e != RN_OK) return e;
   if (groups == 1) return RN_OK;
   return run_fold(region_a, region_b, groups, width, dw, st);
 }
 
+// r, h (residual-add forward): both NULL, or both given; h may be exactly x or r.
 rn_status fwd_entry(int64_t rows, int32_t width, float eps, float woff, rn_act act, rn_dtype dt,
-                    const void* x, const void* z, const float* w, void* y, float* rstd,
-                    rn_stream stream) {
+                    const void* x, const void* r, const void* z, const float* w, void* h, void* y,
+                    float* rstd, rn_stream stream) {
   rn_status e = common_checks(rows, width, eps, dt);
   if (e != RN_OK) return e;
   if (!act_ok(act) || !std::isfinite(woff)) return RN_E_ARG;
   const bool gated = act != RN_ACT_NONE;
   if (!gated && z) return RN_E_ARG;   // no gate: z must be NULL
   if (!w) return RN_E_ARG;
-  if (rows > 0 && (!x || !y || (gated && !z))) return RN_E_ARG;
+  const bool resid = r != nullptr || h != nullptr;
+  if (rows > 0 && (!x || !y || (gated && !z) || (resid && (!r || !h)))) return RN_E_ARG;
   const size_t tb = rows > 0 ? size_t(rows) * size_t(width) * elem_bytes(dt) : 0;
   if (rows > 0 && (!aligned16(x) || !aligned16(y) || !aligned16(w) ||
-                   (gated && !aligned16(z)) || (uintptr_t(rstd) & 3u)))
+                   (gated && !aligned16(z)) || (uintptr_t(rstd) & 3u) ||
+                   !aligned16(r) || !aligned16(h)))
     return RN_E_ALIGN;
-  const Range in[] = {{x, tb}, {z, tb}, {w, size_t(width) * 4}};
-  const Range out[] = {{y, tb}, {rstd, rstd ? size_t(rows) * 4 : 0}};
-  e = check_ranges(in, 3, out, 2);
+  const Range in[] = {{x, tb}, {z, tb}, {w, size_t(width) * 4}, {r, tb}};
+  const Range out[] = {{y, tb}, {rstd, rstd ? size_t(rows) * 4 : 0}, {h, tb}};
+  // h may be exactly x or exactly r (an in-place residual update)
+  e = check_ranges(in, 4, out, 3, 2, h != nullptr && h == x ? 0 : 3);
   if (e != RN_OK) return e;
   if (g_validate_only.load() || rows == 0) return RN_OK;
   Sched s;
@@ -418,12 +432,12 @@ rn_status fwd_entry(int64_t rows, int32_t width, float eps, float woff, rn_act a
   const bool pow2 = (width & (width - 1)) == 0;
   FwdArgs a{rows, width, width / vec_elems(dt), eps, 1.0f / float(width), pow2 ? 1 : 0, woff,
             static_cast<const uint4*>(x), static_cast<const uint4*>(z), w,
-            static_cast<uint4*>(y), rstd};
+            static_cast<uint4*>(y), rstd, static_cast<const uint4*>(r), static_cast<uint4*>(h)};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (dt) {
-    case RN_BF16: return launch_fwd<RN_BF16>(act, s, a, st);
-    case RN_F16: return launch_fwd<RN_F16>(act, s, a, st);
-    default: return launch_fwd<RN_F32>(act, s, a, st);
+    case RN_BF16: return launch_fwd<RN_BF16>(act, resid, s, a, st);
+    case RN_F16: return launch_fwd<RN_F16>(act, resid, s, a, st);
+    default: return launch_fwd<RN_F32>(act, resid, s, a, st);
   }
 }
 
@@ -496,13 +510,13 @@ size_t bwd_stripe_smem_bytes(const Sched& s, int width, bool gated, rn_dtype dt)
 }
 
 // Dynamic shared memory of k_fwd (the kernel's layout).
-size_t fwd_smem_bytes(const Sched& s, bool gated, rn_dtype dt) {
+size_t fwd_smem_bytes(const Sched& s, bool gated, bool resid, rn_dtype dt) {
   const size_t VE = size_t(vec_elems(dt));
   const size_t B = fwd_block_of(s.T, s.K), NT = B / s.T;
   const size_t W = s.T > 32 ? s.T / 32 : 1;
   const size_t red = s.T > 32 ? 2 * NT * W * sizeof(float) : 0;
   const size_t gain = s.T <= 16 ? size_t(s.K) * s.T * VE * sizeof(float) : 0;
-  return red + gain + size_t(fwd_stages_of(s.T)) * (gated ? 2 : 1) * s.K * B * 16;
+  return red + gain + size_t(fwd_stages_of(s.T)) * (1 + gated + resid) * s.K * B * 16;
 }
 
 }  // namespace rn_detail
@@ -515,25 +529,44 @@ extern "C" {
 rn_status rmsnorm_fwd(int64_t rows, int32_t width, float eps, float weight_offset, rn_act act,
                       rn_dtype dt, const void* x, const void* z, const float* w, void* y,
                       float* rstd, rn_stream stream) {
-  return fwd_entry(rows, width, eps, weight_offset, act, dt, x, z, w, y, rstd, stream);
+  return fwd_entry(rows, width, eps, weight_offset, act, dt, x, nullptr, z, w, nullptr, y, rstd,
+                   stream);
+}
+
+rn_status rmsnorm_add_fwd(int64_t rows, int32_t width, float eps, float weight_offset,
+                          rn_act act, rn_dtype dt, const void* x, const void* r, const void* z,
+                          const float* w, void* h, void* y, float* rstd, rn_stream stream) {
+  if (rows > 0 && (!r || !h)) return RN_E_ARG;
+  return fwd_entry(rows, width, eps, weight_offset, act, dt, x, r, z, w, h, y, rstd, stream);
+}
+
+rn_status rmsnorm_add_bwd(int64_t rows, int32_t width, float eps, float weight_offset,
+                          rn_act act, rn_dtype dt, const void* h, const void* z, const float* w,
+                          const void* dy, const void* dh, const float* rstd,
+                          const uint8_t* row_mask, void* dx, void* dz, float* dw, void* ws,
+                          size_t ws_bytes, rn_stream stream) {
+  return bwd_entry(rows, width, eps, weight_offset, act, dt, h, z, w, dy, rstd, row_mask, dh, dx,
+                   dz, dw, ws, ws_bytes, stream);
 }
 
 rn_status rmsnorm_bwd(int64_t rows, int32_t width, float eps, float weight_offset, rn_act act,
                       rn_dtype dt, const void* x, const void* z, const float* w, const void* dy,
-                      const float* rstd, void* dx, void* dz, float* dw, void* ws,
-                      size_t ws_bytes, rn_stream stream) {
-  return bwd_entry(rows, width, eps, weight_offset, act, dt, x, z, w, dy, rstd, dx, dz, dw, ws,
-                   ws_bytes, stream);
+                      const float* rstd, const uint8_t* row_mask, void* dx, void* dz, float* dw,
+                      void* ws, size_t ws_bytes, rn_stream stream) {
+  return bwd_entry(rows, width, eps, weight_offset, act, dt, x, z, w, dy, rstd, row_mask, nullptr,
+                   dx, dz, dw, ws, ws_bytes, stream);
 }
 
 rn_status norm_fwd(int64_t rows, int32_t width, float eps, rn_dtype dt, const void* x,
                    const float* w, void* y, float* rstd, rn_stream stream) {
-  return fwd_entry(rows, width, eps, 1.0f, RN_ACT_NONE, dt, x, nullptr, w, y, rstd, stream);
+  return fwd_entry(rows, width, eps, 1.0f, RN_ACT_NONE, dt, x, nullptr, nullptr, w, nullptr, y,
+                   rstd, stream);
 }
 
 rn_status gated_norm_fwd(int64_t rows, int32_t width, float eps, rn_dtype dt, const void* x,
                          const void* z, const float* w, void* y, float* rstd, rn_stream stream) {
-  return fwd_entry(rows, width, eps, 0.0f, RN_ACT_SILU, dt, x, z, w, y, rstd, stream);
+  return fwd_entry(rows, width, eps, 0.0f, RN_ACT_SILU, dt, x, nullptr, z, w, nullptr, y, rstd,
+                   stream);
 }
 
 size_t norm_bwd_workspace_bytes(int64_t rows, int32_t width) { return ws_bytes_of(rows, width); }
@@ -541,16 +574,16 @@ size_t norm_bwd_workspace_bytes(int64_t rows, int32_t width) { return ws_bytes_o
 rn_status norm_bwd(int64_t rows, int32_t width, float eps, rn_dtype dt, const void* x,
                    const float* w, const void* dy, const float* rstd, void* dx, float* dw,
                    void* ws, size_t ws_bytes, rn_stream stream) {
-  return bwd_entry(rows, width, eps, 1.0f, RN_ACT_NONE, dt, x, nullptr, w, dy, rstd, dx, nullptr,
-                   dw, ws, ws_bytes, stream);
+  return bwd_entry(rows, width, eps, 1.0f, RN_ACT_NONE, dt, x, nullptr, w, dy, rstd, nullptr,
+                   nullptr, dx, nullptr, dw, ws, ws_bytes, stream);
 }
 
 rn_status gated_norm_bwd(int64_t rows, int32_t width, float eps, rn_dtype dt, const void* x,
                          const void* z, const float* w, const void* dy, const float* rstd,
                          void* dx, void* dz, float* dw, void* ws, size_t ws_bytes,
                          rn_stream stream) {
-  return bwd_entry(rows, width, eps, 0.0f, RN_ACT_SILU, dt, x, z, w, dy, rstd, dx, dz, dw, ws,
-                   ws_bytes, stream);
+  return bwd_entry(rows, width, eps, 0.0f, RN_ACT_SILU, dt, x, z, w, dy, rstd, nullptr, nullptr,
+                   dx, dz, dw, ws, ws_bytes, stream);
 }
 
 rn_status rn_fold_rows(int64_t n, int32_t width, const float* in, float* out, rn_stream stream) {
@@ -703,6 +736,6 @@ extern "C" rn_status gated_norm_bwd_static_ws(int64_t rows, int32_t width, float
       if (e != RN_OK) return e;
     }
   }
-  return bwd_entry(rows, width, eps, 0.0f, RN_ACT_SILU, dt, x, z, w, dy, rstd, dx, dz, dw, ws,
-                   kStaticScratchBytes, stream);
+  return bwd_entry(rows, width, eps, 0.0f, RN_ACT_SILU, dt, x, z, w, dy, rstd, nullptr, nullptr,
+                   dx, dz, dw, ws, kStaticScratchBytes, stream);
 }

@@ -39,6 +39,8 @@ struct FwdArgs {
   const float* w;
   uint4* y;
   float* rstd;
+  const uint4* r;   // residual-add forward: h = fmt(x + r) is normalised ...
+  uint4* h;         // ... and stored here
 };
 
 struct BwdArgs {
@@ -52,6 +54,8 @@ struct BwdArgs {
   const float* w;
   const uint4* dy;
   const float* rstd;
+  const uint8_t* mask;   // rows with mask[r] == 0 add nothing to dw (NULL: every row)
+  const uint4* dres;     // residual-add backward: dx = dnorm + dres (one rounding)
   uint4* dx;
   uint4* dz;
   float* part;      // [groups][H] fp32 group partials (or dw when one group)
@@ -104,16 +108,16 @@ int sm_count();
 int grid_cap(int64_t want);
 rn_status launch_status();   // RN_OK, or RN_E_CUDA with the error recorded
 // dynamic shared memory of k_fwd / k_bwd (their layouts)
-size_t fwd_smem_bytes(const Sched& s, bool gated, rn_dtype dt);
+size_t fwd_smem_bytes(const Sched& s, bool gated, bool resid, rn_dtype dt);
 size_t bwd_smem_bytes(const Sched& s, int lpc, int width, bool gated, rn_dtype dt);
 size_t bwd_stripe_smem_bytes(const Sched& s, int width, bool gated, rn_dtype dt);
 
 // ---- row kernels, one instantiation per element format (rows_*.cu) ------------
 template <int DT>
-rn_status launch_fwd(int act, const Sched& s, const FwdArgs& a, cudaStream_t st);
+rn_status launch_fwd(int act, bool resid, const Sched& s, const FwdArgs& a, cudaStream_t st);
 template <int DT>
-rn_status launch_bwd(int act, const Sched& s, int lpc, const BwdArgs& a, int64_t groups,
-                     cudaStream_t st);
+rn_status launch_bwd(int act, bool resid, const Sched& s, int lpc, const BwdArgs& a,
+                     int64_t groups, cudaStream_t st);
 
 // Lets `kernel` use `smem` bytes of dynamic shared memory (the default limit is
 // 48 KB) and returns how many of its CTAs fit on one SM.  `done` and `per_sm`

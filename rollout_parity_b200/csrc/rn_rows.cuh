@@ -412,14 +412,17 @@ __device__ __forceinline__ void cp_async_wait() {
 // rows (c + i*grid)*NT + j.  Per row: sum of squares, the team reduction,
 // rstd, the epilogue, y and rstd stores.
 // ---------------------------------------------------------------------------
-template <int DT, int T, int K, int ACT, bool EXACT>
+// RESID: the residual-add forward; x and r are staged, h = fmt(x + r) (fp32
+// sum, one rounding) is stored and takes x's place.
+template <int DT, int T, int K, int ACT, bool EXACT, bool RESID>
 __global__ void __launch_bounds__(fwd_block_of(T, K), fwd_min_blocks_of(T, K))
 k_fwd(const FwdArgs a) {
   using F = Fmt<DT>;
   constexpr bool GATED = ACT != kActNone;
   constexpr int VE = F::VE;
   constexpr int S = fwd_stages_of(T);
-  constexpr int NTEN = GATED ? 2 : 1;   // staged tensors: x (, z)
+  constexpr int NTEN = 1 + GATED + RESID;   // staged tensors: x (, z) (, r)
+  constexpr int TR = GATED ? 2 : 1;         // slot of r
   constexpr int B = fwd_block_of(T, K);
   constexpr int NT = B / T;
   constexpr int W = T > 32 ? T / 32 : 1;
@@ -456,6 +459,7 @@ k_fwd(const FwdArgs a) {
           if (EXACT || k * T + t < nv) {
             cp_async16(slot(sl, 0, k), a.x + off + k * T);
             if constexpr (GATED) cp_async16(slot(sl, 1, k), a.z + off + k * T);
+            if constexpr (RESID) cp_async16(slot(sl, TR, k), a.r + off + k * T);
           }
         }
       }
@@ -481,6 +485,18 @@ k_fwd(const FwdArgs a) {
     }
     const int64_t row = row_of(i);
     const bool act = row < a.rows;
+    if constexpr (RESID) {   // h = fmt(x + r): the stored value is what is normalised
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        float2 xf[VE / 2], rf[VE / 2];
+        F::unpack2(xr[k], xf);
+        F::unpack2(*slot(sl, TR, k), rf);
+#pragma unroll
+        for (int q = 0; q < VE / 2; ++q) xf[q] = add2(xf[q], rf[q]);
+        xr[k] = F::pack2v(xf);
+        if (act && (EXACT || k * T + t < nv)) st_stream(a.h + row * nv + t + k * T, xr[k]);
+      }
+    }
     float ss[1] = {thread_sumsq<DT, T, K, EXACT>(xr, nv, t)};
     team_sum<T, 1>(ss, red, phase, team, NT, mask);
     const float r = rsqrtf(__fadd_rn(mean_of(ss[0], a.H, a.inv_h, a.h_pow2), a.eps));
@@ -521,7 +537,7 @@ k_fwd(const FwdArgs a) {
 // call it in lockstep.
 //   g = u * a(z);  m = mean(g * dy * xh);  dx = rstd * (g*dy - xh*m)
 //   dz = dy * xh * u * a'(z)
-template <int DT, int T, int K, int ACT, bool EXACT, typename G>
+template <int DT, int T, int K, int ACT, bool EXACT, bool RESID, typename G>
 __device__ __forceinline__ void bwd_row(const BwdArgs& a, const G& gain, const uint4 (&xr)[K],
                                         const uint4 (&dr)[K], const uint4 (&zr)[K],
                                         float rs_staged, bool have_rstd, int64_t row, bool act,
@@ -531,6 +547,12 @@ __device__ __forceinline__ void bwd_row(const BwdArgs& a, const G& gain, const u
   constexpr bool GATED = ACT != kActNone;
   constexpr int VE = F::VE;
   const int nv = a.nv;
+  uint4 rv[RESID ? K : 1];   // dres of this row, loaded early to hide its latency
+  if constexpr (RESID) {
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+      if (act && (EXACT || k * T + t < nv)) rv[k] = __ldcs(a.dres + row * nv + t + k * T);
+  }
   float rs = rs_staged;
   if (!have_rstd) {   // uniform branch
     float ss[1] = {thread_sumsq<DT, T, K, EXACT>(xr, nv, t)};
@@ -589,6 +611,12 @@ __device__ __forceinline__ void bwd_row(const BwdArgs& a, const G& gain, const u
           d[k][q] = qv;
         }
       }
+      if constexpr (RESID) {   // dx = dnorm + dres, rounded once
+        float2 rf[VE / 2];
+        F::unpack2(rv[k], rf);
+#pragma unroll
+        for (int q = 0; q < VE / 2; ++q) dxv[q] = add2(dxv[q], rf[q]);
+      }
       st_stream(a.dx + off + k * T, F::pack2v(dxv));
       if constexpr (GATED) st_stream(a.dz + off + k * T, F::pack2v(dzv));
     }
@@ -603,7 +631,7 @@ __device__ __forceinline__ void bwd_row(const BwdArgs& a, const G& gain, const u
 //   g = u * a(z);  m = mean(g * dy * xh);  dx = rstd * (g*dy - xh*m)
 //   dz = dy * xh * u * a'(z);  dw leaf += dy * xh * a(z)
 // ---------------------------------------------------------------------------
-template <int DT, int T, int K, int ACT, bool EXACT>
+template <int DT, int T, int K, int ACT, bool EXACT, bool RESID>
 __global__ void __launch_bounds__(bwd_max_block_of(T), bwd_min_blocks_of(T, K))
 k_bwd(const BwdArgs a) {
   using F = Fmt<DT>;
@@ -685,9 +713,10 @@ k_bwd(const BwdArgs a) {
         if constexpr (GATED) zr[k] = *slot(sl, 2, k);
       }
       float2 d[K][VE / 2];
-      bwd_row<DT, T, K, ACT, EXACT>(a, gain, xr, dr, zr, have_rstd ? rsm[sl * bd + tid] : 0.0f,
+      bwd_row<DT, T, K, ACT, EXACT, RESID>(a, gain, xr, dr, zr,
+                                          have_rstd ? rsm[sl * bd + tid] : 0.0f,
                                    have_rstd, row, act, t, red, phase, team, NT, mask, d);
-      if (act) {
+      if (act && (a.mask == nullptr || __ldg(a.mask + row) != 0)) {   // masked rows add nothing
 #pragma unroll
         for (int k = 0; k < K; ++k) {
           if (EXACT || k * T + t < nv) {
@@ -720,7 +749,7 @@ k_bwd(const BwdArgs a) {
 // pending subtrees (the level-by-level pairwise tree), whose root is the group
 // partial.  Same bits as k_bwd.
 // ---------------------------------------------------------------------------
-template <int DT, int T, int K, int ACT>
+template <int DT, int T, int K, int ACT, bool RESID>
 __global__ void __launch_bounds__(32, bwd_min_blocks_of(T, K))
 k_bwd_stripe(const BwdArgs a, int lpc) {
   using F = Fmt<DT>;
@@ -802,7 +831,8 @@ k_bwd_stripe(const BwdArgs a, int lpc) {
         if constexpr (GATED) zr[k] = *slot(sl, 2, k);
       }
       float2 d[K][VE / 2];
-      bwd_row<DT, T, K, ACT, true>(a, gain, xr, dr, zr, have_rstd ? rsm[sl * 32 + tid] : 0.0f,
+      bwd_row<DT, T, K, ACT, true, RESID>(a, gain, xr, dr, zr,
+                                           have_rstd ? rsm[sl * 32 + tid] : 0.0f,
                                   have_rstd, row, act, t, nullptr, phase, team, RPS, 0xffffffffu,
                                   d);
       // transpose the step's contributions: row `team` of the buffer
@@ -820,7 +850,8 @@ k_bwd_stripe(const BwdArgs a, int lpc) {
       const int64_t step_row = base + int64_t(st) * RPS;
 #pragma unroll
       for (int r = 0; r < RPS; ++r) {
-        if (step_row + r < a.rows) {   // rows past the batch contribute nothing
+        // rows past the batch or outside the mask contribute nothing
+        if (step_row + r < a.rows && (a.mask == nullptr || __ldg(a.mask + step_row + r) != 0)) {
           const float4* src = reinterpret_cast<const float4*>(tbuf + r * TS);
 #pragma unroll
           for (int c = 0; c < C4; ++c) lacc[c] = add4(lacc[c], src[c * 32 + tid]);
@@ -846,38 +877,39 @@ k_bwd_stripe(const BwdArgs a, int lpc) {
 // pick_sched can return for each element size
 // ---------------------------------------------------------------------------
 // The forward is persistent: one wave of CTAs (as many as fit on every SM).
-template <int DT, int T, int K, int ACT, bool EXACT>
+template <int DT, int T, int K, int ACT, bool EXACT, bool RESID>
 rn_status launch_fwd_tk(const Sched& s, const FwdArgs& a, cudaStream_t st) {
   constexpr int B = fwd_block_of(T, K);
-  const size_t smem = fwd_smem_bytes(s, ACT != kActNone, rn_dtype(DT));
+  const size_t smem = fwd_smem_bytes(s, ACT != kActNone, RESID, rn_dtype(DT));
   static std::atomic<size_t> done{0};
   static std::atomic<int> per_sm{0};
-  const int nb = prepare_kernel(k_fwd<DT, T, K, ACT, EXACT>, B, smem, done, per_sm);
+  const int nb = prepare_kernel(k_fwd<DT, T, K, ACT, EXACT, RESID>, B, smem, done, per_sm);
   const int64_t nblk = (a.rows + B / T - 1) / (B / T);
   const int64_t wave = int64_t(nb) * sm_count();
   const int grid = grid_cap(nblk < wave ? nblk : wave);
-  return launch_pdl(k_fwd<DT, T, K, ACT, EXACT>, dim3(grid), dim3(B), smem, st, a);
+  return launch_pdl(k_fwd<DT, T, K, ACT, EXACT, RESID>, dim3(grid), dim3(B), smem, st, a);
 }
 
 // The backward runs one CTA per group of leaves (grid-stride if capped).
-template <int DT, int T, int K, int ACT, bool EXACT>
+template <int DT, int T, int K, int ACT, bool EXACT, bool RESID>
 rn_status launch_bwd_tk(const Sched& s, int lpc, const BwdArgs& a, int64_t groups,
                         cudaStream_t st) {
   if constexpr (stripe_shape(T, K, Fmt<DT>::VE, EXACT)) {
     const size_t smem = bwd_stripe_smem_bytes(s, a.H, ACT != kActNone, rn_dtype(DT));
     static std::atomic<size_t> done{0};
     static std::atomic<int> per_sm{0};
-    (void)prepare_kernel(k_bwd_stripe<DT, T, K, ACT>, 32, smem, done, per_sm);
-    return launch_pdl(k_bwd_stripe<DT, T, K, ACT>, dim3(grid_cap(groups)), dim3(32), smem, st,
-                      a, lpc);
+    (void)prepare_kernel(k_bwd_stripe<DT, T, K, ACT, RESID>, 32, smem, done, per_sm);
+    return launch_pdl(k_bwd_stripe<DT, T, K, ACT, RESID>, dim3(grid_cap(groups)), dim3(32), smem,
+                      st, a, lpc);
+  } else {   // (k_bwd is not instantiated for the stripe shapes)
+    const int block = lpc * T;
+    const size_t smem = bwd_smem_bytes(s, lpc, a.H, ACT != kActNone, rn_dtype(DT));
+    static std::atomic<size_t> done{0};
+    static std::atomic<int> per_sm{0};
+    (void)prepare_kernel(k_bwd<DT, T, K, ACT, EXACT, RESID>, block, smem, done, per_sm);
+    return launch_pdl(k_bwd<DT, T, K, ACT, EXACT, RESID>, dim3(grid_cap(groups)), dim3(block),
+                      smem, st, a);
   }
-  const int block = lpc * T;
-  const size_t smem = bwd_smem_bytes(s, lpc, a.H, ACT != kActNone, rn_dtype(DT));
-  static std::atomic<size_t> done{0};
-  static std::atomic<int> per_sm{0};
-  (void)prepare_kernel(k_bwd<DT, T, K, ACT, EXACT>, block, smem, done, per_sm);
-  return launch_pdl(k_bwd<DT, T, K, ACT, EXACT>, dim3(grid_cap(groups)), dim3(block), smem,
-                    st, a);
 }
 
 // (T, K, exact) shapes reachable for widths 8..16384 (multiples of 8):
@@ -905,11 +937,11 @@ rn_status launch_bwd_tk(const Sched& s, int lpc, const BwdArgs& a, int64_t group
   X(1024, 3, false) X(1024, 3, true) X(1024, 4, false) X(1024, 4, true)                         \
   X(128, 5, true) X(256, 3, true) X(256, 5, true)
 
-template <int DT, int ACT>
+template <int DT, int ACT, bool RESID>
 rn_status launch_fwd_act(const Sched& s, const FwdArgs& a, cudaStream_t st) {
   const bool ex = a.nv == s.T * s.K;
 #define RN_FWD_CASE(T_, K_, EX_) \
-  if (s.T == T_ && s.K == K_ && ex == EX_) return launch_fwd_tk<DT, T_, K_, ACT, EX_>(s, a, st);
+  if (s.T == T_ && s.K == K_ && ex == EX_) return launch_fwd_tk<DT, T_, K_, ACT, EX_, RESID>(s, a, st);
   if constexpr (DT == RN_F32) {
     RN_SHAPES_32(RN_FWD_CASE)
   } else {
@@ -919,13 +951,13 @@ rn_status launch_fwd_act(const Sched& s, const FwdArgs& a, cudaStream_t st) {
   return RN_E_WIDTH;
 }
 
-template <int DT, int ACT>
+template <int DT, int ACT, bool RESID>
 rn_status launch_bwd_act(const Sched& s, int lpc, const BwdArgs& a, int64_t groups,
                          cudaStream_t st) {
   const bool ex = a.nv == s.T * s.K;
 #define RN_BWD_CASE(T_, K_, EX_)                \
   if (s.T == T_ && s.K == K_ && ex == EX_)      \
-    return launch_bwd_tk<DT, T_, K_, ACT, EX_>(s, lpc, a, groups, st);
+    return launch_bwd_tk<DT, T_, K_, ACT, EX_, RESID>(s, lpc, a, groups, st);
   if constexpr (DT == RN_F32) {
     RN_SHAPES_32(RN_BWD_CASE)
   } else {
@@ -935,25 +967,37 @@ rn_status launch_bwd_act(const Sched& s, int lpc, const BwdArgs& a, int64_t grou
   return RN_E_WIDTH;
 }
 
-template <int DT>
-rn_status launch_fwd(int act, const Sched& s, const FwdArgs& a, cudaStream_t st) {
+template <int DT, bool RESID>
+rn_status launch_fwd_r(int act, const Sched& s, const FwdArgs& a, cudaStream_t st) {
   switch (act) {
-    case kActNone: return launch_fwd_act<DT, kActNone>(s, a, st);
-    case kActSilu: return launch_fwd_act<DT, kActSilu>(s, a, st);
-    case kActSigmoid: return launch_fwd_act<DT, kActSigmoid>(s, a, st);
+    case kActNone: return launch_fwd_act<DT, kActNone, RESID>(s, a, st);
+    case kActSilu: return launch_fwd_act<DT, kActSilu, RESID>(s, a, st);
+    case kActSigmoid: return launch_fwd_act<DT, kActSigmoid, RESID>(s, a, st);
     default: return RN_E_ARG;
   }
 }
 
 template <int DT>
-rn_status launch_bwd(int act, const Sched& s, int lpc, const BwdArgs& a, int64_t groups,
-                     cudaStream_t st) {
+rn_status launch_fwd(int act, bool resid, const Sched& s, const FwdArgs& a, cudaStream_t st) {
+  return resid ? launch_fwd_r<DT, true>(act, s, a, st) : launch_fwd_r<DT, false>(act, s, a, st);
+}
+
+template <int DT, bool RESID>
+rn_status launch_bwd_r(int act, const Sched& s, int lpc, const BwdArgs& a, int64_t groups,
+                       cudaStream_t st) {
   switch (act) {
-    case kActNone: return launch_bwd_act<DT, kActNone>(s, lpc, a, groups, st);
-    case kActSilu: return launch_bwd_act<DT, kActSilu>(s, lpc, a, groups, st);
-    case kActSigmoid: return launch_bwd_act<DT, kActSigmoid>(s, lpc, a, groups, st);
+    case kActNone: return launch_bwd_act<DT, kActNone, RESID>(s, lpc, a, groups, st);
+    case kActSilu: return launch_bwd_act<DT, kActSilu, RESID>(s, lpc, a, groups, st);
+    case kActSigmoid: return launch_bwd_act<DT, kActSigmoid, RESID>(s, lpc, a, groups, st);
     default: return RN_E_ARG;
   }
+}
+
+template <int DT>
+rn_status launch_bwd(int act, bool resid, const Sched& s, int lpc, const BwdArgs& a,
+                     int64_t groups, cudaStream_t st) {
+  return resid ? launch_bwd_r<DT, true>(act, s, lpc, a, groups, st)
+               : launch_bwd_r<DT, false>(act, s, lpc, a, groups, st);
 }
 
 }  // namespace rn_detail

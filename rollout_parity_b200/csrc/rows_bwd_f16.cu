@@ -4,5 +4,6 @@
 #include "rn_rows.cuh"
 
 namespace rn_detail {
-template rn_status launch_bwd<RN_F16>(int, const Sched&, int, const BwdArgs&, int64_t, cudaStream_t);
+template rn_status launch_bwd<RN_F16>(int, bool, const Sched&, int, const BwdArgs&, int64_t,
+                                        cudaStream_t);
 }  // namespace rn_detail

@@ -4,5 +4,5 @@
 #include "rn_rows.cuh"
 
 namespace rn_detail {
-template rn_status launch_fwd<RN_F32>(int, const Sched&, const FwdArgs&, cudaStream_t);
+template rn_status launch_fwd<RN_F32>(int, bool, const Sched&, const FwdArgs&, cudaStream_t);
 }  // namespace rn_detail

@@ -114,6 +114,77 @@ def rmsnorm_fwd(x: torch.Tensor, w: torch.Tensor, eps: float = 1e-6, weight_offs
     return y, rstd
 
 
+def rmsnorm_add_fwd(x: torch.Tensor, r: torch.Tensor, w: torch.Tensor, eps: float = 1e-6,
+                    weight_offset: float = 1.0, z: Optional[torch.Tensor] = None, act=None, *,
+                    h: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                    rstd: Optional[torch.Tensor] = None, want_rstd: bool = True, stream=None):
+    """Residual-add forward: h = x + r (rounded once to x's dtype) and the norm
+    of h.  Returns (h, y, rstd).  h may be x or r itself (in place)."""
+    rows, width = _rows_width(x)
+    a = act_code(act)
+    _mat("r", r, x)
+    if a == Act.NONE:
+        if z is not None:
+            raise ValueError("z given without a gate activation")
+    else:
+        _mat("z", z, x)
+    _vec("w", w, width, x.device)
+    h = torch.empty_like(x) if h is None else _mat("h", h, x)
+    y = torch.empty_like(x) if y is None else _mat("y", y, x)
+    if rstd is None and want_rstd:
+        rstd = torch.empty(rows, dtype=torch.float32, device=x.device)
+    if rstd is not None:
+        _vec("rstd", rstd, rows, x.device)
+    with torch.cuda.device(x.device):
+        check("rmsnorm_add_fwd",
+              load().rmsnorm_add_fwd(rows, width, eps, weight_offset, int(a), _dt(x), _ptr(x),
+                                     _ptr(r), _ptr(z), _ptr(w), _ptr(h), _ptr(y), _ptr(rstd),
+                                     _stream(x, stream)))
+    return h, y, rstd
+
+
+def rmsnorm_add_bwd(h: torch.Tensor, w: torch.Tensor, dy: torch.Tensor,
+                    dh: Optional[torch.Tensor] = None, rstd: Optional[torch.Tensor] = None,
+                    eps: float = 1e-6, weight_offset: float = 1.0,
+                    z: Optional[torch.Tensor] = None, act=None, *,
+                    row_mask: Optional[torch.Tensor] = None,
+                    dx: Optional[torch.Tensor] = None, dz: Optional[torch.Tensor] = None,
+                    dw: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                    stream=None):
+    """Residual-add backward: the norm's gradient at h plus dh (the gradient
+    of the residual output), the gradient of both x and r.  Returns (dx, dz, dw)."""
+    rows, width = _rows_width(h)
+    a = act_code(act)
+    if a == Act.NONE:
+        if z is not None or dz is not None:
+            raise ValueError("z or dz given without a gate activation")
+    else:
+        _mat("z", z, h)
+        dz = torch.empty_like(h) if dz is None else _mat("dz", dz, h)
+    _vec("w", w, width, h.device)
+    _mat("dy", dy, h)
+    if dh is not None:
+        _mat("dh", dh, h)
+    if rstd is not None:
+        _vec("rstd", rstd, rows, h.device)
+    if row_mask is not None:
+        if row_mask.dtype not in (torch.bool, torch.uint8) or tuple(row_mask.shape) != (rows,) \
+                or row_mask.device != h.device or not row_mask.is_contiguous():
+            raise ValueError(f"row_mask must be a contiguous bool/uint8 [{rows}] tensor on {h.device}")
+        row_mask = row_mask.view(torch.uint8)
+    dx = torch.empty_like(h) if dx is None else _mat("dx", dx, h)
+    dw = torch.empty(width, dtype=torch.float32, device=h.device) if dw is None else \
+        _vec("dw", dw, width, h.device)
+    ws, nws = _ws(rows, width, h.device, ws)
+    with torch.cuda.device(h.device):
+        check("rmsnorm_add_bwd",
+              load().rmsnorm_add_bwd(rows, width, eps, weight_offset, int(a), _dt(h), _ptr(h),
+                                     _ptr(z), _ptr(w), _ptr(dy), _ptr(dh), _ptr(rstd),
+                                     _ptr(row_mask), _ptr(dx), _ptr(dz), _ptr(dw), _ptr(ws), nws,
+                                     _stream(h, stream)))
+    return dx, dz, dw
+
+
 def norm_fwd(x: torch.Tensor, w: torch.Tensor, eps: float = 1e-6, *,
              y: Optional[torch.Tensor] = None, rstd: Optional[torch.Tensor] = None,
              want_rstd: bool = True, stream=None):
@@ -162,11 +233,13 @@ def _ws(rows, width, device, ws):
 def rmsnorm_bwd(x: torch.Tensor, w: torch.Tensor, dy: torch.Tensor,
                 rstd: Optional[torch.Tensor] = None, eps: float = 1e-6, weight_offset: float = 1.0,
                 z: Optional[torch.Tensor] = None, act=None, *,
+                row_mask: Optional[torch.Tensor] = None,
                 dx: Optional[torch.Tensor] = None, dz: Optional[torch.Tensor] = None,
                 dw: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
                 stream=None):
     """General backward.  Returns (dx, dz, dw); dz is None without a gate.
-    rstd=None recomputes it."""
+    rstd=None recomputes it.  row_mask ([rows] bool or uint8): rows where it is
+    zero are left out of dw (dx and dz are still every row's)."""
     rows, width = _rows_width(x)
     a = act_code(act)
     if a == Act.NONE:
@@ -179,6 +252,11 @@ def rmsnorm_bwd(x: torch.Tensor, w: torch.Tensor, dy: torch.Tensor,
     _mat("dy", dy, x)
     if rstd is not None:
         _vec("rstd", rstd, rows, x.device)
+    if row_mask is not None:
+        if row_mask.dtype not in (torch.bool, torch.uint8) or tuple(row_mask.shape) != (rows,) \
+                or row_mask.device != x.device or not row_mask.is_contiguous():
+            raise ValueError(f"row_mask must be a contiguous bool/uint8 [{rows}] tensor on {x.device}")
+        row_mask = row_mask.view(torch.uint8)
     dx = torch.empty_like(x) if dx is None else _mat("dx", dx, x)
     dw = torch.empty(width, dtype=torch.float32, device=x.device) if dw is None else \
         _vec("dw", dw, width, x.device)
@@ -186,8 +264,8 @@ def rmsnorm_bwd(x: torch.Tensor, w: torch.Tensor, dy: torch.Tensor,
     with torch.cuda.device(x.device):
         check("rmsnorm_bwd",
               load().rmsnorm_bwd(rows, width, eps, weight_offset, int(a), _dt(x), _ptr(x), _ptr(z),
-                                 _ptr(w), _ptr(dy), _ptr(rstd), _ptr(dx), _ptr(dz), _ptr(dw),
-                                 _ptr(ws), nws, _stream(x, stream)))
+                                 _ptr(w), _ptr(dy), _ptr(rstd), _ptr(row_mask), _ptr(dx),
+                                 _ptr(dz), _ptr(dw), _ptr(ws), nws, _stream(x, stream)))
     return dx, dz, dw
 
 

@@ -205,8 +205,8 @@ def rbwd(lib, rows=R, width=H, eps=1e-6, woff=1.0, act=Act.SIGMOID, dt=DType.BF1
     ptr.update(kw)
     nws = lib.norm_bwd_workspace_bytes(rows, width)
     return lib.rmsnorm_bwd(rows, width, eps, woff, act, dt, ptr["x"], ptr["z"], ptr["w"],
-                           ptr["dy"], ptr["rstd"], ptr["dx"], ptr["dz"], ptr["dw"], ptr["ws"],
-                           nws, None)
+                           ptr["dy"], ptr["rstd"], ptr.get("mask"), ptr["dx"], ptr["dz"],
+                           ptr["dw"], ptr["ws"], nws, None)
 
 
 GENERAL_CASES = [
@@ -227,6 +227,21 @@ GENERAL_CASES = [
     ("y aliases z", dict(y=P(Z), dx=P(Z)), Status.E_ARG),
     ("rows 0", dict(rows=0, x=0, z=0, y=0, dy=0, dx=0, dz=0, ws=0, rstd=0), Status.OK),
 ]
+
+
+MASK_CASES = [
+    ("row mask", dict(mask=P(10)), Status.OK),
+    ("row mask unaligned is fine", dict(mask=P(10, 3)), Status.OK),
+    ("row mask inside dx", dict(mask=P(DX, 64)), Status.E_ARG),
+    ("row mask over ws", dict(mask=P(WS, 16)), Status.E_ARG),
+    ("row mask may share x", dict(mask=P(X, 64)), Status.OK),
+]
+
+
+@pytest.mark.parametrize("name,kw,want", MASK_CASES, ids=[c[0] for c in MASK_CASES])
+def test_row_mask_checks(lib, name, kw, want):
+    with validate_only(lib):
+        assert rbwd(lib, **kw) == want
 
 
 @pytest.mark.parametrize("name,kw,want", GENERAL_CASES, ids=[c[0] for c in GENERAL_CASES])
@@ -252,6 +267,61 @@ def test_binding_activation_names():
     assert rn.act_code("SiLU") == Act.SILU and rn.act_code("sigmoid") == Act.SIGMOID
     with pytest.raises(ValueError):
         rn.act_code("gelu")
+
+
+HH, RR, DH = 11, 12, 13
+
+
+def afwd(lib, rows=R, width=H, act=Act.SILU, **kw):
+    ptr = dict(x=P(X), r=P(RR), z=P(Z), w=P(W), h=P(HH), y=P(Y), rstd=P(RS))
+    ptr.update(kw)
+    return lib.rmsnorm_add_fwd(rows, width, 1e-6, 0.0, act, DType.BF16, ptr["x"], ptr["r"],
+                               ptr["z"], ptr["w"], ptr["h"], ptr["y"], ptr["rstd"], None)
+
+
+def abwd(lib, rows=R, width=H, act=Act.SILU, **kw):
+    ptr = dict(h=P(HH), z=P(Z), w=P(W), dy=P(DY), dh=P(DH), rstd=P(RS), dx=P(DX), dz=P(DZ),
+               dw=P(DW), ws=P(WS))
+    ptr.update(kw)
+    return lib.rmsnorm_add_bwd(rows, width, 1e-6, 0.0, act, DType.BF16, ptr["h"], ptr["z"],
+                               ptr["w"], ptr["dy"], ptr["dh"], ptr["rstd"], None, ptr["dx"],
+                               ptr["dz"], ptr["dw"], ptr["ws"],
+                               lib.norm_bwd_workspace_bytes(rows, width), None)
+
+
+ADD_FWD_CASES = [
+    ("valid", {}, Status.OK),
+    ("h is r", dict(h=P(RR)), Status.OK),
+    ("h is x", dict(h=P(X)), Status.OK),
+    ("h shifted into r", dict(h=P(RR, 16)), Status.E_ARG),
+    ("h is y", dict(h=P(Y)), Status.E_ARG),
+    ("r NULL", dict(r=0), Status.E_ARG),
+    ("h NULL", dict(h=0), Status.E_ARG),
+    ("r misaligned", dict(r=P(RR, 2)), Status.E_ALIGN),
+    ("no gate", dict(act=Act.NONE, z=0), Status.OK),
+]
+
+
+@pytest.mark.parametrize("name,kw,want", ADD_FWD_CASES, ids=[c[0] for c in ADD_FWD_CASES])
+def test_add_fwd_checks(lib, name, kw, want):
+    with validate_only(lib):
+        assert afwd(lib, **kw) == want
+
+
+ADD_BWD_CASES = [
+    ("valid", {}, Status.OK),
+    ("dh NULL", dict(dh=0), Status.OK),
+    ("dx is dh", dict(dx=P(DH)), Status.OK),
+    ("dx shifted into dh", dict(dx=P(DH, 32)), Status.E_ARG),
+    ("dz is dh", dict(dz=P(DH)), Status.E_ARG),
+    ("dh misaligned", dict(dh=P(DH, 8)), Status.E_ALIGN),
+]
+
+
+@pytest.mark.parametrize("name,kw,want", ADD_BWD_CASES, ids=[c[0] for c in ADD_BWD_CASES])
+def test_add_bwd_checks(lib, name, kw, want):
+    with validate_only(lib):
+        assert abwd(lib, **kw) == want
 
 
 @pytest.mark.parametrize("rows", [1, 31, 32, 33, 256, 257, 4096, 262144, 1 << 30])
