@@ -205,11 +205,20 @@ def cfg_sigmoid_f32_2048(seed: int = 0) -> Workload:
                 act="sigmoid", weight_offset=1.0, name="sigmoid_off1_16384x2048_f32")
 
 
+def cfg_qk_norm(width: int, rows: int, seed: int = 0) -> Workload:
+    """Per-head RMSNorm of q/k rows at head dim 256 or 512 (offset 1, no gate),
+    bf16, w ~ N(0, 0.1): rows = tokens x heads."""
+    return make("general", rows, width, "bf16", seed=seed, w_mean=0.0, w_std=0.1, act="none",
+                weight_offset=1.0, name=f"qk_norm_{rows}x{width}_bf16")
+
+
 VARIANTS = {
     "sigmoid_262144x128_bf16_outliers": cfg_sigmoid_heads,
     "silu_262144x128_f16_outliers": cfg_f16_heads,
     "norm_16384x5120_bf16": cfg_norm_5120,
     "sigmoid_off1_16384x2048_f32": cfg_sigmoid_f32_2048,
+    "qk_norm_131072x256_bf16": lambda seed=0: cfg_qk_norm(256, 131072, seed),
+    "qk_norm_65536x512_bf16": lambda seed=0: cfg_qk_norm(512, 65536, seed),
 }
 ALL = {**CONFIGS, **VARIANTS}
 
