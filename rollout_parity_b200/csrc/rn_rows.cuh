@@ -848,10 +848,18 @@ k_bwd_stripe(const BwdArgs a, int lpc) {
       }
       __syncwarp();
       const int64_t step_row = base + int64_t(st) * RPS;
+      // the step's rows that count for dw, one bit each: inside the batch and,
+      // when a mask is given, selected (lane l < RPS looks at row step_row + l)
+      unsigned valid;
+      {
+        const int64_t rr = step_row + (tid & (RPS - 1));
+        bool ok = rr < a.rows;
+        if (ok && a.mask != nullptr) ok = __ldg(a.mask + rr) != 0;
+        valid = __ballot_sync(0xffffffffu, ok);
+      }
 #pragma unroll
       for (int r = 0; r < RPS; ++r) {
-        // rows past the batch or outside the mask contribute nothing
-        if (step_row + r < a.rows && (a.mask == nullptr || __ldg(a.mask + step_row + r) != 0)) {
+        if ((valid >> r) & 1u) {   // rows past the batch or outside the mask add nothing
           const float4* src = reinterpret_cast<const float4*>(tbuf + r * TS);
 #pragma unroll
           for (int c = 0; c < C4; ++c) lacc[c] = add4(lacc[c], src[c * 32 + tid]);
