@@ -179,7 +179,8 @@ bool pick_sched(int32_t width, rn_dtype dt, Sched* s) {
   const int nv = width / vec_elems(dt);
   // up to 32 vectors: up to four vectors (64 B) per thread, so a 128-wide
   // 16-bit row is 4 lanes x 32 elements
-  if (nv <= 32) { s->T = pow2ceil(nv) / 4 > 1 ? pow2ceil(nv) / 4 : 1; s->K = (nv + s->T - 1) / s->T; }
+  if (nv == 16 && vec_elems(dt) == 8) { s->T = 8; s->K = 2; }   // H = 128, 16-bit
+  else if (nv <= 32) { s->T = pow2ceil(nv) / 4 > 1 ? pow2ceil(nv) / 4 : 1; s->K = (nv + s->T - 1) / s->T; }
   else if (nv <= 128) { s->T = 32; s->K = (nv + 31) / 32; }
   else if (nv <= 512) { s->T = 128; s->K = (nv + 127) / 128; }
   else if (nv <= 2048) {
@@ -191,12 +192,27 @@ bool pick_sched(int32_t width, rn_dtype dt, Sched* s) {
     else { s->T = 512; s->K = (nv + 511) / 512; }
   }
   else { s->T = 1024; s->K = (nv + 1023) / 1024; }
+  s->TF = s->T;
+  return true;
+}
+
+// The backward's kernel shape: the forward's, except at 16 vectors of 16-bit
+// elements (H = 128), where the forward's 8 x 2 team runs the backward as 4 x 4
+// (k_bwd_stripe: half the warps' rows per step, twice the work per thread)
+// and reproduces the forward's sum-of-squares order with the interleaved join.
+bool bwd_sched(int32_t width, rn_dtype dt, Sched* s) {
+  if (!pick_sched(width, dt, s)) return false;
+  if (vec_elems(dt) == 8 && width / 8 == 16) { s->T = 4; s->K = 4; }   // TF stays 8
   return true;
 }
 
 constexpr size_t kSmemCap = 96 * 1024;   // leaves per CTA shrink until the backward fits
 
 int64_t n_leaves_of(int64_t rows) { return (rows + kLeafRows - 1) / kLeafRows; }
+
+bool is_stripe(const Sched& s, int width, rn_dtype dt) {
+  return stripe_shape(s.T, s.K, vec_elems(dt), width / vec_elems(dt) == s.T * s.K);
+}
 
 // Leaves one backward CTA folds (a power of two).  k_bwd: sized for the gated
 // op's staging so that every activation uses the same geometry.  k_bwd_stripe
@@ -206,7 +222,7 @@ int64_t n_leaves_of(int64_t rows) { return (rows + kLeafRows - 1) / kLeafRows; }
 // each.  The bits never depend on this choice.
 int leaves_per_cta(const Sched& s, int width, rn_dtype dt, int64_t rows) {
   const int req = g_leaves_per_cta.load();
-  if (stripe_shape(s.T, s.K, vec_elems(dt), width / vec_elems(dt) == s.T * s.K)) {
+  if (is_stripe(s, width, dt)) {
     if (req > 0) return req < 8 ? req : 8;
     const int64_t slots = int64_t(8) * sm_count();
     const int64_t leaves = n_leaves_of(rows);
@@ -382,7 +398,7 @@ rn_status bwd_entry(int64_t rows, int32_t width, float eps, float woff, rn_act a
     return RN_OK;
   }
   Sched s;
-  pick_sched(width, dt, &s);
+  bwd_sched(width, dt, &s);
   const int lpc = leaves_per_cta(s, width, dt, rows);
   const int64_t leaves = n_leaves_of(rows);
   const int64_t groups = (leaves + lpc - 1) / lpc;
@@ -603,10 +619,10 @@ rn_status rn_fold_rows(int64_t n, int32_t width, const float* in, float* out, rn
 }
 
 const char* rn_describe(int32_t width, rn_dtype dt) {
-  Sched s;
-  if (!pick_sched(width, dt, &s)) return "unsupported";
-  const int lpc = leaves_per_cta(s, width, dt, 262144);
-  const bool stripe = stripe_shape(s.T, s.K, vec_elems(dt), width / vec_elems(dt) == s.T * s.K);
+  Sched s, sb;
+  if (!pick_sched(width, dt, &s) || !bwd_sched(width, dt, &sb)) return "unsupported";
+  const int lpc = leaves_per_cta(sb, width, dt, 262144);
+  const bool stripe = is_stripe(sb, width, dt);
   std::snprintf(t_describe, sizeof t_describe,
                 "backend=cuda-sm100a lib=librn kernels=k_fwd,%s,k_fold,k_fold1 dtype=%s width=%d "
                 "acc=fp32 team_threads=%d vectors_per_thread=%d elems_per_vector=%d "
@@ -621,7 +637,7 @@ const char* rn_describe(int32_t width, rn_dtype dt) {
 
 int32_t rn_bwd_launches(int64_t rows, int32_t width, rn_dtype dt) {
   Sched s;
-  if (rows <= 0 || rows > kMaxRows || !pick_sched(width, dt, &s)) return 0;
+  if (rows <= 0 || rows > kMaxRows || !bwd_sched(width, dt, &s)) return 0;
   const int lpc = leaves_per_cta(s, width, dt, rows);
   const int64_t groups = (n_leaves_of(rows) + lpc - 1) / lpc;
   return 1 + fold_passes(groups);

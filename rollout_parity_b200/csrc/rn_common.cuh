@@ -23,9 +23,12 @@ constexpr int kMaxGrid = 1 << 20;
 enum Act { kActNone = RN_ACT_NONE, kActSilu = RN_ACT_SILU, kActSigmoid = RN_ACT_SIGMOID };
 
 // A row of width H is owned by a team of T threads, each holding K 16-byte
-// vectors (vector v = k*T + t).  (T, K) depends on (H, dtype) only.
+// vectors (vector v = k*T + t).  (T, K) depends on (H, dtype) only.  TF is the
+// forward's team size, which fixes the declared sum-of-squares order; a
+// backward schedule with TF == 2T and K == 4 reproduces that order (see
+// thread_sumsq).
 struct Sched {
-  int T = 0, K = 0;
+  int T = 0, K = 0, TF = 0;
 };
 
 struct FwdArgs {

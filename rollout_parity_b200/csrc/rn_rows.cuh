@@ -330,7 +330,12 @@ __device__ __forceinline__ void vector_dots(const float2 (&a)[K][VE / 2],
 // Sum of squares of this thread's elements: each 16-byte vector folded in
 // ascending order with fma from -0.0, then the thread's K vector sums joined
 // by the pairwise tree.  K independent chains instead of one K*VE-long chain.
-template <int DT, int T, int K, bool EXACT>
+// XJ (K == 4): the order of a team of 2T threads holding 2 vectors each --
+// lane l < 2T holds vectors l and l + 2T and its butterfly's first step adds
+// lane l^T, so thread t of this team of T forms (v_t + v_{t+2T}) +
+// (v_{t+T} + v_{t+3T}) = (p0 + p2) + (p1 + p3) and the butterfly over T lanes
+// continues from there: the same bits as the wider team.
+template <int DT, int T, int K, bool EXACT, bool XJ = false>
 __device__ __forceinline__ float thread_sumsq(const uint4 (&x)[K], int nv, int t) {
   using F = Fmt<DT>;
   float2 f[K][F::VE / 2];
@@ -338,7 +343,12 @@ __device__ __forceinline__ float thread_sumsq(const uint4 (&x)[K], int nv, int t
   for (int k = 0; k < K; ++k) F::unpack2(x[k], f[k]);
   float p[K];
   vector_dots<F::VE, T, K, EXACT>(f, f, nv, t, p);
-  return pairwise_tree<K>(p);
+  if constexpr (XJ) {
+    static_assert(K == 4, "the interleaved join pairs four vectors");
+    return __fadd_rn(__fadd_rn(p[0], p[2]), __fadd_rn(p[1], p[3]));
+  } else {
+    return pairwise_tree<K>(p);
+  }
 }
 
 // Writes the partial of this CTA's group of NT leaves (an aligned
@@ -537,7 +547,7 @@ k_fwd(const FwdArgs a) {
 // call it in lockstep.
 //   g = u * a(z);  m = mean(g * dy * xh);  dx = rstd * (g*dy - xh*m)
 //   dz = dy * xh * u * a'(z)
-template <int DT, int T, int K, int ACT, bool EXACT, bool RESID, typename G>
+template <int DT, int T, int K, int ACT, bool EXACT, bool RESID, bool XJ, typename G>
 __device__ __forceinline__ void bwd_row(const BwdArgs& a, const G& gain, const uint4 (&xr)[K],
                                         const uint4 (&dr)[K], const uint4 (&zr)[K],
                                         float rs_staged, bool have_rstd, int64_t row, bool act,
@@ -555,7 +565,7 @@ __device__ __forceinline__ void bwd_row(const BwdArgs& a, const G& gain, const u
   }
   float rs = rs_staged;
   if (!have_rstd) {   // uniform branch
-    float ss[1] = {thread_sumsq<DT, T, K, EXACT>(xr, nv, t)};
+    float ss[1] = {thread_sumsq<DT, T, K, EXACT, XJ>(xr, nv, t)};
     team_sum<T, 1>(ss, red, phase, team, NT, mask);
     rs = rsqrtf(__fadd_rn(mean_of(ss[0], a.H, a.inv_h, a.h_pow2), a.eps));
   }
@@ -713,8 +723,8 @@ k_bwd(const BwdArgs a) {
         if constexpr (GATED) zr[k] = *slot(sl, 2, k);
       }
       float2 d[K][VE / 2];
-      bwd_row<DT, T, K, ACT, EXACT, RESID>(a, gain, xr, dr, zr,
-                                          have_rstd ? rsm[sl * bd + tid] : 0.0f,
+      bwd_row<DT, T, K, ACT, EXACT, RESID, false>(a, gain, xr, dr, zr,
+                                                 have_rstd ? rsm[sl * bd + tid] : 0.0f,
                                    have_rstd, row, act, t, red, phase, team, NT, mask, d);
       if (act && (a.mask == nullptr || __ldg(a.mask + row) != 0)) {   // masked rows add nothing
 #pragma unroll
@@ -749,7 +759,7 @@ k_bwd(const BwdArgs a) {
 // pending subtrees (the level-by-level pairwise tree), whose root is the group
 // partial.  Same bits as k_bwd.
 // ---------------------------------------------------------------------------
-template <int DT, int T, int K, int ACT, bool RESID>
+template <int DT, int T, int K, int ACT, bool RESID, bool XJ>
 __global__ void __launch_bounds__(32, bwd_min_blocks_of(T, K))
 k_bwd_stripe(const BwdArgs a, int lpc) {
   using F = Fmt<DT>;
@@ -831,8 +841,8 @@ k_bwd_stripe(const BwdArgs a, int lpc) {
         if constexpr (GATED) zr[k] = *slot(sl, 2, k);
       }
       float2 d[K][VE / 2];
-      bwd_row<DT, T, K, ACT, true, RESID>(a, gain, xr, dr, zr,
-                                           have_rstd ? rsm[sl * 32 + tid] : 0.0f,
+      bwd_row<DT, T, K, ACT, true, RESID, XJ>(a, gain, xr, dr, zr,
+                                               have_rstd ? rsm[sl * 32 + tid] : 0.0f,
                                   have_rstd, row, act, t, nullptr, phase, team, RPS, 0xffffffffu,
                                   d);
       // transpose the step's contributions: row `team` of the buffer
@@ -899,16 +909,32 @@ rn_status launch_fwd_tk(const Sched& s, const FwdArgs& a, cudaStream_t st) {
 }
 
 // The backward runs one CTA per group of leaves (grid-stride if capped).
+// The backward schedules a (T, K) the forward never uses only as the
+// interleaved form of a wider forward team (XJ); every other shape runs with the
+// forward's own schedule.
+template <int DT, int T, int K, int ACT, bool RESID, bool XJ>
+rn_status launch_stripe(const Sched& s, int lpc, const BwdArgs& a, int64_t groups,
+                        cudaStream_t st) {
+  const size_t smem = bwd_stripe_smem_bytes(s, a.H, ACT != kActNone, rn_dtype(DT));
+  static std::atomic<size_t> done{0};
+  static std::atomic<int> per_sm{0};
+  (void)prepare_kernel(k_bwd_stripe<DT, T, K, ACT, RESID, XJ>, 32, smem, done, per_sm);
+  return launch_pdl(k_bwd_stripe<DT, T, K, ACT, RESID, XJ>, dim3(grid_cap(groups)), dim3(32),
+                    smem, st, a, lpc);
+}
+
 template <int DT, int T, int K, int ACT, bool EXACT, bool RESID>
 rn_status launch_bwd_tk(const Sched& s, int lpc, const BwdArgs& a, int64_t groups,
                         cudaStream_t st) {
-  if constexpr (stripe_shape(T, K, Fmt<DT>::VE, EXACT)) {
-    const size_t smem = bwd_stripe_smem_bytes(s, a.H, ACT != kActNone, rn_dtype(DT));
-    static std::atomic<size_t> done{0};
-    static std::atomic<int> per_sm{0};
-    (void)prepare_kernel(k_bwd_stripe<DT, T, K, ACT, RESID>, 32, smem, done, per_sm);
-    return launch_pdl(k_bwd_stripe<DT, T, K, ACT, RESID>, dim3(grid_cap(groups)), dim3(32), smem,
-                      st, a, lpc);
+  if constexpr (Fmt<DT>::VE == 8 && EXACT && T == 8 && K == 2) {
+    return RN_E_WIDTH;   // the forward's shape at 16 vectors; its backward runs as 4 x 4
+  } else if constexpr (Fmt<DT>::VE == 8 && EXACT && T == 4 && K == 4) {
+    // 16 vectors of 16-bit elements: the forward's team is 8 x 2
+    if (s.TF != 8) return RN_E_WIDTH;
+    return launch_stripe<DT, T, K, ACT, RESID, true>(s, lpc, a, groups, st);
+  } else if constexpr (stripe_shape(T, K, Fmt<DT>::VE, EXACT)) {
+    if (s.TF != T) return RN_E_WIDTH;
+    return launch_stripe<DT, T, K, ACT, RESID, false>(s, lpc, a, groups, st);
   } else {   // (k_bwd is not instantiated for the stripe shapes)
     const int block = lpc * T;
     const size_t smem = bwd_smem_bytes(s, lpc, a.H, ACT != kActNone, rn_dtype(DT));
@@ -924,7 +950,7 @@ rn_status launch_bwd_tk(const Sched& s, int lpc, const BwdArgs& a, int64_t group
 // 16-bit elements (8 per vector, 1..2048 vectors a row) and fp32 (4 per
 // vector, 2..4096 vectors a row); exact = the row fills every vector slot.
 #define RN_SHAPES_16(X)                                                                         \
-  X(1, 1, true) X(1, 2, true) X(1, 3, true) X(1, 4, true)                                       \
+  X(1, 1, true) X(1, 2, true) X(1, 3, true) X(1, 4, true) X(8, 2, true)                         \
   X(2, 3, false) X(2, 3, true) X(2, 4, false) X(2, 4, true)                                     \
   X(4, 3, false) X(4, 3, true) X(4, 4, false) X(4, 4, true)                                     \
   X(8, 3, false) X(8, 3, true) X(8, 4, false) X(8, 4, true)                                     \

@@ -337,12 +337,13 @@ def test_workspace_bytes_invalid(lib):
     assert lib.norm_bwd_workspace_bytes(64, 100) == 0
 
 
-@pytest.mark.parametrize("width,dt,team", [(128, DType.BF16, 4), (128, DType.F32, 8),
+@pytest.mark.parametrize("width,dt,team", [(128, DType.BF16, 8), (128, DType.F32, 8),
                                            (8, DType.BF16, 1), (2048, DType.BF16, 128),
                                            (8192, DType.BF16, 512), (5120, DType.BF16, 128),
                                            (6144, DType.BF16, 256), (10240, DType.BF16, 256),
                                            (5120, DType.F32, 256), (4104, DType.BF16, 512),
-                                           (16384, DType.F32, 1024), (128, DType.F16, 4),
+                                           (16384, DType.F32, 1024), (128, DType.F16, 8),
+                                           (64, DType.F32, 4), (120, DType.BF16, 4),
                                            (5120, DType.F16, 128), (2048, DType.F16, 128)])
 def test_describe(lib, width, dt, team):
     d = lib.rn_describe(width, dt).decode()
