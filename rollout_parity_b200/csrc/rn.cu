@@ -177,9 +177,9 @@ bool act_ok(rn_act act) { return act == RN_ACT_NONE || act == RN_ACT_SILU || act
 bool pick_sched(int32_t width, rn_dtype dt, Sched* s) {
   if (!width_ok(width) || !dtype_ok(dt)) return false;
   const int nv = width / vec_elems(dt);
-  // up to 32 vectors: up to four vectors (64 B) per thread, so a 128-wide
-  // 16-bit row is 4 lanes x 32 elements
-  if (nv == 16 && vec_elems(dt) == 8) { s->T = 8; s->K = 2; }   // H = 128, 16-bit
+  // up to 32 vectors: up to four vectors (64 B) per thread; a 128-wide 16-bit
+  // row is 8 lanes x 16 elements (its backward runs 4 x 32, see bwd_sched)
+  if (nv == 16 && vec_elems(dt) == 8) { s->T = 8; s->K = 2; }
   else if (nv <= 32) { s->T = pow2ceil(nv) / 4 > 1 ? pow2ceil(nv) / 4 : 1; s->K = (nv + s->T - 1) / s->T; }
   else if (nv <= 128) { s->T = 32; s->K = (nv + 31) / 32; }
   else if (nv <= 512) { s->T = 128; s->K = (nv + 127) / 128; }
