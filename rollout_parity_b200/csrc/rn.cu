@@ -109,41 +109,53 @@ k_fold(const float* __restrict__ in, int64_t n, int H, float* __restrict__ out) 
 }
 
 // The last fold pass when at most kFold1Rows = 1024 partial rows remain: a CTA
-// of 32 warps covers 32 columns (one float per lane); warp g streams rows
-// [32g, 32g + 32) through the binary counter of pending subtrees, and the warps'
-// results (aligned blocks of 32 rows: perfect subtrees) are joined in shared
-// memory by the pairwise tree.  One launch where k_fold would need two.
+// of 32 warps covers 8 columns.  Warp w takes rows [32w, 32w + 32); its lane
+// (g, c) streams rows [32w + 8g, 32w + 8g + 8) of column c through the binary
+// counter of pending subtrees, the four 8-row subtrees of a warp are joined by
+// shuffles (g with g+1, then the pairs), and the 32 warp results (aligned
+// blocks of 32 rows: perfect subtrees) by the pairwise tree in shared memory.
+// Absent nodes are skipped, never added as zeros.  One launch where k_fold
+// would need two, spread over H/8 CTAs.
 constexpr int kFold1Rows = 1024;
 __global__ void __launch_bounds__(1024)
 k_fold1(const float* __restrict__ in, int64_t n, int H, float* __restrict__ out) {
   griddep_trigger();
   griddep_wait();      // the partials of the previous kernel are complete and visible
-  const int lane = threadIdx.x & 31, g = threadIdx.x >> 5;
-  const int c = blockIdx.x * 32 + lane;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int cl = lane & 7, g = lane >> 3;
+  const int c = blockIdx.x * 8 + cl;
   const bool col_ok = c < H;
-  const int64_t start = int64_t(g) * 32;
+  const int64_t start = int64_t(w) * 32 + int64_t(g) * 8;
   const int64_t left = n - start;
-  const int cnt = left <= 0 ? 0 : (left >= 32 ? 32 : int(left));
-  float v[32];
+  const int cnt = left <= 0 ? 0 : (left >= 8 ? 8 : int(left));
+  float v[8];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = (col_ok && i < cnt) ? __ldcg(in + (start + i) * H + c) : 0.0f;
-  TreeCounter<5, float> tc;
+  for (int i = 0; i < 8; ++i) v[i] = (col_ok && i < cnt) ? __ldcg(in + (start + i) * H + c) : 0.0f;
+  TreeCounter<3, float> tc;
 #pragma unroll
-  for (int i = 0; i < 32; ++i)
+  for (int i = 0; i < 8; ++i)
     if (i < cnt) tc.push(i, v[i]);
-  __shared__ float sm[32][33];
-  sm[g][lane] = cnt > 0 ? tc.finish(cnt) : 0.0f;
+  float r = cnt > 0 ? tc.finish(cnt) : 0.0f;
+  // the warp's four 8-row subtrees: (g0 + g1), (g2 + g3), then the pairs
+  const int64_t wleft = n - int64_t(w) * 32;
+  const int ng8 = wleft <= 0 ? 0 : (wleft >= 32 ? 4 : int((wleft + 7) / 8));   // present subtrees
+  const float r1 = __shfl_down_sync(0xffffffffu, r, 8);
+  if ((g & 1) == 0 && g + 1 < ng8) r = __fadd_rn(r, r1);
+  const float r2 = __shfl_down_sync(0xffffffffu, r, 16);
+  if (g == 0 && 2 < ng8) r = __fadd_rn(r, r2);
+  __shared__ float sm[32][8];
+  if (g == 0) sm[w][cl] = r;
   __syncthreads();
-  if (g == 0 && col_ok) {
-    const int ng = int((n + 31) / 32);
+  if (w == 0 && g == 0 && col_ok) {
+    const int nw = int((n + 31) / 32);
     float p[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) p[i] = sm[i][lane];
+    for (int i = 0; i < 32; ++i) p[i] = sm[i][cl];
 #pragma unroll
     for (int sft = 1; sft < 32; sft <<= 1) {
 #pragma unroll
       for (int l = 0; l + sft < 32; l += 2 * sft)
-        if (l + sft < ng) p[l] = __fadd_rn(p[l], p[l + sft]);
+        if (l + sft < nw) p[l] = __fadd_rn(p[l], p[l + sft]);
     }
     out[c] = p[0];
   }
@@ -340,7 +352,7 @@ rn_status run_fold(float* a, float* b, int64_t n, int H, float* dw, cudaStream_t
   while (n > 1) {
     int S = g_fold_rows.load();
     if (use_fold1(n))
-      return launch_pdl(k_fold1, dim3(unsigned((H + 31) / 32)), dim3(1024), 0, st, src, n, H, dw);
+      return launch_pdl(k_fold1, dim3(unsigned((H + 7) / 8)), dim3(1024), 0, st, src, n, H, dw);
     if (S <= 0) S = fold_rows_default(n);
     const int B = S / kFoldRG;
     const int64_t nout = (n + S - 1) / S;
