@@ -394,7 +394,7 @@ def run_ours(a):
             "bwd_gbs": round(achieved, 1),
             "invariance": inv,
             "roofline": {"bound": "hbm",
-                         "kernel": "rmsnorm_bwd call (k_bwd + k_fold passes)",
+                         "kernel": "rmsnorm_bwd call (backward kernel + dw fold pass)",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_source": src,
                          "traffic": traffic, "algorithmic_bytes": bwd_b},
