@@ -21,12 +21,16 @@
 //    same pairwise tree to them.  The gate and the offset never enter the
 //    sum of squares, so rstd is bitwise the same for every activation and
 //    offset.
-//  * The backward runs one team per 32-row leaf: the team walks its leaf's
-//    rows in ascending order, writes dx (and dz), and keeps the leaf's dw
-//    partial in registers (a left fold started from -0.0, i.e. from the first
-//    row).  The leaves of a CTA (an aligned power-of-two group) are joined in
-//    shared memory by the pairwise tree; the group partials go to the
-//    workspace and the fold kernel (rn.cu) joins them with the same tree.
+//  * The backward's dw: each 32-row leaf is the left fold of its rows'
+//    contributions in ascending order from -0.0; the leaves of a CTA (an
+//    aligned power-of-two group) are joined by the pairwise tree; the group
+//    partials go to the workspace and the fold kernels (rn.cu) join them with
+//    the same tree.  k_bwd gives each leaf a team that walks its rows;
+//    k_bwd_stripe (narrow rows) lets a warp's teams take consecutive rows of
+//    one leaf and folds the columns after a shared-memory transpose.
+//  * Variants are template flags: the gate activation, the residual add
+//    (forward: h = x + r is stored and normalised; backward: dx = dnorm + dh),
+//    and a row mask that leaves rows out of dw.
 //  * Every thread stages its own 16-byte vectors of a row with cp.async, S-1
 //    rows ahead of the row it computes, and reads back only what it copied
 //    (cp.async.wait_group makes a thread's own copies visible to it), so the
@@ -35,8 +39,8 @@
 //  * fp32 arithmetic with explicit rounding intrinsics (__fmul_rn, __fadd_rn,
 //    __fmaf_rn, __fdiv_rn, and the two-lane __fmul2_rn, __ffma2_rn on element
 //    pairs) wherever the compiler could otherwise contract or reorder, so the
-//    declared order is the executed order.  expf
-//    and rsqrtf are CUDA's own (no fast-math build).
+//    declared order is the executed order.  expf and rsqrtf are CUDA's own
+//    (no fast-math build).
 #pragma once
 
 #include <cuda_bf16.h>
