@@ -35,7 +35,8 @@
  *
  * Numerical contract (RL-Kernel RFC #415, section 4 "Numerical contract"):
  *   - every sum accumulates in fp32 and every intermediate is fp32; the only
- *     narrowing is the round-to-nearest-even store of y, dx, dz;
+ *     narrowing is the round-to-nearest-even store of y, dx, dz (and of h,
+ *     the residual sum, in rmsnorm_add_fwd);
  *   - the addition order depends on the width and dtype only: each thread
  *     adds its own elements in ascending order, a fixed xor butterfly joins
  *     the lanes of a row, a fixed pairwise tree joins the warps of a row.
@@ -45,7 +46,8 @@
  *   - dw uses no atomics: rows are folded in ascending order inside 32-row
  *     leaves, and leaves are joined by a level-by-level pairwise tree whose
  *     shape depends on the row count only (rn_describe prints it); it is
- *     bitwise the same across runs and launch geometries;
+ *     bitwise the same across runs and launch geometries, and a row left out
+ *     by a row mask stands for the tree's identity (-0.0);
  *   - unsupported shapes fail closed with a status; there is no fallback.
  *
  * Data layout and ownership
@@ -66,10 +68,12 @@
  *   RN_E_ARG       rows < 0 or > 2^36, eps negative or not finite, the
  *                  weight offset not finite, an unknown activation, a
  *                  required pointer is NULL (or z / dz given without a
- *                  gate), or an output overlaps an input or another output;
+ *                  gate), or an output overlaps an input or another output
+ *                  (except the in-place forms the residual-add calls allow);
  *   RN_E_DTYPE     dt is not RN_BF16, RN_F16 or RN_F32;
  *   RN_E_WIDTH     width is not a multiple of 8 in [8, 16384];
- *   RN_E_ALIGN     a tensor pointer is not 16-byte aligned (rstd: 4 bytes);
+ *   RN_E_ALIGN     a tensor pointer is not 16-byte aligned (rstd: 4 bytes;
+ *                  row_mask: any address);
  *   RN_E_WORKSPACE the backward's workspace is NULL or smaller than
  *                  norm_bwd_workspace_bytes(rows, width);
  *   RN_E_CUDA      a launch failed (rn_last_cuda_error() gives the code).
