@@ -96,3 +96,63 @@ def test_backward_launch_count_narrow_rows(lib, width, dt, ve):
         lpc = leaves_per_cta(width, ve, rows)
         groups = -(-(-(-rows // 32)) // lpc)
         assert lib.rn_bwd_launches(rows, width, dt) == 1 + fold_passes(groups), rows
+
+
+# ---- shared memory: every launch shape fits the 227 KB a CTA may use -------------
+SMEM_LIMIT = 227 * 1024
+
+
+def fwd_block(t, k):
+    return (128 if k <= 2 else 64) if t <= 16 else (128 if t == 32 else t)
+
+
+def fwd_stages(t):
+    return 3 if t <= 32 else (2 if t <= 512 else 1)
+
+
+def bwd_stages(t, k):
+    return 3 if t <= 16 else (4 if t <= 128 else ((3 if k <= 2 else 2) if t <= 512 else 1))
+
+
+def fwd_smem(t, k, ve, tensors):
+    b = fwd_block(t, k)
+    nt, w = b // t, (t // 32 if t > 32 else 1)
+    red = 2 * nt * w * 4 if t > 32 else 0
+    gain = k * t * ve * 4 if t <= 16 else 0
+    return red + gain + fwd_stages(t) * tensors * k * b * 16
+
+
+def bwd_smem(t, k, ve, lpc, width, tensors):
+    bd, w = lpc * t, (t // 32 if t > 32 else 1)
+    red = 2 * lpc * w * 4 if t > 32 else 0
+    gain = k * t * ve * 4 if t <= 16 else 0
+    stages = bwd_stages(t, k) * tensors * k * bd * 16
+    leaves = lpc * width * 4 if lpc > 1 else 0
+    return red + gain + stages + leaves + bwd_stages(t, k) * bd * 4
+
+
+def bwd_lpc(t, k, ve, width):
+    lpc = (8 * t if t <= 32 else (256 if t <= 128 else t)) // t
+    if t > 32 and width > 2048:
+        lpc = 1
+    lpc = min(lpc, 8)
+    while lpc > 1 and bwd_smem(t, k, ve, lpc, width, 3) > 96 * 1024:
+        lpc //= 2
+    return lpc
+
+
+@pytest.mark.parametrize("ve", [8, 4])
+def test_every_shape_fits_shared_memory(ve):
+    worst = 0
+    for width in range(8, 16385, 8):
+        t, k = fwd_shape(width, ve)
+        for tensors in (1, 2, 3):            # x; + z or r; + both
+            worst = max(worst, fwd_smem(t, k, ve, tensors))
+        tb, kb = bwd_shape(width, ve)
+        stripe = width // ve == tb * kb and tb <= 8 and (tb * kb * ve) % 128 == 0
+        if stripe:                            # gain, stages, rstd stages, transpose buffer
+            s = kb * tb * ve * 4 + 3 * 3 * kb * 32 * 16 + 3 * 32 * 4 + (32 // tb) * (width + 4) * 4
+        else:                                 # dh is read into registers, not staged
+            s = bwd_smem(tb, kb, ve, bwd_lpc(tb, kb, ve, width), width, 3)
+        worst = max(worst, s)
+    assert worst <= SMEM_LIMIT, worst
