@@ -252,8 +252,8 @@ rn_status rn_fold_rows(int64_t n, int32_t width, const float* in, float* out,
  * Gated RMSNorm backward that allocates nothing: the same computation,
  * arguments and results as gated_norm_bwd, but the dw-partial scratch is a
  * fixed 8 MiB block of static device memory inside this library instead of a
- * caller-supplied workspace.  (The paper has no counterpart of this call; it
- * is an addition of this library.)
+ * caller-supplied workspace.  (RFC #415 and PR #468 have no counterpart of
+ * this call; it is an addition of this library.)
  *
  * Who needs it: hosts that hand a library only the input and output buffers of
  * each call and own every other byte of device memory -- plugin interfaces,

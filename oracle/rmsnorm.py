@@ -287,7 +287,7 @@ def rmsnorm_dz_scale(x, w, dy, eps: float, weight_offset: float, z, act: str) ->
 # format and normalised:
 #     h = fmt(x + r),   y = h * rho(h) * u * a(z)
 # The sum is formed in fp32 and rounded once to the format, the kernel's
-# precision for that rounding decision (the pages fix none).  Backward: the
+# precision for that rounding decision (RFC #415 and PR #468 fix none).  Backward: the
 # gradient reaching h is the norm's plus dh, the gradient of the residual
 # output, and both x and r receive it:  dx = dr = dnorm(h; dy) + dh.
 # ---------------------------------------------------------------------------

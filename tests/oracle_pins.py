@@ -10,7 +10,7 @@ pin fails for each.
 The operators are those of RL-Kernel PR #468 ("[WS1][CUDA][Qwen3-Next] Gated
 RMSNorm CUDA kernel for the GDN block", Summary): zero-centred RMSNorm
 y = x*rstd*(1+w) and gated RMSNorm y = x*rstd*w*silu(z), and their gradients.
-The pages print no worked numeric example, so the worked examples here are
+RFC #415 and PR #468 print no worked numeric example, so the worked examples here are
 derived by hand with exact rational arithmetic; the derivations are written out
 next to each one.
 """

@@ -74,7 +74,8 @@ def test_config_gated_heads(cuda_lib, outlier_round):
     wl = workloads.cfg_gated_heads(outlier_round=outlier_round).to(DEV)
     out = run(cuda_lib, wl)
     stats = compare(out, wl)   # every row: the oracle handles 262144 x 128 in seconds
-    # the pages report ~99.999% of forward elements correctly rounded at this size
+    # PR #468 (Prior art & reuse decision) reports ~99.999% of forward elements
+    # correctly rounded at this size
     assert stats["y"]["correctly_rounded_frac"] >= 0.9999, stats["y"]
 
 

@@ -1,7 +1,7 @@
 """Residual-add RMSNorm on the GPU (rmsnorm_add_fwd / rmsnorm_add_bwd).
 
-The pages name a norm variant "with a residual" (RL-Kernel PR #468, Notes) and
-define nothing more; the reading is the usual fused form: h = x + r, formed in
+RL-Kernel PR #468 (Notes) mentions a norm variant that also adds a residual
+and defines nothing more about it; the reading is the usual fused form: h = x + r, formed in
 fp32 and rounded once to the tensors' format, stored and normalised; the
 backward gives x and r the norm's gradient at h plus dh.  h is a rounding
 decision both sides take in fp32, so it is compared bit for bit; the rest
