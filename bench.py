@@ -344,7 +344,9 @@ def run_ours(a):
         ms = float(t.item())
     ms_step = ms / K
     value = world * step_b * K / (ms / 1e3) / 1e9
-    launches = K * (1 + lib.rn_bwd_launches(R, H, dtc))
+    # our kernels per step: the forward, the backward and its fold passes, and
+    # with N ranks the rn_fold_rows pass of the dw exchange
+    launches = K * (1 + lib.rn_bwd_launches(R, H, dtc) + (1 if exchange is not None else 0))
 
     inv = invariance_checks(rn, sets[0], R, H, eps, wl0) \
         if rank == 0 and not a.no_invariance else None
@@ -476,13 +478,18 @@ def run_e2e(rn, wl, dev, steps, step_b, world, dist):
         odx.copy_(dx, non_blocking=True)
         if gated:
             odz.copy_(dz, non_blocking=True)
-        odw.copy_(dw, non_blocking=True)
+        # with N ranks the step's dw is the whole batch's (the all-gather fold)
+        odw.copy_(dw if dist is None else fold_dw(dw), non_blocking=True)
 
+    fold_dw = None
+    if dist is not None:
+        from rollout_parity_b200.parallel import fold_gathered_dw as fold_dw
     for _ in range(3):
         step()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
+        torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s.record()
     for _ in range(steps):
@@ -497,7 +504,8 @@ def run_e2e(rn, wl, dev, steps, step_b, world, dist):
     return {"value": round(world * step_b * steps / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 4),
-            "api": "rollout_parity_b200.rmsnorm_fwd/rmsnorm_bwd"}
+            "api": "rollout_parity_b200.rmsnorm_fwd/rmsnorm_bwd" +
+                   ("" if dist is None else " + parallel.fold_gathered_dw")}
 
 
 # ---------------------------------------------------------------------------
