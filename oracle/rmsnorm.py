@@ -281,8 +281,8 @@ def rmsnorm_dz_scale(x, w, dy, eps: float, weight_offset: float, z, act: str) ->
 
 
 # ---------------------------------------------------------------------------
-# Residual add.  [PR468] names an RMSNorm variant "with a residual" ("Notes",
-# on the strict profile's norm choice) and defines nothing more; read as the
+# Residual add.  [PR468] mentions an RMSNorm variant that also adds a residual
+# ("Notes", on the strict profile's norm choice) and defines nothing more; read as the
 # usual fused form: the residual stream h = x + r is stored in the tensors'
 # format and normalised:
 #     h = fmt(x + r),   y = h * rho(h) * u * a(z)

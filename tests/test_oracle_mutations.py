@@ -296,6 +296,80 @@ def m_bf16_round_ties_up(o):
     o.round_to_format = round_to_format
 
 
+def m_rstd_sqrt_not_rsqrt(o):
+    def rstd(x, eps):
+        x = np.asarray(x, dtype=np.float64)
+        return np.sqrt(np.sum(x * x, axis=1) / x.shape[1] + eps)
+    o.rstd = rstd
+
+
+def m_rstd_mean_over_rows(o):
+    # the mean square taken down a column (over the batch) instead of along the row
+    def rstd(x, eps):
+        x = np.asarray(x, dtype=np.float64)
+        col = np.sum(x * x, axis=0) / x.shape[0]
+        return 1.0 / np.sqrt(np.resize(col, x.shape[0]) + eps)
+    o.rstd = rstd
+
+
+def m_dx_mean_drops_xh(o):
+    def _dx(x, g, dy, rho):
+        m = np.sum(g * dy, axis=1) / x.shape[1]
+        return rho[:, None] * (g * dy - x * rho[:, None] * m[:, None])
+    o._dx = _dx
+
+
+def m_dw_rows_shifted(o):
+    # each row's contribution pairs its xh with the next row's dy (an index slip)
+    real = o.rmsnorm_bwd
+
+    def rmsnorm_bwd(x, w, dy, eps, weight_offset=1.0, z=None, act="none", row_mask=None):
+        dx, dz, _ = real(x, w, dy, eps, weight_offset, z, act, row_mask)
+        _, _, dw = real(x, w, np.roll(np.asarray(dy, dtype=np.float64), 1, axis=0), eps,
+                        weight_offset, z, act, row_mask)
+        return dx, dz, dw
+    o.rmsnorm_bwd = rmsnorm_bwd
+
+
+def m_sigmoid_derivative_sign(o):
+    real = o._act
+
+    def _act(z, act):
+        a, da = real(z, act)
+        if act == "sigmoid":
+            s = o.sigmoid(z)
+            da = s * (1.0 + s)
+        return a, da
+    o._act = _act
+
+
+def m_general_dz_drops_weight(o):
+    real = o.rmsnorm_bwd
+
+    def rmsnorm_bwd(x, w, dy, eps, weight_offset=1.0, z=None, act="none", row_mask=None):
+        dx, dz, dw = real(x, w, dy, eps, weight_offset, z, act, row_mask)
+        if dz is not None:
+            u = o._gain(w, weight_offset)[None, :]
+            with np.errstate(all="ignore"):
+                dz = np.where(u != 0, dz / u, dz)
+        return dx, dz, dw
+    o.rmsnorm_bwd = rmsnorm_bwd
+
+
+def m_residual_subtracts(o):
+    def residual_add(x, r, fmt):
+        if fmt == "f64":
+            return o._rows(x) - o._rows(r)
+        s = np.asarray(x, dtype=np.float32) - np.asarray(r, dtype=np.float32)
+        return o.round_to_format(s, fmt).reshape(o._rows(x).shape)
+    o.residual_add = residual_add
+
+
+def m_f16_round_as_bf16(o):
+    real = o.round_to_format
+    o.round_to_format = lambda a, fmt: real(a, "bf16" if fmt == "f16" else fmt)
+
+
 MUTANTS = [m for name, m in sorted(globals().items()) if name.startswith("m_")]
 
 
