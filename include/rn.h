@@ -152,8 +152,8 @@ rn_status rmsnorm_bwd(int64_t rows, int32_t width, float eps, float weight_offse
                       void* ws, size_t ws_bytes, rn_stream stream);
 
 /*
- * Residual-add forward (PR #468 Notes name a norm "with a residual"; read as
- * the usual fused form):
+ * Residual-add forward (PR #468 Notes mention a norm that also adds a
+ * residual; read as the usual fused form):
  *   h[r, j] = fmt(x[r, j] + r_in[r, j])   fp32 sum, rounded once to dt, written;
  *   y = rmsnorm_fwd of h (the stored, rounded h), rstd likewise.
  * x, r: [rows, width] dt, read.  h, y: [rows, width] dt, written; h may be
