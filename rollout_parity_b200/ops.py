@@ -332,7 +332,14 @@ def rn_fold_rows(partials: torch.Tensor, *, out: Optional[torch.Tensor] = None,
 
 
 def rn_describe(width: int, dtype=torch.bfloat16) -> str:
-    dt = _DT[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    """The provenance string for (width, dtype): kernels, team shape, reduction
+    order, dw tree, accumulator; "unsupported" for an invalid pair."""
+    if isinstance(dtype, torch.dtype):
+        if dtype not in _DT:
+            return "unsupported"
+        dt = _DT[dtype]
+    else:
+        dt = int(dtype)
     return load().rn_describe(width, dt).decode()
 
 
