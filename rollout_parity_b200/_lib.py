@@ -5,6 +5,7 @@ from __future__ import annotations
 import ctypes
 import enum
 import os
+import threading
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "librn.so")
@@ -73,24 +74,28 @@ SIGNATURES = {
 }
 
 _lib = None
+_lock = threading.Lock()
 
 
 def load(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Load librn.so once and attach the signatures."""
+    """Load librn.so once (thread-safe) and attach the signatures."""
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(path):
-        raise RuntimeError(
-            f"librn.so not found at {path}; build it with `python -m rollout_parity_b200.build` "
-            "(there is no CPU or Python fallback)")
-    lib = ctypes.CDLL(path)
-    for name, (res, args) in SIGNATURES.items():
-        f = getattr(lib, name)
-        f.restype = res
-        f.argtypes = args
-    _lib = lib
-    return lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"librn.so not found at {path}; build it with `python -m rollout_parity_b200.build` "
+                "(there is no CPU or Python fallback)")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(lib, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = lib
+    return _lib
 
 
 def check(fn: str, status: int) -> None:

@@ -73,6 +73,10 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 
 
 def _stream(x: torch.Tensor, stream) -> int:
+    """The cudaStream_t handle: the tensors' current stream when None, a
+    torch.cuda.Stream's handle, or a raw handle passed as an int."""
+    if isinstance(stream, int):
+        return stream
     s = torch.cuda.current_stream(x.device) if stream is None else stream
     return s.cuda_stream
 
