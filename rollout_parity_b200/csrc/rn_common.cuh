@@ -122,25 +122,42 @@ template <int DT>
 rn_status launch_bwd(int act, bool resid, const Sched& s, int lpc, const BwdArgs& a,
                      int64_t groups, cudaStream_t st);
 
-// Lets `kernel` use `smem` bytes of dynamic shared memory (the default limit is
-// 48 KB) and returns how many of its CTAs fit on one SM.  `done` and `per_sm`
-// cache the answer of the first call for this kernel and size class.
+// What prepare_kernel has done for one kernel, per device: the largest dynamic
+// shared-memory size it has allowed there and how many CTAs of that size fit
+// on one SM.  Both are properties of a device, so a process that drives
+// several GPUs prepares the kernel on each of them.
+constexpr int kMaxDevices = 64;
+struct KernelPrep {
+  std::atomic<size_t> done[kMaxDevices];
+  std::atomic<int> per_sm[kMaxDevices];
+};
+
+// Lets `kernel` use `smem` bytes of dynamic shared memory on the current device
+// (the default limit is 48 KB) and returns how many of its CTAs fit on one SM
+// there.  The answer is cached per device in `prep`; on a device number beyond
+// the cache the attribute is set again at every call.
 template <typename Kern>
-int prepare_kernel(Kern kernel, int block, size_t smem, std::atomic<size_t>& done,
-                   std::atomic<int>& per_sm) {
-  if (smem > done.load()) {
-    if (smem > 48 * 1024)
-      (void)cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, block, smem) != cudaSuccess ||
-        nb <= 0) {
-      (void)cudaGetLastError();
-      nb = 1;
-    }
-    per_sm.store(nb);
-    done.store(smem);
+int prepare_kernel(Kern kernel, int block, size_t smem, KernelPrep& prep) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    dev = -1;
   }
-  return per_sm.load();
+  const bool cached = dev >= 0 && dev < kMaxDevices;
+  if (cached && smem <= prep.done[dev].load()) return prep.per_sm[dev].load();
+  if (smem > 48 * 1024)
+    (void)cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  int nb = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, block, smem) != cudaSuccess ||
+      nb <= 0) {
+    (void)cudaGetLastError();
+    nb = 1;
+  }
+  if (cached) {
+    prep.per_sm[dev].store(nb);
+    prep.done[dev].store(smem);
+  }
+  return nb;
 }
 
 // Launches `kern` with programmatic stream serialization: it may be scheduled

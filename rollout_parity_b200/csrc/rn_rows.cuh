@@ -903,9 +903,8 @@ template <int DT, int T, int K, int ACT, bool EXACT, bool RESID>
 rn_status launch_fwd_tk(const Sched& s, const FwdArgs& a, cudaStream_t st) {
   constexpr int B = fwd_block_of(T, K);
   const size_t smem = fwd_smem_bytes(s, ACT != kActNone, RESID, rn_dtype(DT));
-  static std::atomic<size_t> done{0};
-  static std::atomic<int> per_sm{0};
-  const int nb = prepare_kernel(k_fwd<DT, T, K, ACT, EXACT, RESID>, B, smem, done, per_sm);
+  static KernelPrep prep;
+  const int nb = prepare_kernel(k_fwd<DT, T, K, ACT, EXACT, RESID>, B, smem, prep);
   const int64_t nblk = (a.rows + B / T - 1) / (B / T);
   const int64_t wave = int64_t(nb) * sm_count();
   const int grid = grid_cap(nblk < wave ? nblk : wave);
@@ -920,9 +919,8 @@ template <int DT, int T, int K, int ACT, bool RESID, bool XJ>
 rn_status launch_stripe(const Sched& s, int lpc, const BwdArgs& a, int64_t groups,
                         cudaStream_t st) {
   const size_t smem = bwd_stripe_smem_bytes(s, a.H, ACT != kActNone, rn_dtype(DT));
-  static std::atomic<size_t> done{0};
-  static std::atomic<int> per_sm{0};
-  (void)prepare_kernel(k_bwd_stripe<DT, T, K, ACT, RESID, XJ>, 32, smem, done, per_sm);
+  static KernelPrep prep;
+  (void)prepare_kernel(k_bwd_stripe<DT, T, K, ACT, RESID, XJ>, 32, smem, prep);
   return launch_pdl(k_bwd_stripe<DT, T, K, ACT, RESID, XJ>, dim3(grid_cap(groups)), dim3(32),
                     smem, st, a, lpc);
 }
@@ -942,9 +940,8 @@ rn_status launch_bwd_tk(const Sched& s, int lpc, const BwdArgs& a, int64_t group
   } else {   // (k_bwd is not instantiated for the stripe shapes)
     const int block = lpc * T;
     const size_t smem = bwd_smem_bytes(s, lpc, a.H, ACT != kActNone, rn_dtype(DT));
-    static std::atomic<size_t> done{0};
-    static std::atomic<int> per_sm{0};
-    (void)prepare_kernel(k_bwd<DT, T, K, ACT, EXACT, RESID>, block, smem, done, per_sm);
+    static KernelPrep prep;
+    (void)prepare_kernel(k_bwd<DT, T, K, ACT, EXACT, RESID>, block, smem, prep);
     return launch_pdl(k_bwd<DT, T, K, ACT, EXACT, RESID>, dim3(grid_cap(groups)), dim3(block),
                       smem, st, a);
   }

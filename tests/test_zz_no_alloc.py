@@ -55,6 +55,8 @@ def test_static_scratch_backward_matches_workspace_backward_twice(cuda_lib):
 def test_static_scratch_backward_rejects_shapes_beyond_its_scratch():
     # the size check comes before any CUDA call, so this runs without a GPU
     import rollout_parity_b200 as rn
+    from rollout_parity_b200 import build as rn_build
+    rn_build.build()                       # a fresh checkout has no librn.so yet
     lib = rn.load()
     rows = 262144 * 2                      # 9.4 MiB of partials at width 128
     assert lib.norm_bwd_workspace_bytes(rows, 128) > STATIC_SCRATCH_BYTES
