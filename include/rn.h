@@ -78,7 +78,8 @@
  *                  norm_bwd_workspace_bytes(rows, width);
  *   RN_E_CUDA      a launch failed (rn_last_cuda_error() gives the code).
  * rows == 0 is valid: the forward enqueues nothing and the backward sets
- * dw to +0.0.
+ * every element of dw to -0.0, the empty sum (see rmsnorm_bwd's row_mask:
+ * the same value as a call whose mask leaves out every row).
  */
 #ifndef RN_H_
 #define RN_H_
@@ -140,8 +141,9 @@ rn_status rmsnorm_fwd(int64_t rows, int32_t width, float eps, float weight_offse
  *   out of dw (they add nothing, whatever their values -- padding may hold
  *   anything); dx and dz are written for every row.  A left-out row stands
  *   for the additive identity (-0.0) in dw's fixed tree, so the tree's shape
- *   still depends on the row count only; a column no row contributes to is
- *   -0.0.  (PR #468 Notes: the dw entry point takes a mask.)
+ *   still depends on the row count only.  dw over no contributing row is the
+ *   empty sum, -0.0 in every column, whether every row is left out or
+ *   rows == 0.  (PR #468 Notes: the dw entry point takes a mask.)
  * With RN_ACT_NONE, z and dz must be NULL.  Arguments otherwise as
  * gated_norm_bwd (workspace: norm_bwd_workspace_bytes).
  */
@@ -270,7 +272,10 @@ rn_status rn_fold_rows(int64_t n, int32_t width, const float* in, float* out,
  *    process exits;
  *  - the first call on each device looks up the scratch's device address (with
  *    that device current) and keeps it; make that first call before any
- *    stream capture;
+ *    stream capture.  The address kept is that of the device's context at
+ *    the time: after cudaDeviceReset (or any other reset of that context)
+ *    the library's device memory is set up anew and the kept address is
+ *    stale, so do not use this call on a device after resetting it;
  *  - all calls on a device share the one scratch, which keeps whatever the last
  *    call left there (nothing in it needs to start at zero).  Calls that can
  *    run at the same time on the GPU -- on different streams, or from several
@@ -294,8 +299,8 @@ const char* rn_describe(int32_t width, rn_dtype dt);
 /*
  * Number of kernels one norm_bwd / gated_norm_bwd call with these sizes
  * enqueues under the current geometry (the backward kernel plus its dw fold
- * passes); 0 when rows == 0 (dw is cleared with a memset) or the shape is
- * unsupported.  The forward always enqueues one kernel when rows > 0.
+ * passes); 1 when rows == 0 (the kernel that sets dw to -0.0); 0 when the
+ * shape is unsupported.  The forward always enqueues one kernel when rows > 0.
  */
 int32_t rn_bwd_launches(int64_t rows, int32_t width, rn_dtype dt);
 

@@ -53,7 +53,9 @@ The zero-centred and gated operators above are (offset 1, no gate) and
 Row mask for dw ([PR468] "Changes to existing code, in detail": the dw entry
 point takes a mask; read as one flag per row, rows with the flag clear left out
 of dw's sum, e.g. padding):  dw_j = sum over rows r with mask_r of
-dy_rj * xh_rj * a(z_rj); dx and dz are unchanged.
+dy_rj * xh_rj * a(z_rj); dx and dz are unchanged.  A sum over no row (no rows
+at all, or a mask that selects none) is -0.0, the identity of IEEE addition
+(see _sum_over_rows).
 
 Parity pins (``tests/oracle_pins.py``, run by ``tests/test_oracle_pins.py``,
 with planted mistakes in ``tests/test_oracle_mutations.py``):
@@ -130,6 +132,18 @@ def gated_norm_fwd(x, z, w, eps: float):
     return xh * w[None, :] * silu(z), rho
 
 
+def _sum_over_rows(c) -> np.ndarray:
+    """dw's sum over rows, per column, started from -0.0.
+
+    -0.0 is the identity of IEEE addition (-0.0 + v == v for every v, +0.0
+    included), so starting there changes no sum that has a term; it fixes the
+    value of the empty sum -- a batch of no rows, or a row mask that selects
+    none -- at -0.0 in every column.  The pages fix no value for that case
+    ([PR468] Notes only say the T == 0 call returns early); this is the
+    reading taken."""
+    return np.sum(np.asarray(c, dtype=np.float64), axis=0, initial=-0.0)
+
+
 def _dx(x, g, dy, rho):
     width = x.shape[1]
     xh = x * rho[:, None]
@@ -144,7 +158,7 @@ def norm_bwd(x, w, dy, eps: float):
     rho = rstd(x, eps)
     g = np.broadcast_to((1.0 + w)[None, :], x.shape)
     dx = _dx(x, g, dy, rho)
-    dw = np.sum(dy * (x * rho[:, None]), axis=0)
+    dw = _sum_over_rows(dy * (x * rho[:, None]))
     return dx, dw
 
 
@@ -158,7 +172,7 @@ def gated_norm_bwd(x, z, w, dy, eps: float):
     g = w[None, :] * (z * s)
     dx = _dx(x, g, dy, rho)
     dz = dy * xh * w[None, :] * s * (1.0 + z * (1.0 - s))
-    dw = np.sum(dy * xh * (z * s), axis=0)
+    dw = _sum_over_rows(dy * xh * (z * s))
     return dx, dz, dw
 
 
@@ -249,7 +263,7 @@ def rmsnorm_bwd(x, w, dy, eps: float, weight_offset: float = 1.0, z=None, act: s
     contrib = dy * xh * a * np.ones_like(x)
     if row_mask is not None:
         contrib = contrib[np.asarray(row_mask).astype(bool)]
-    dw = np.sum(contrib, axis=0)
+    dw = _sum_over_rows(contrib)
     return dx, dz, dw
 
 

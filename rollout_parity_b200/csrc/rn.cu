@@ -161,6 +161,13 @@ k_fold1(const float* __restrict__ in, int64_t n, int H, float* __restrict__ out)
   }
 }
 
+// dw of a call with no rows: every column is the empty sum, -0.0 (the identity
+// of IEEE addition, the value the fixed tree gives a column no row reaches).
+__global__ void k_fill_neg_zero(float* __restrict__ out, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = -0.0f;
+}
+
 // Test kernel: the reciprocal used by the sigmoid, for checking against IEEE
 // division over every float in [1, 2].
 __global__ void k_test_rcp(const float* __restrict__ d, float* __restrict__ out, int64_t n,
@@ -404,10 +411,9 @@ rn_status bwd_entry(int64_t rows, int32_t width, float eps, float woff, rn_act a
   if (g_validate_only.load()) return RN_OK;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (rows == 0) {
-    if (cudaMemsetAsync(dw, 0, size_t(width) * sizeof(float), st) != cudaSuccess)
-      return launch_status();
-    return RN_OK;
+  if (rows == 0) {   // dw is the empty sum
+    k_fill_neg_zero<<<(width + 255) / 256, 256, 0, st>>>(dw, width);
+    return launch_status();
   }
   Sched s;
   bwd_sched(width, dt, &s);
@@ -649,7 +655,8 @@ const char* rn_describe(int32_t width, rn_dtype dt) {
 
 int32_t rn_bwd_launches(int64_t rows, int32_t width, rn_dtype dt) {
   Sched s;
-  if (rows <= 0 || rows > kMaxRows || !bwd_sched(width, dt, &s)) return 0;
+  if (rows < 0 || rows > kMaxRows || !bwd_sched(width, dt, &s)) return 0;
+  if (rows == 0) return 1;   // the fill of dw
   const int lpc = leaves_per_cta(s, width, dt, rows);
   const int64_t groups = (n_leaves_of(rows) + lpc - 1) / lpc;
   return 1 + fold_passes(groups);

@@ -101,11 +101,23 @@ def test_left_out_rows_may_hold_anything(cuda_lib, act, off, rows, width, dtype)
     assert torch.equal(bits(dw), bits(dw_clean))
 
 
-def test_everything_left_out_gives_negative_zero(cuda_lib):
-    wl = make("silu", 0.0, 4096, 128, "bf16", seed=3)
-    m = torch.zeros(4096, dtype=torch.uint8, device=DEV)
+@pytest.mark.parametrize("act,off,rows,width,dtype", CASES[:3], ids=IDS[:3])
+def test_everything_left_out_is_the_oracles_empty_sum(cuda_lib, act, off, rows, width, dtype):
+    # no row contributes: the oracle's empty sum, sign included (-0.0), and the
+    # same bits as a call with no rows at all
+    wl = make(act, off, rows, width, dtype, seed=3)
+    m = torch.zeros(rows, dtype=torch.uint8, device=DEV)
     _, _, dw = bwd(cuda_lib, wl, m)
-    assert (bits(dw) == torch.tensor(-2 ** 31, dtype=torch.int32, device=DEV)).all()
+    _, _, want = oracle.rmsnorm_bwd(f64(wl.x), f64(wl.w), f64(wl.dy), wl.eps, off,
+                                    None if wl.z is None else f64(wl.z), act,
+                                    row_mask=m.cpu().numpy())
+    got = dw.cpu().numpy()
+    assert np.array_equal(got, want) and np.array_equal(np.signbit(got), np.signbit(want))
+    e = wl.x[:0]
+    dw0 = torch.full_like(dw, 7.0)
+    cuda_lib.rmsnorm_bwd(e, wl.w, e, None, wl.eps, off, None if wl.z is None else wl.z[:0], act,
+                         dw=dw0)
+    assert torch.equal(bits(dw0), bits(dw))
 
 
 def test_all_ones_mask_is_no_mask(cuda_lib):

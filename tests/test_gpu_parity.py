@@ -8,6 +8,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from gpu_util import compare, oracle_rows, run, sample_rows
 from numerics import bf16_round, to64
 from rollout_parity_b200 import workloads
@@ -102,7 +103,18 @@ def test_empty_batch(cuda_lib):
     dw = torch.full((128,), 7.0, device=DEV)
     cuda_lib.gated_norm_bwd(x, z, w, x, None, dw=dw)
     torch.cuda.synchronize()
-    assert torch.equal(dw, torch.zeros_like(dw)) and not torch.signbit(dw).any()
+    # the empty sum: the oracle's value, sign included (-0.0 in every column)
+    e = np.zeros((0, 128))
+    _, _, want = oracle.gated_norm_bwd(e, e, np.ones(128), e, 1e-6)
+    got = dw.cpu().numpy()
+    assert np.array_equal(got, want) and np.array_equal(np.signbit(got), np.signbit(want))
+    for act, off in (("none", 1.0), ("sigmoid", 0.0)):
+        dw = torch.full((128,), 7.0, device=DEV)
+        cuda_lib.rmsnorm_bwd(x, w, x, None, 1e-6, off, None if act == "none" else z, act, dw=dw)
+        _, _, want = oracle.rmsnorm_bwd(e, np.ones(128), e, 1e-6, off,
+                                        None if act == "none" else e, act)
+        got = dw.cpu().numpy()
+        assert np.array_equal(np.signbit(got), np.signbit(want)) and not got.any(), act
 
 
 def test_constant_rows_closed_form(cuda_lib):
