@@ -462,6 +462,178 @@ def pin_residual_finite_differences(orc):
         _close(dx, _fd(lambda a: L(x, a), r), rtol=1e-7, atol=1e-8, what=f"{act} d/dr")
 
 
+# --------------------------------------------------------------------------
+# the cancellation scales behind the dx / dz tolerance
+# --------------------------------------------------------------------------
+L7 = math.log(7.0)
+
+
+def pin_cancellation_scales_worked(orc):
+    """The scale T of the dx / dz tolerance (|gpu - ref| <= 2 ulp + 2^-16 T),
+    hand-derived on the worked examples above.
+    dx: T = max(|rho*g*dy|, |rho*xh| * mean_k |g_k dy_k xh_k|).
+      Zero-centred example (rho = 2/5, xh = [2,4,4,8]/5, g*dy = [1,-3/2,0,1]):
+      |rho*g*dy| = [2/5, 3/5, 0, 2/5]; |g*dy*xh| = [2/5, 6/5, 0, 8/5], mean 4/5;
+      |rho*xh| * 4/5 = [16, 32, 32, 64]/125  ->  T = [2/5, 3/5, 32/125, 64/125]
+      (with |m| = 1/5 in place of the mean of magnitudes the last two would be
+      8/125 and 2/5).
+      Gated example (g = [3L/4, -L/2, 0, -3L/4], L = ln 3): |rho*g*dy| =
+      [3L/10, L/5, 0, 3L/20]; |g*dy*xh| = [3L/10, 2L/5, 0, 3L/5], mean 13L/40;
+      |rho*xh| * 13L/40 = [13L/250, 13L/125, 13L/125, 26L/125]
+      ->  T = [3L/10, L/5, 13L/125, 26L/125].
+      Sigmoid gate, offset 1 (g = [3/4, 3/8, 0, 3/2]): |rho*g*dy| =
+      [3/10, 3/20, 0, 3/10]; |g*dy*xh| = [3/10, 3/10, 0, 6/5], mean 9/20;
+      |rho*xh| * 9/20 = [9, 18, 18, 36]/125  ->  T = [3/10, 3/20, 18/125, 3/10].
+    dz: T = |dy*xh*u*s| * max(1, |z(1-s)|) (silu), |dy*xh*u*s| (sigmoid).
+      Gated example: dy*xh*w*s = [3/10, -2/5, 4, -3/5] and |z(1-s)| =
+      [L/4, 3L/4, 0, L/4], all below 1  ->  T = [3/10, 2/5, 4, 3/5].
+      Sigmoid, offset 1: dy*xh*u*s = [3/10, -3/10, 0, 6/5].
+    A second example where the silu factor exceeds 1: H = 2, x = [3, 4],
+      eps = 7/2 (rho = 1/4, xh = [3/4, 1]), z = [-ln 7, ln 3] (s = [1/8, 3/4],
+      |z(1-s)| = [7 ln7/8 > 1, ln3/4 < 1]), w = [2, -1], dy = [1, -4]:
+      dy*xh*w*s = [3/16, 3]  ->  dz T = [21 ln7/128, 3];
+      with offset 1 (u = [3, 0]): silu T = [63 ln7/256, 0], sigmoid [9/32, 0];
+      dx (gated): g*dy = [-ln7/4, 3 ln3], |rho*g*dy| = [ln7/16, 3 ln3/4];
+      |g*dy*xh| = [3 ln7/16, 3 ln3], mean (3 ln7/16 + 3 ln3)/2;
+      |rho*xh| * mean = [(3/32), (1/8)] * (3 ln7/16 + 3 ln3)
+      ->  T = [(9/32)(ln7/16 + ln3), 3 ln3/4]."""
+    L = L3
+    x = [[1.0, 2.0, 2.0, 4.0]]
+    w = [0.0, 0.5, -1.0, 1.0]
+    dy = [[1.0, -1.0, 2.0, 0.5]]
+    z = [[L, -L, 0.0, L]]
+    wg = [1.0, 2.0, 5.0, -1.0]
+    t_norm = [[2 / 5, 3 / 5, 32 / 125, 64 / 125]]
+    _close(orc.dx_cancellation_scale(x, w, dy, 0.0), t_norm, what="dx T, zero-centred")
+    _close(orc.rmsnorm_dx_scale(x, w, dy, 0.0, 1.0), t_norm, what="general dx T, offset 1")
+    t_gated = [[3 * L / 10, L / 5, 13 * L / 125, 26 * L / 125]]
+    _close(orc.dx_cancellation_scale(x, wg, dy, 0.0, z=z), t_gated, what="dx T, gated")
+    _close(orc.rmsnorm_dx_scale(x, wg, dy, 0.0, 0.0, z, "silu"), t_gated,
+           what="general dx T, silu")
+    _close(orc.dz_cancellation_scale(x, z, wg, dy, 0.0), [[0.3, 0.4, 4.0, 0.6]],
+           what="dz T, gated")
+    _close(orc.rmsnorm_dz_scale(x, wg, dy, 0.0, 0.0, z, "silu"), [[0.3, 0.4, 4.0, 0.6]],
+           what="general dz T, silu")
+    _close(orc.rmsnorm_dx_scale(x, w, dy, 0.0, 1.0, z, "sigmoid"),
+           [[3 / 10, 3 / 20, 18 / 125, 3 / 10]], what="general dx T, sigmoid offset 1")
+    _close(orc.rmsnorm_dz_scale(x, w, dy, 0.0, 1.0, z, "sigmoid"), [[0.3, 0.3, 0.0, 1.2]],
+           what="general dz T, sigmoid offset 1")
+    x2, z2, w2, dy2 = [[3.0, 4.0]], [[-L7, L]], [2.0, -1.0], [[1.0, -4.0]]
+    _close(orc.dz_cancellation_scale(x2, z2, w2, dy2, 3.5), [[21 * L7 / 128, 3.0]],
+           what="dz T, silu factor above 1")
+    _close(orc.rmsnorm_dz_scale(x2, w2, dy2, 3.5, 0.0, z2, "silu"), [[21 * L7 / 128, 3.0]],
+           what="general dz T, silu factor above 1")
+    _close(orc.rmsnorm_dz_scale(x2, w2, dy2, 3.5, 1.0, z2, "silu"), [[63 * L7 / 256, 0.0]],
+           what="general dz T, silu offset 1")
+    _close(orc.rmsnorm_dz_scale(x2, w2, dy2, 3.5, 1.0, z2, "sigmoid"), [[9 / 32, 0.0]],
+           what="general dz T, sigmoid offset 1")
+    t2 = [[(9 / 32) * (L7 / 16 + L), 3 * L / 4]]
+    _close(orc.dx_cancellation_scale(x2, w2, dy2, 3.5, z=z2), t2, what="dx T, second example")
+    _close(orc.rmsnorm_dx_scale(x2, w2, dy2, 3.5, 0.0, z2, "silu"), t2,
+           what="general dx T, second example")
+
+
+def _f32_backward(x, z, w, dy, eps, act, offset):
+    """An fp32 evaluation of dx and dz, independent of the oracle and of the
+    kernels: numpy float32 arithmetic, sums in plain ascending order (the
+    order whose rounding error grows fastest), the sigmoid in its
+    overflow-free form."""
+    f = np.float32
+    x, dy, w = x.astype(f), dy.astype(f), w.astype(f)
+    R, H = x.shape
+    u = (w + f(offset)).astype(f) if offset != 0 else w
+    ss = np.zeros(R, f)
+    for j in range(H):
+        ss = (ss + x[:, j] * x[:, j]).astype(f)
+    rho = (f(1) / np.sqrt((ss / f(H) + f(eps)).astype(f))).astype(f)
+    xh = (x * rho[:, None]).astype(f)
+    if act == "none":
+        a, c, s = np.ones_like(x), None, None
+    else:
+        z = z.astype(f)
+        e = np.exp(-np.abs(z)).astype(f)
+        s = np.where(z >= 0, f(1) / (f(1) + e), e / (f(1) + e)).astype(f)
+        a = (z * s).astype(f) if act == "silu" else s
+        c = (f(1) + z * (f(1) - s)).astype(f) if act == "silu" else (f(1) - s).astype(f)
+    gd = ((u[None, :] * a).astype(f) * dy).astype(f)
+    acc = np.zeros(R, f)
+    for j in range(H):
+        acc = (acc + gd[:, j] * xh[:, j]).astype(f)
+    m = (acc / f(H)).astype(f)
+    dx = (rho[:, None] * (gd - (xh * m[:, None]).astype(f)).astype(f)).astype(f)
+    dz = None if act == "none" else \
+        (((((dy * xh).astype(f) * u[None, :]).astype(f) * s).astype(f) * c).astype(f))
+    return dx, dz
+
+
+def pin_cancellation_scales_bound_fp32_error(orc):
+    """The scale is large enough: an fp32 evaluation of dx and dz (ascending
+    sums; rows with 1% of channels x50 in x, z and dy, as the outlier workload
+    has) stays within 2^-16 * T of the fp64 result, at widths 128 and 2048,
+    for every gate: dx in every element, dz wherever the sigmoid is an fp32
+    normal number (z > -87).  Below that s(z) = e^z keeps fewer than 24 bits in
+    fp32, or none past z < -103; those dz are below 1e-37, where the bf16 and
+    fp16 tolerances' own spacing (2^-133, 2^-24) is far larger than dz."""
+    rng = np.random.default_rng(31)
+    for H in (128, 2048):
+        for act, off in (("none", 1.0), ("silu", 0.0), ("sigmoid", 1.0)):
+            R = 16
+            x, z, dy = (rng.normal(size=(R, H)) for _ in range(3))
+            w = rng.normal(1.0 if off == 0.0 else 0.0, 0.3, H)
+            cols = rng.choice(H, max(1, round(0.01 * H)), replace=False)
+            for a in (x, z, dy):
+                a[:, cols] *= 50.0
+            x, z, dy, w = (a.astype(np.float32).astype(np.float64) for a in (x, z, dy, w))
+            zz = None if act == "none" else z
+            dx64, dz64, _ = orc.rmsnorm_bwd(x, w, dy, 1e-6, off, zz, act)
+            dx32, dz32 = _f32_backward(x, z, w, dy, 1e-6, act, off)
+            T = orc.rmsnorm_dx_scale(x, w, dy, 1e-6, off, zz, act)
+            assert np.all(np.abs(dx32 - dx64) <= 2.0 ** -16 * T), (H, act, "dx")
+            if act != "none":
+                Tz = orc.rmsnorm_dz_scale(x, w, dy, 1e-6, off, z, act)
+                normal = z > -87.0
+                assert np.all((np.abs(dz32 - dz64) <= 2.0 ** -16 * Tz)[normal]), (H, act, "dz")
+                if act == "silu" and off == 0.0:
+                    assert np.array_equal(Tz, orc.dz_cancellation_scale(x, z, w, dy, 1e-6))
+                    assert np.array_equal(T, orc.dx_cancellation_scale(x, w, dy, 1e-6, z=z))
+            if act == "none" and off == 1.0:
+                assert np.array_equal(T, orc.dx_cancellation_scale(x, w, dy, 1e-6))
+
+
+# --------------------------------------------------------------------------
+# the empty sum
+# --------------------------------------------------------------------------
+def pin_empty_and_signed_zero_sums(orc):
+    """dw over no row -- a batch of no rows, or a mask selecting none -- is
+    -0.0 in every column (IEEE addition's identity: the reading taken where the
+    pages fix no value).  Sums that have terms follow IEEE's sign rules: a
+    column whose every term is -0.0 sums to -0.0, and one +0.0 term among them
+    makes +0.0 (IEEE 754, section 6.3)."""
+    H = 4
+    for act, off in (("none", 1.0), ("silu", 0.0), ("sigmoid", 1.0)):
+        x0 = np.zeros((0, H))
+        zz = None if act == "none" else x0
+        _, _, dw = orc.rmsnorm_bwd(x0, np.ones(H), x0, 1e-6, off, zz, act)
+        assert dw.shape == (H,) and np.all(dw == 0) and np.all(np.signbit(dw)), (act, dw)
+        x = np.array([[1.0, 2.0, 0.0, 0.0], [3.0, -1.0, 0.0, 0.0], [2.0, 2.0, 0.0, 0.0]])
+        dy = np.array([[1.0, 1.0, -1.0, -1.0], [2.0, -1.0, -2.0, 3.0], [1.0, 1.0, -1.0, -1.0]])
+        z = np.full_like(x, 0.5)
+        zz = None if act == "none" else z
+        _, _, dwm = orc.rmsnorm_bwd(x, np.ones(H), dy, 1e-6, off, zz, act,
+                                    row_mask=np.zeros(3, np.uint8))
+        assert np.all(dwm == 0) and np.all(np.signbit(dwm)), (act, dwm)
+        # column 2: x = +0 and dy < 0 in every row: every term is -0.0;
+        # column 3: one row has dy > 0, a +0.0 term among -0.0 terms
+        _, _, dws = orc.rmsnorm_bwd(x, np.ones(H), dy, 1e-6, off, zz, act)
+        assert dws[2] == 0 and np.signbit(dws[2]), (act, dws)
+        assert dws[3] == 0 and not np.signbit(dws[3]), (act, dws)
+    _, dw = orc.norm_bwd(np.zeros((0, H)), np.ones(H), np.zeros((0, H)), 1e-6)
+    assert np.all(np.signbit(dw)) and np.all(dw == 0), dw
+    _, _, dw = orc.gated_norm_bwd(np.zeros((0, H)), np.zeros((0, H)), np.ones(H),
+                                  np.zeros((0, H)), 1e-6)
+    assert np.all(np.signbit(dw)) and np.all(dw == 0), dw
+
+
 ALL_PINS = [
     pin_worked_example_norm,
     pin_worked_example_eps,
@@ -483,6 +655,9 @@ ALL_PINS = [
     pin_round_to_format,
     pin_residual_add_example,
     pin_residual_finite_differences,
+    pin_cancellation_scales_worked,
+    pin_cancellation_scales_bound_fp32_error,
+    pin_empty_and_signed_zero_sums,
 ]
 
 

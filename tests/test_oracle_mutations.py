@@ -370,6 +370,86 @@ def m_f16_round_as_bf16(o):
     o.round_to_format = lambda a, fmt: real(a, "bf16" if fmt == "f16" else fmt)
 
 
+# --- the cancellation scales of the dx / dz tolerance ----------------------
+def m_dx_scale_times_1024(o):
+    real = o.dx_cancellation_scale
+    o.dx_cancellation_scale = lambda *a, **k: 1024.0 * real(*a, **k)
+
+
+def m_dx_scale_over_1024(o):
+    real = o.dx_cancellation_scale
+    o.dx_cancellation_scale = lambda *a, **k: real(*a, **k) / 1024.0
+
+
+def m_dx_scale_uses_abs_m(o):
+    def dx_cancellation_scale(x, w, dy, eps, z=None):
+        x, dy = o._rows(x), o._rows(dy)
+        w = np.asarray(w, dtype=np.float64)
+        rho = o.rstd(x, eps)
+        xh = x * rho[:, None]
+        g = np.broadcast_to((1.0 + w)[None, :], x.shape) if z is None else \
+            w[None, :] * o.silu(o._rows(z))
+        m = np.abs(np.sum(g * dy * xh, axis=1)) / x.shape[1]
+        return np.maximum(np.abs(rho[:, None] * g * dy), np.abs(rho[:, None] * xh * m[:, None]))
+    o.dx_cancellation_scale = dx_cancellation_scale
+
+
+def m_dz_scale_drops_silu_factor(o):
+    def dz_cancellation_scale(x, z, w, dy, eps):
+        x, z, dy = o._rows(x), o._rows(z), o._rows(dy)
+        rho = o.rstd(x, eps)
+        return np.abs(dy * x * rho[:, None] * np.asarray(w)[None, :] * o.sigmoid(z))
+    o.dz_cancellation_scale = dz_cancellation_scale
+
+
+def m_dz_scale_times_1024(o):
+    real = o.dz_cancellation_scale
+    o.dz_cancellation_scale = lambda *a, **k: 1024.0 * real(*a, **k)
+
+
+def m_general_dx_scale_over_1024(o):
+    real = o.rmsnorm_dx_scale
+    o.rmsnorm_dx_scale = lambda *a, **k: real(*a, **k) / 1024.0
+
+
+def m_general_dx_scale_times_1024(o):
+    real = o.rmsnorm_dx_scale
+    o.rmsnorm_dx_scale = lambda *a, **k: 1024.0 * real(*a, **k)
+
+
+def m_general_dx_scale_drops_mean_term(o):
+    def rmsnorm_dx_scale(x, w, dy, eps, weight_offset=1.0, z=None, act="none"):
+        x, dy = o._rows(x), o._rows(dy)
+        rho = o.rstd(x, eps)
+        a, _ = o._act(None if z is None else o._rows(z), act)
+        g = np.broadcast_to(o._gain(w, weight_offset)[None, :] * a, x.shape)
+        return np.abs(rho[:, None] * g * dy)
+    o.rmsnorm_dx_scale = rmsnorm_dx_scale
+
+
+def m_general_dz_scale_over_1024(o):
+    real = o.rmsnorm_dz_scale
+    o.rmsnorm_dz_scale = lambda *a, **k: real(*a, **k) / 1024.0
+
+
+def m_general_dz_scale_drops_silu_factor(o):
+    def rmsnorm_dz_scale(x, w, dy, eps, weight_offset, z, act):
+        x, z, dy = o._rows(x), o._rows(z), o._rows(dy)
+        rho = o.rstd(x, eps)
+        return np.abs(dy * x * rho[:, None] * o._gain(w, weight_offset)[None, :] * o.sigmoid(z))
+    o.rmsnorm_dz_scale = rmsnorm_dz_scale
+
+
+def m_general_dz_scale_silu_factor_for_sigmoid(o):
+    real = o.rmsnorm_dz_scale
+    o.rmsnorm_dz_scale = lambda x, w, dy, eps, off, z, act: real(x, w, dy, eps, off, z, "silu")
+
+
+# --- the empty sum --------------------------------------------------------
+def m_empty_sum_is_positive_zero(o):
+    o._sum_over_rows = lambda c: np.sum(np.asarray(c, dtype=np.float64), axis=0)
+
+
 MUTANTS = [m for name, m in sorted(globals().items()) if name.startswith("m_")]
 
 
