@@ -25,7 +25,8 @@ e2e       = the same metric through the public Python API with host buffers:
             every step copies x, z, dy, w from pinned host memory and y, rstd,
             dx, dz, dw back.
 --impl reference times the fp64 CPU oracle (the repository's checker) on
-the host cores, one bounded row sample per step.
+every host core (one worker process per core, each on its own block of
+rows), one bounded row sample per step.
 """
 from __future__ import annotations
 
@@ -352,9 +353,11 @@ def run_ours(a):
         if rank == 0 and not a.no_invariance else None
     e2e = run_e2e(rn, host[0], dev, a.e2e_steps, step_b, world, dist) if a.e2e_steps > 0 \
         else None
-    cpu = None
+    cpu = acc = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         cpu = cpu_baseline(host[0], fwd_b, bwd_b)
+        # the oracle as the checker of set 0's outputs (its inputs are host[0])
+        acc = accuracy(host[0], sets[0])
 
     if rank == 0:
         peak, src = peaks()
@@ -400,7 +403,8 @@ def run_ours(a):
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_source": src,
                          "traffic": traffic, "algorithmic_bytes": bwd_b},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+            "cpu_baseline": cpu, "accuracy": acc, "e2e": e2e, "gpu_launches": launches,
+            "clocks": clk,
             "source_sha1": src_sha(),
         }
         print(json.dumps(line), flush=True)
@@ -516,28 +520,193 @@ def _oracle_step(orc, wl, x, z, w, dy):
     orc.rmsnorm_bwd(x, w, dy, wl.eps, wl.weight_offset, z, wl.act)
 
 
-def cpu_baseline(wl, fwd_b, bwd_b, min_s=10.0, max_s=30.0):
+def host_info():
+    """The host's usable cores and CPU model (recorded beside every CPU figure)."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    model = "unknown"
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                model = ln.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"nproc": cores, "cpu_model": model}
+
+
+# Worker side of OraclePool.  A worker is a fresh interpreter (the pool is
+# started with "spawn": nothing of the parent's CUDA state is inherited, and
+# spawn is safe after the parent has used the GPU, where fork is not).
+_POOL = {}
+
+
+def _pool_init(names, shapes, eps, weight_offset, act):
+    from multiprocessing import shared_memory
     import oracle
-    f = workloads.as_f64
-    x, z, w, dy = f(wl.x), f(wl.z), f(wl.w), f(wl.dy)
-    if wl.rows * wl.width > (1 << 26):        # bound host memory and time: a row sample
-        n = max(32, (1 << 26) // wl.width)
-        x, dy = x[:n], dy[:n]
-        z = None if z is None else z[:n]
-        fwd_b, bwd_b = bytes_model(n, wl.width, esize_of(wl), wl.gated)
-    else:
-        n = wl.rows
+    _POOL["orc"] = oracle
+    _POOL["shm"] = [shared_memory.SharedMemory(name=n) for n in names]
+    _POOL["arr"] = [np.ndarray(sh, dtype=np.float64, buffer=m.buf)
+                    for m, sh in zip(_POOL["shm"], shapes)]
+    _POOL["p"] = (eps, weight_offset, act)
+
+
+def _pool_rows(block):
+    a, b = block
+    x, dy, w = _POOL["arr"][0], _POOL["arr"][1], _POOL["arr"][2]
+    z = _POOL["arr"][3] if len(_POOL["arr"]) > 3 else None
+    eps, off, act = _POOL["p"]
+    orc = _POOL["orc"]
+    zz = None if z is None else z[a:b]
+    orc.rmsnorm_fwd(x[a:b], w, eps, off, zz, act)
+    _, _, dw = orc.rmsnorm_bwd(x[a:b], w, dy[a:b], eps, off, zz, act)
+    return dw
+
+
+class OraclePool:
+    """The fp64 oracle over rows [0, n) of a workload on every host core: one
+    worker process per core, each running the unmodified oracle on its own
+    contiguous block of rows, read from shared memory.  pass_() runs one
+    forward + backward over all n rows."""
+
+    def __init__(self, wl, n, procs=None):
+        import multiprocessing as mp
+        from multiprocessing import shared_memory
+        f = workloads.as_f64
+        arrays = [f(wl.x[:n]), f(wl.dy[:n]), f(wl.w)]
+        if wl.z is not None:
+            arrays.append(f(wl.z[:n]))
+        self.shm = []
+        for a in arrays:
+            m = shared_memory.SharedMemory(create=True, size=max(8, a.nbytes))
+            np.ndarray(a.shape, dtype=np.float64, buffer=m.buf)[...] = a
+            self.shm.append(m)
+        self.procs = procs or host_info()["nproc"]
+        step = -(-n // self.procs)
+        self.blocks = [(i, min(n, i + step)) for i in range(0, n, step)]
+        self.pool = mp.get_context("spawn").Pool(
+            self.procs, initializer=_pool_init,
+            initargs=([m.name for m in self.shm], [a.shape for a in arrays], wl.eps,
+                      wl.weight_offset, wl.act))
+        self.pass_()                      # workers started and warm
+
+    def pass_(self):
+        return self.pool.map(_pool_rows, self.blocks, chunksize=1)
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+        for m in self.shm:
+            m.close()
+            m.unlink()
+
+
+def _time_passes(fn, min_s, max_s):
     reps, t0 = 0, time.perf_counter()
     while True:
-        _oracle_step(oracle, wl, x, z, w, dy)
+        fn()
         reps += 1
         el = time.perf_counter() - t0
         if el >= min_s or el * (reps + 1) / reps > max_s:
-            break
-    return {"value": round((fwd_b + bwd_b) * reps / el / 1e9, 4), "unit": "GB/s", "cores": 1,
-            "kind": "oracle",
+            return reps, el
+
+
+def accuracy(wl, out, max_elems=1 << 26):
+    """Parity statistics of one step's outputs against the fp64 oracle, over
+    the workload's rows (its first rows when it has more than ``max_elems``
+    elements): for 16-bit outputs the fraction of y elements correctly rounded
+    (equal to the oracle's value rounded once), the fraction within the plain
+    2-ulp bound, the elements that pass only through the cancellation floor
+    (dx, dz: 2^-16 times the oracle's cancellation scale), those out of
+    tolerance and the largest error in ulps; relative L2 for fp32 tensors.
+    ``out`` holds the device outputs for ``wl``'s inputs."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import numerics
+    import oracle
+    f = workloads.as_f64
+    R, H = wl.rows, wl.width
+    n = R if R * H <= max_elems else max(32, max_elems // H)
+    fmt = {"bf16": numerics.BF16, "f16": numerics.F16}.get(wl.dtype)
+    off, act, eps = wl.weight_offset, wl.act, wl.eps
+    names = ["y", "dx"] + (["dz"] if wl.gated else [])
+    cnt = {k: {} for k in names}
+    l2 = {k: [0.0, 0.0] for k in names + ["rstd"]}
+    dw_ref = np.zeros(H)
+    w = f(wl.w)
+    step = max(1, (1 << 21) // H)
+    for a in range(0, n, step):
+        b = min(n, a + step)
+        x, dy = f(wl.x[a:b]), f(wl.dy[a:b])
+        z = None if wl.z is None else f(wl.z[a:b])
+        ref = {}
+        ref["y"], rho = oracle.rmsnorm_fwd(x, w, eps, off, z, act)
+        ref["dx"], ref["dz"], dw = oracle.rmsnorm_bwd(x, w, dy, eps, off, z, act)
+        dw_ref += dw
+        scale = {"y": None, "dx": oracle.rmsnorm_dx_scale(x, w, dy, eps, off, z, act)}
+        if wl.gated:
+            scale["dz"] = oracle.rmsnorm_dz_scale(x, w, dy, eps, off, z, act)
+        for k in names:
+            g = f(out[k][a:b])
+            if fmt is not None:
+                c = numerics.counts_16(g, ref[k], fmt, scale[k])
+                for key, v in c.items():
+                    cnt[k][key] = max(cnt[k].get(key, 0.0), v) if key == "max_err_ulps" \
+                        else cnt[k].get(key, 0) + v
+            l2[k][0] += float(np.sum((g - ref[k]) ** 2))
+            l2[k][1] += float(np.sum(ref[k] ** 2))
+        gr = f(out["rstd"][a:b])
+        l2["rstd"][0] += float(np.sum((gr - rho) ** 2))
+        l2["rstd"][1] += float(np.sum(rho ** 2))
+    rel = lambda k: round(float(np.sqrt(l2[k][0] / l2[k][1])), 9) if l2[k][1] > 0 else 0.0
+    res = {"rows_checked": n, "of_rows": R,
+           "tolerance": ("16-bit: |gpu - oracle| <= 2 ulp (+ 2^-16 x cancellation scale "
+                         "for dx, dz); fp32: relative L2 <= 1e-4")}
+    for k in names:
+        e = {"rel_l2": rel(k)}
+        if fmt is not None:
+            c, m = cnt[k], max(1, cnt[k]["n"])
+            e.update({"correctly_rounded_pct": round(100.0 * c["correctly_rounded"] / m, 5),
+                      "plain_2ulp_pct": round(100.0 * c["plain_pass"] / m, 5),
+                      "floor_hits": c["floor_hits"], "out_of_tolerance": c["out_of_tolerance"],
+                      "max_err_ulps": round(c["max_err_ulps"], 3), "elements": c["n"]})
+        res[k] = e
+    res["rstd"] = {"rel_l2": rel("rstd")}
+    if n == R:
+        g = f(out["dw"])
+        den = float(np.linalg.norm(dw_ref))
+        res["dw"] = {"rel_l2": round(float(np.linalg.norm(g - dw_ref)) / den, 9) if den else 0.0}
+    return res
+
+
+def cpu_baseline(wl, fwd_b, bwd_b, min_s=10.0, max_s=30.0):
+    """The fp64 oracle, as it stands, over (a bounded sample of) the workload's
+    rows: on every host core (the reported figure) and on one thread."""
+    import oracle
+    f = workloads.as_f64
+    n = wl.rows
+    if wl.rows * wl.width > (1 << 26):        # bound host memory and time: a row sample
+        n = max(32, (1 << 26) // wl.width)
+        fwd_b, bwd_b = bytes_model(n, wl.width, esize_of(wl), wl.gated)
+    x, dy, w = f(wl.x[:n]), f(wl.dy[:n]), f(wl.w)
+    z = None if wl.z is None else f(wl.z[:n])
+    reps1, el1 = _time_passes(lambda: _oracle_step(oracle, wl, x, z, w, dy), min_s, max_s)
+    one = round((fwd_b + bwd_b) * reps1 / el1 / 1e9, 4)
+    host = host_info()
+    pool = OraclePool(wl, n)
+    try:
+        reps, el = _time_passes(pool.pass_, min_s, max_s)
+    finally:
+        pool.close()
+    return {"value": round((fwd_b + bwd_b) * reps / el / 1e9, 4), "unit": "GB/s",
+            "cores": pool.procs, "kind": "oracle",
             "sample": f"fp64 numpy oracle fwd+bwd over rows [0, {n}) of the {wl.rows}-row "
-                      f"workload, {reps} passes in {el:.1f} s, single thread"}
+                      f"workload, split in {len(pool.blocks)} row blocks over {pool.procs} "
+                      f"worker processes (one per core), {reps} passes in {el:.1f} s",
+            "single_thread": {"value": one, "unit": "GB/s", "cores": 1,
+                              "sample": f"same rows, one thread, {reps1} passes in {el1:.1f} s"},
+            "host": host}
 
 
 def run_reference(a):
@@ -547,29 +716,34 @@ def run_reference(a):
         return
     import oracle
     wl = workloads.ALL[a.workload]()
-    R, H, eps = wl.rows, wl.width, wl.eps
+    R, H = wl.rows, wl.width
     f = workloads.as_f64
     fz = (lambda t: None) if not wl.gated else f
-    # size the per-step row sample so the whole run stays near a minute of CPU
+    host = host_info()
+    # size the per-step row sample so the whole run stays near a minute on the
+    # host's cores (a single-thread probe, scaled by the core count)
     probe = min(R, max(32, 4096 * 128 // H))
     t0 = time.perf_counter()
     _oracle_step(oracle, wl, f(wl.x[:probe]), fz(wl.z[:probe] if wl.gated else None), f(wl.w),
                  f(wl.dy[:probe]))
-    per_row = (time.perf_counter() - t0) / probe
+    per_row = (time.perf_counter() - t0) / probe / host["nproc"]
     n = int(60.0 / per_row / max(1, a.steps + a.warmup))
-    n = max(32, min(R, n // 32 * 32))
-    x, w, dy = f(wl.x[:n]), f(wl.w), f(wl.dy[:n])
-    z = f(wl.z[:n]) if wl.gated else None
-    for _ in range(a.warmup):
-        _oracle_step(oracle, wl, x, z, w, dy)
-    t0 = time.perf_counter()
-    for _ in range(a.steps):
-        _oracle_step(oracle, wl, x, z, w, dy)
-    el = time.perf_counter() - t0
+    n = max(32, min(R, (1 << 26) // H, n // 32 * 32))
+    pool = OraclePool(wl, n)
+    try:
+        for _ in range(a.warmup):
+            pool.pass_()
+        t0 = time.perf_counter()
+        for _ in range(a.steps):
+            pool.pass_()
+        el = time.perf_counter() - t0
+    finally:
+        pool.close()
     fwd_b, bwd_b = bytes_model(n, H, esize_of(wl), wl.gated)
     value = (fwd_b + bwd_b) * a.steps / el / 1e9
-    sample = (f"fp64 numpy oracle fwd+bwd on rows [0, {n}) of the {R}-row workload per step "
-              f"(single thread)")
+    sample = (f"fp64 numpy oracle fwd+bwd on rows [0, {n}) of the {R}-row workload per step, "
+              f"split in {len(pool.blocks)} row blocks over {pool.procs} worker processes "
+              f"(one per core)")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
@@ -580,8 +754,8 @@ def run_reference(a):
                    "op": op_name(wl),
                    "rows": R, "width": H, "sample_rows_per_step": n},
         "rows_per_s": round(n * a.steps / el, 1),
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": pool.procs,
+                         "kind": "oracle", "sample": sample, "host": host},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

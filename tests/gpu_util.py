@@ -2,6 +2,9 @@
 with the fp64 oracle."""
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -82,8 +85,24 @@ def oracle_dw(wl, chunk=4096):
     return tot
 
 
+def record(wl, stats, idx=None):
+    """Appends one JSON line of parity statistics to the file named by the
+    RN_ACCURACY_RECORD environment variable, when it is set (the accuracy
+    record kept beside the profiles); a no-op otherwise."""
+    path = os.environ.get("RN_ACCURACY_RECORD")
+    if not path:
+        return
+    line = {"test": os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0],
+            "workload": wl.name, "rows": wl.rows, "width": wl.width, "dtype": wl.dtype,
+            "act": wl.act, "weight_offset": wl.weight_offset,
+            "rows_checked": wl.rows if idx is None else int(len(idx)), "stats": stats}
+    with open(path, "a") as f:
+        f.write(json.dumps(line) + "\n")
+
+
 def compare(out, wl, idx=None, with_dw=True):
-    """Assert the parity tolerances; return statistics."""
+    """Assert the parity tolerances; return statistics (and record them, see
+    record())."""
     ref = oracle_rows(wl, idx)
     g = (lambda k: out[k]) if idx is None else (lambda k: out[k][idx.to(out[k].device)
                                                                  if torch.is_tensor(idx) else idx])
@@ -95,6 +114,7 @@ def compare(out, wl, idx=None, with_dw=True):
         stats["dz"] = check_out(g("dz"), ref["dz"], scale=ref["sdz"], what="dz")
     if with_dw:
         stats["dw"] = check_out(out["dw"], oracle_dw(wl), what="dw")
+    record(wl, stats, idx)
     return stats
 
 

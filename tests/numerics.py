@@ -66,27 +66,49 @@ def to64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").to(torch.float64).numpy()
 
 
+def counts_16(g: np.ndarray, ref: np.ndarray, fmt, scale=None, ulps=2.0,
+              floor=2.0 ** -16) -> dict:
+    """Counts behind the 16-bit tolerance for values ``g`` of format ``fmt``
+    (exact in fp64) against the fp64 reference: elements equal to the
+    reference rounded once to the format (correctly rounded), within the plain
+    ``ulps`` bound, passing only through the cancellation floor
+    (floor * scale), and out of tolerance; the largest error in ulps."""
+    ulp = ulp16(ref, fmt)
+    err = np.abs(g - ref)
+    lim_plain = ulps * ulp
+    lim = lim_plain if scale is None else lim_plain + floor * np.asarray(scale)
+    bad = ~(err <= lim)          # NaN counts as out of tolerance
+    return {
+        "n": int(g.size),
+        "correctly_rounded": int(np.sum(g == round16(ref, fmt))),
+        "plain_pass": int(np.sum(err <= lim_plain)),
+        "floor_hits": int(np.sum((err > lim_plain) & ~bad)),
+        "out_of_tolerance": int(np.sum(bad)),
+        "max_err_ulps": float(np.max(err / ulp)) if g.size else 0.0,
+    }
+
+
 def check_16(got: torch.Tensor, ref: np.ndarray, scale=None, what="", ulps=2.0,
              floor=2.0 ** -16) -> dict:
     """Assert the 16-bit (bf16 or fp16) tolerance; return pass statistics."""
     fmt = FMT_OF[got.dtype]
-    ulp = lambda v: ulp16(v, fmt)
     g = to64(got)
     ref = np.asarray(ref, dtype=np.float64)
     assert g.shape == ref.shape, (what, g.shape, ref.shape)
     assert np.all(np.isfinite(g)), f"{what}: non-finite output"
-    err = np.abs(g - ref)
-    lim_plain = ulps * ulp(ref)
-    lim = lim_plain if scale is None else lim_plain + floor * np.asarray(scale)
-    bad = err > lim
+    c = counts_16(g, ref, fmt, scale, ulps, floor)
+    n = max(1, c["n"])
     stats = {
-        "n": int(g.size),
-        "max_err_ulps": float(np.max(err / ulp(ref))) if g.size else 0.0,
-        "plain_2ulp_pass_frac": float(np.mean(err <= lim_plain)) if g.size else 1.0,
-        "floor_hits": int(np.sum((err > lim_plain) & ~bad)),
-        "correctly_rounded_frac": float(np.mean(g == round16(ref, fmt))) if g.size else 1.0,
+        "n": c["n"],
+        "max_err_ulps": c["max_err_ulps"],
+        "plain_2ulp_pass_frac": c["plain_pass"] / n if c["n"] else 1.0,
+        "floor_hits": c["floor_hits"],
+        "correctly_rounded_frac": c["correctly_rounded"] / n if c["n"] else 1.0,
     }
-    if np.any(bad):
+    if c["out_of_tolerance"]:
+        err = np.abs(g - ref)
+        lim = ulps * ulp16(ref, fmt) + (0.0 if scale is None else floor * np.asarray(scale))
+        bad = err > lim
         i = np.unravel_index(np.argmax(err - lim), err.shape)
         raise AssertionError(
             f"{what}: {int(bad.sum())}/{g.size} elements out of tolerance; worst at {i}: "
