@@ -247,26 +247,51 @@ def run_ours(a):
         return lib.rmsnorm_fwd(R, H, eps, woff, actc, dtc, p["x"], p["z"], p["w"], p["y"],
                                p["rstd"], stp)
 
+    exchange = None
+    if world > 1:
+        # data parallel: every rank returns its 256-row chunk partials of dw; they
+        # are all-gathered in rank order and folded with the declared tree every
+        # step, so the step's dw is that of the whole N-rank batch, bitwise
+        from rollout_parity_b200 import parallel
+        from rollout_parity_b200.ops import rn_fold_tree
+        rows_per_rank = parallel.check_chunk_split(R, device=dev)
+        nch = int(lib.rmsnorm_bwd_chunk_count(R))
+        n_all = sum(-(-r // 256) for r in rows_per_rank)
+        fold_ws = torch.empty(max(16, int(lib.rn_fold_tree_workspace_bytes(n_all, H))),
+                              dtype=torch.uint8, device=dev)
+        for s_, p_ in zip(sets, P):
+            s_["chunks"] = torch.empty(nch, H, dtype=torch.float32, device=dev)
+            p_["chunks"] = s_["chunks"].data_ptr()
+
+        def exchange(s_):
+            parallel.chunk_split_dw(
+                s_["chunks"], R, rows_per_rank=rows_per_rank,
+                fold=lambda g: rn_fold_tree(g, out=s_["dw"], ws=fold_ws))
+        a.no_graph = True      # NCCL calls stay outside graph capture
+
     def bwd(p, stp=sp):
+        if exchange is not None:
+            return lib.rmsnorm_bwd_chunks(R, H, eps, woff, actc, dtc, p["x"], p["z"], p["w"],
+                                          p["dy"], p["rstd"], None, p["dx"], p["dz"],
+                                          p["chunks"], p["ws"], nws, stp)
         return lib.rmsnorm_bwd(R, H, eps, woff, actc, dtc, p["x"], p["z"], p["w"], p["dy"],
                                p["rstd"], None, p["dx"], p["dz"], p["dw"], p["ws"], nws, stp)
 
     for p in P:                       # every set gets its rstd before any backward
         check("rmsnorm_fwd", fwd(p))
-    for k in range(a.warmup):
+    n_launch = None                   # our kernels per step, counted by the library
+    for k in range(max(1, a.warmup)):
         check("rmsnorm_fwd", fwd(P[k % nsets]))
+        nl = lib.rn_last_launches()
         check("rmsnorm_bwd", bwd(P[(k + 2) % nsets]))
+        nl += lib.rn_last_launches()
+        if exchange is not None:
+            exchange(sets[(k + 2) % nsets])
+            nl += lib.rn_last_launches()
+        n_launch = nl
     torch.cuda.synchronize()
 
     K = a.steps
-    exchange = None
-    if world > 1:
-        # data parallel: the ranks' dw are joined every step by an all-gather and
-        # the same pairwise fold, so the step's dw is that of the whole N-rank batch
-        from rollout_parity_b200 import parallel
-        parallel.check_shard_rows(R, device=dev)
-        exchange = parallel.fold_gathered_dw
-        a.no_graph = True      # NCCL calls stay outside graph capture
     G = K if a.no_graph else graph_steps(K)
     # per-call events for the roofline: G steps recorded in a separate graph (or,
     # without graphs, every step of the timed loop)
@@ -321,7 +346,7 @@ def run_ours(a):
             e[1].record(stream)
             s2 = bwd(P[(k + 2) % nsets])
             if exchange is not None:
-                exchange(sets[(k + 2) % nsets]["dw"])
+                exchange(sets[(k + 2) % nsets])
             e[2].record(stream)
             if s1 or s2:
                 check("rmsnorm_fwd", s1)
@@ -346,8 +371,8 @@ def run_ours(a):
     ms_step = ms / K
     value = world * step_b * K / (ms / 1e3) / 1e9
     # our kernels per step: the forward, the backward and its fold passes, and
-    # with N ranks the rn_fold_rows pass of the dw exchange
-    launches = K * (1 + lib.rn_bwd_launches(R, H, dtc) + (1 if exchange is not None else 0))
+    # with N ranks the rn_fold_tree passes of the dw exchange
+    launches = K * n_launch
 
     inv = invariance_checks(rn, sets[0], R, H, eps, wl0) \
         if rank == 0 and not a.no_invariance else None
@@ -381,8 +406,8 @@ def run_ours(a):
                        "accumulate": "fp32",
                        "bytes_per_step": step_b,
                        "parallelism": (f"data parallel x{world}: rows split across ranks, dw "
-                                       "all-gathered and folded each step" if world > 1
-                                       else "one GPU"),
+                                       "chunk partials all-gathered and folded each step"
+                                       if world > 1 else "one GPU"),
                        "launch": ("python loop" if a.no_graph else
                                   f"CUDA graph of {G} steps replayed {K // G} times"),
                        "per_call_timing": ("events in the timed loop" if a.no_graph else
@@ -475,19 +500,23 @@ def run_e2e(rn, wl, dev, steps, step_b, world, dist):
         w.copy_(hw, non_blocking=True)
         zz = z if gated else None
         rn.rmsnorm_fwd(x, w, eps, wl.weight_offset, zz, wl.act, y=y, rstd=rstd)
-        rn.rmsnorm_bwd(x, w, dy, rstd, eps, wl.weight_offset, zz, wl.act, dx=dx,
-                       dz=dz if gated else None, dw=dw, ws=ws)
+        if dist is None:
+            rn.rmsnorm_bwd(x, w, dy, rstd, eps, wl.weight_offset, zz, wl.act, dx=dx,
+                           dz=dz if gated else None, dw=dw, ws=ws)
+            odw.copy_(dw, non_blocking=True)
+        else:   # with N ranks the step's dw is the whole batch's (chunk partials folded)
+            _, _, ch = rn.rmsnorm_bwd_chunks(x, w, dy, rstd, eps, wl.weight_offset, zz, wl.act,
+                                             dx=dx, dz=dz if gated else None, ws=ws)
+            odw.copy_(chunk_split_dw(ch, R, rows_per_rank=rows_per_rank), non_blocking=True)
         oy.copy_(y, non_blocking=True)
         ors.copy_(rstd, non_blocking=True)
         odx.copy_(dx, non_blocking=True)
         if gated:
             odz.copy_(dz, non_blocking=True)
-        # with N ranks the step's dw is the whole batch's (the all-gather fold)
-        odw.copy_(dw if dist is None else fold_dw(dw), non_blocking=True)
 
-    fold_dw = None
     if dist is not None:
-        from rollout_parity_b200.parallel import fold_gathered_dw as fold_dw
+        from rollout_parity_b200.parallel import check_chunk_split, chunk_split_dw
+        rows_per_rank = check_chunk_split(R, device=dev)
     for _ in range(3):
         step()
     torch.cuda.synchronize()
@@ -508,8 +537,8 @@ def run_e2e(rn, wl, dev, steps, step_b, world, dist):
     return {"value": round(world * step_b * steps / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 4),
-            "api": "rollout_parity_b200.rmsnorm_fwd/rmsnorm_bwd" +
-                   ("" if dist is None else " + parallel.fold_gathered_dw")}
+            "api": "rollout_parity_b200.rmsnorm_fwd/rmsnorm_bwd" if dist is None else
+                   "rollout_parity_b200.rmsnorm_fwd/rmsnorm_bwd_chunks + parallel.chunk_split_dw"}
 
 
 # ---------------------------------------------------------------------------

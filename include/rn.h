@@ -238,6 +238,47 @@ rn_status gated_norm_bwd(int64_t rows, int32_t width, float eps, rn_dtype dt,
                          float* dw, void* ws, size_t ws_bytes, rn_stream stream);
 
 /*
+ * Data-parallel dw (RFC #415 section 4: the result must not depend on rank
+ * placement).  dw's declared tree over 32-row leaves is, from its third level
+ * up, the same level-by-level pairwise tree over 256-row chunks, whose node for
+ * chunk c is the tree over leaves 8c .. 8c+7 (fewer for a ragged last chunk).
+ * So when a batch is split across ranks in row order on 256-row boundaries
+ * (every rank but the last holds a multiple of 256 rows), each rank can return
+ * its chunk partials, and the tree over all ranks' chunk partials in rank
+ * order is bitwise the dw of one call over the whole batch.
+ *
+ * rmsnorm_bwd_chunk_count: ceil(rows / 256), the chunk partials of `rows`
+ * rows (0 for rows < 0 or > 2^36).
+ *
+ * rmsnorm_bwd_chunks: rmsnorm_bwd (same arguments, same dx and dz, same
+ * workspace), except that dw_chunks [rmsnorm_bwd_chunk_count(rows)][width]
+ * fp32, written, receives the chunk partials instead of their fold.  rows == 0
+ * writes nothing (dw_chunks may then be NULL).  A left-out row (row_mask) is
+ * the identity -0.0, as in rmsnorm_bwd.
+ */
+int64_t rmsnorm_bwd_chunk_count(int64_t rows);
+rn_status rmsnorm_bwd_chunks(int64_t rows, int32_t width, float eps, float weight_offset,
+                             rn_act act, rn_dtype dt, const void* x, const void* z,
+                             const float* w, const void* dy, const float* rstd,
+                             const uint8_t* row_mask, void* dx, void* dz, float* dw_chunks,
+                             void* ws, size_t ws_bytes, rn_stream stream);
+
+/*
+ * The level-by-level pairwise tree over n >= 1 rows of fp32 partials, in row
+ * order (node 2i + node 2i+1 at each level, an odd last node carried up):
+ * out[width] = tree(in[0], ..., in[n-1]).  Folding the chunk partials of
+ * rmsnorm_bwd_chunks gives that call's dw bits; folding several ranks' chunk
+ * partials concatenated in rank order gives the dw of the whole batch.
+ * in: [n][width] fp32 device, read.  out: [width] fp32 device, written.
+ * ws: device workspace of ws_bytes >= rn_fold_tree_workspace_bytes(n, width),
+ * 16-byte aligned, contents irrelevant.  No overlap between in, out and ws.
+ * RN_E_ARG for n < 1 or > 2^36; other errors as the backward's.
+ */
+size_t rn_fold_tree_workspace_bytes(int64_t n, int32_t width);
+rn_status rn_fold_tree(int64_t n, int32_t width, const float* in, float* out, void* ws,
+                       size_t ws_bytes, rn_stream stream);
+
+/*
  * Joins n rows of fp32 dw partials with the same level-by-level pairwise tree
  * the backward uses: out[width] = tree(in[0], ..., in[n-1]), in row order.
  * A backward call's dw is the root of that tree over its 32-row leaves, so
@@ -309,6 +350,14 @@ const char* rn_status_string(rn_status s);
 
 /* The cudaError_t behind this thread's last RN_E_CUDA (0 if none). */
 int rn_last_cuda_error(void);
+
+/*
+ * Number of kernels the last call made on this thread enqueued (forward,
+ * backward, chunk backward, rn_fold_tree, rn_fold_rows; 0 after a failed
+ * check or in validate-only mode).  For bookkeeping: a benchmark counts the
+ * library's kernels per step with it.
+ */
+int32_t rn_last_launches(void);
 
 /*
  * Test knobs (process-wide; not for production use).  They change how work

@@ -20,6 +20,8 @@ from .ops import (  # noqa: F401
     rmsnorm_add_bwd,
     rmsnorm_add_fwd,
     rmsnorm_bwd,
+    rmsnorm_bwd_chunks,
+    rn_fold_tree,
     rmsnorm_fwd,
     workspace,
 )

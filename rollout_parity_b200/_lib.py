@@ -63,11 +63,17 @@ SIGNATURES = {
                                c_vp, c_vp, c_vp, c_sz, c_vp]),
     "gated_norm_bwd_static_ws": (c_i32, [c_i64, c_i32, c_f32, c_i32, c_vp, c_vp, c_vp, c_vp,
                                          c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "rmsnorm_bwd_chunk_count": (c_i64, [c_i64]),
+    "rmsnorm_bwd_chunks": (c_i32, [c_i64, c_i32, c_f32, c_f32, c_i32, c_i32, c_vp, c_vp, c_vp,
+                                   c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "rn_fold_tree_workspace_bytes": (c_sz, [c_i64, c_i32]),
+    "rn_fold_tree": (c_i32, [c_i64, c_i32, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "rn_fold_rows": (c_i32, [c_i64, c_i32, c_vp, c_vp, c_vp]),
     "rn_describe": (ctypes.c_char_p, [c_i32, c_i32]),
     "rn_bwd_launches": (c_i32, [c_i64, c_i32, c_i32]),
     "rn_status_string": (ctypes.c_char_p, [c_i32]),
     "rn_last_cuda_error": (ctypes.c_int, []),
+    "rn_last_launches": (c_i32, []),
     "rn_test_set_geometry": (c_i32, [c_i32, c_i32, c_i32]),
     "rn_test_set_validate_only": (None, [c_i32]),
     "rn_test_rcp_1to2": (c_i32, [c_i64, c_vp, c_vp, c_i32, c_vp]),

@@ -28,6 +28,7 @@ using namespace rn_detail;
 
 std::atomic<int> g_max_ctas{0}, g_leaves_per_cta{0}, g_fold_rows{0}, g_validate_only{0};
 thread_local int t_last_cuda = 0;
+thread_local int t_launches = 0;   // kernels the current / last call enqueued
 thread_local char t_describe[512];
 
 // ---------------------------------------------------------------------------
@@ -350,16 +351,21 @@ rn_status launch_fold(int B, dim3 grid, cudaStream_t st, const float* in, int64_
   }
 }
 
-// Folds n group partials (rows of width H in `a`) into dw, ping-ponging
-// between the two workspace regions a and b.
-rn_status run_fold(float* a, float* b, int64_t n, int H, float* dw, cudaStream_t st) {
-  float* src = a;
+// Folds n rows of partials (width H, in `src`) into dw with the level-by-level
+// pairwise tree.  The first pass reads src and writes b; later passes
+// ping-pong between b and a (so src may be a itself).  Every pass folds
+// aligned blocks of rows (perfect subtrees), so the bits do not depend on the
+// rows per pass.
+rn_status run_fold(const float* src, float* a, float* b, int64_t n, int H, float* dw,
+                   cudaStream_t st) {
+  const float* in = src;
   float* dst = b;
+  float* other = a;
   rn_status e = RN_OK;
   while (n > 1) {
     int S = g_fold_rows.load();
     if (use_fold1(n))
-      return launch_pdl(k_fold1, dim3(unsigned((H + 7) / 8)), dim3(1024), 0, st, src, n, H, dw);
+      return launch_pdl(k_fold1, dim3(unsigned((H + 7) / 8)), dim3(1024), 0, st, in, n, H, dw);
     if (S <= 0) S = fold_rows_default(n);
     const int B = S / kFoldRG;
     const int64_t nout = (n + S - 1) / S;
@@ -367,27 +373,66 @@ rn_status run_fold(float* a, float* b, int64_t n, int H, float* dw, cudaStream_t
     const int gy = (H / 4 + 31) / 32;    // <= 128 column tiles
     if (nout > 0x7fffffff) return RN_E_ARG;   // unreachable for rows <= 2^36
     dim3 grid(unsigned(nout), gy);
-    e = launch_fold(B, grid, st, src, n, H, o);
+    e = launch_fold(B, grid, st, in, n, H, o);
     if (e != RN_OK) return e;
+    if (o == dw) return RN_OK;
     n = nout;
-    float* tmp = src;
-    src = dst;
-    dst = tmp;
+    in = dst;
+    float* tmp = dst;
+    dst = other;
+    other = tmp;
+  }
+  if (in != dw) {   // one row from the start: dw is that row
+    if (cudaMemcpyAsync(dw, in, size_t(H) * sizeof(float), cudaMemcpyDeviceToDevice, st) !=
+        cudaSuccess)
+      return launch_status();
   }
   return RN_OK;
 }
 
+// Workspace of rn_fold_tree: the first pass's output (at most ceil(n/8) rows)
+// and the second's (at most ceil(n/64) rows).
+size_t fold_ws_bytes_of(int64_t n, int32_t width) {
+  if (n <= 0 || n > kMaxRows || !width_ok(width)) return 0;
+  const int64_t r1 = (n + kFoldRG - 1) / kFoldRG;
+  const int64_t r2 = (r1 + kFoldRG - 1) / kFoldRG;
+  return size_t(r1 + r2) * size_t(width) * sizeof(float);
+}
+
+constexpr int kChunkLeaves = 8;                       // 256 rows: one chunk partial
+constexpr int kChunkRows = kChunkLeaves * kLeafRows;
+
 // dres (residual-add backward) may be NULL; dx may be exactly dres.
+// Leaves per backward CTA when the call returns chunk partials: 8 (a CTA's
+// group partial is then a chunk partial) when the kernel takes 8, else 1 (and
+// one fold pass of 8 leaf partials per chunk follows).
+int chunk_leaves_per_cta(const Sched& s, int width, rn_dtype dt) {
+  const int req = g_leaves_per_cta.load();
+  if (is_stripe(s, width, dt)) return req == 1 ? 1 : kChunkLeaves;
+  if (req == 1) return 1;
+  int lpc = bwd_max_block_of(s.T) / s.T;
+  if (s.T > 32 && width > 2048) lpc = 1;
+  if (lpc >= kChunkLeaves && bwd_smem_bytes(s, kChunkLeaves, width, true, dt) <= kSmemCap)
+    return kChunkLeaves;
+  return 1;
+}
+
+int64_t n_chunks_of(int64_t rows) { return (rows + kChunkRows - 1) / kChunkRows; }
+
+// chunks: dw receives the chunk partials [n_chunks_of(rows)][width] instead of
+// their fold.
 rn_status bwd_entry(int64_t rows, int32_t width, float eps, float woff, rn_act act, rn_dtype dt,
                     const void* x, const void* z, const float* w, const void* dy,
                     const float* rstd, const uint8_t* mask, const void* dres, void* dx, void* dz,
-                    float* dw, void* ws, size_t ws_bytes, rn_stream stream) {
+                    float* dw, void* ws, size_t ws_bytes, rn_stream stream,
+                    bool chunks = false) {
+  t_launches = 0;
   rn_status e = common_checks(rows, width, eps, dt);
   if (e != RN_OK) return e;
   if (!act_ok(act) || !std::isfinite(woff)) return RN_E_ARG;
   const bool gated = act != RN_ACT_NONE;
   if (!gated && (z || dz)) return RN_E_ARG;   // no gate: z and dz must be NULL
-  if (!w || !dw) return RN_E_ARG;
+  if (!w || (!dw && !(chunks && rows == 0))) return RN_E_ARG;   // no rows: no chunk partial
   if (rows > 0 && (!x || !dy || !dx || (gated && (!z || !dz)))) return RN_E_ARG;
   const size_t tb = rows > 0 ? size_t(rows) * size_t(width) * elem_bytes(dt) : 0;
   const size_t need = ws_bytes_of(rows, width);
@@ -404,44 +449,56 @@ rn_status bwd_entry(int64_t rows, int32_t width, float eps, float woff, rn_act a
   const Range in[] = {{x, tb}, {z, tb}, {w, size_t(width) * 4},
                       {dy, tb}, {rstd, rstd ? size_t(rows) * 4 : 0},
                       {mask, mask ? size_t(rows) : 0}, {dres, tb}};
-  const Range out[] = {{dx, tb}, {dz, tb}, {dw, size_t(width) * 4},
+  const size_t dw_bytes = size_t(chunks ? n_chunks_of(rows) : 1) * size_t(width) * 4;
+  const Range out[] = {{dx, tb}, {dz, tb}, {dw, dw_bytes},
                        {ws, rows > 0 ? need : 0}};
   e = check_ranges(in, 7, out, 4, 0, 6);   // dx may be dres itself
   if (e != RN_OK) return e;
   if (g_validate_only.load()) return RN_OK;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (rows == 0 && chunks) return RN_OK;   // no chunk, nothing to write
   if (rows == 0) {   // dw is the empty sum
     k_fill_neg_zero<<<(width + 255) / 256, 256, 0, st>>>(dw, width);
     return launch_status();
   }
   Sched s;
   bwd_sched(width, dt, &s);
-  const int lpc = leaves_per_cta(s, width, dt, rows);
+  const int lpc = chunks ? chunk_leaves_per_cta(s, width, dt) : leaves_per_cta(s, width, dt, rows);
   const int64_t leaves = n_leaves_of(rows);
   const int64_t groups = (leaves + lpc - 1) / lpc;
   float* region_a = static_cast<float*>(ws);
   float* region_b = region_a + size_t(leaves) * width;
+  // where the backward kernel's group partials go: dw itself when they are
+  // the result (one group, or chunk partials), else the workspace
+  const bool direct = chunks ? lpc == kChunkLeaves : groups == 1;
   const bool pow2 = (width & (width - 1)) == 0;
   BwdArgs a{rows, width, width / vec_elems(dt), eps, 1.0f / float(width), pow2 ? 1 : 0, woff,
             static_cast<const uint4*>(x), static_cast<const uint4*>(z), w,
             static_cast<const uint4*>(dy), rstd, mask, static_cast<const uint4*>(dres),
             static_cast<uint4*>(dx), static_cast<uint4*>(dz),
-            groups == 1 ? dw : region_a};
+            direct ? dw : region_a};
   switch (dt) {
     case RN_BF16: e = launch_bwd<RN_BF16>(act, dres != nullptr, s, lpc, a, groups, st); break;
     case RN_F16: e = launch_bwd<RN_F16>(act, dres != nullptr, s, lpc, a, groups, st); break;
     default: e = launch_bwd<RN_F32>(act, dres != nullptr, s, lpc, a, groups, st); break;
   }
   if (e != RN_OK) return e;
-  if (groups == 1) return RN_OK;
-  return run_fold(region_a, region_b, groups, width, dw, st);
+  if (direct) return RN_OK;
+  if (chunks) {   // leaf partials (lpc == 1): one pass folds each chunk's 8 leaves
+    const int64_t nc = n_chunks_of(rows);
+    if (nc > 0x7fffffff) return RN_E_ARG;   // unreachable for rows <= 2^36
+    return launch_fold(1, dim3(unsigned(nc), unsigned((width / 4 + 31) / 32)), st, region_a,
+                       leaves, width, dw);
+  }
+  return run_fold(region_a, region_a, region_b, groups, width, dw, st);
 }
 
 // r, h (residual-add forward): both NULL, or both given; h may be exactly x or r.
 rn_status fwd_entry(int64_t rows, int32_t width, float eps, float woff, rn_act act, rn_dtype dt,
                     const void* x, const void* r, const void* z, const float* w, void* h, void* y,
                     float* rstd, rn_stream stream) {
+  t_launches = 0;
   rn_status e = common_checks(rows, width, eps, dt);
   if (e != RN_OK) return e;
   if (!act_ok(act) || !std::isfinite(woff)) return RN_E_ARG;
@@ -515,6 +572,7 @@ rn_status launch_status() {
     t_last_cuda = int(e);
     return RN_E_CUDA;
   }
+  ++t_launches;
   return RN_OK;
 }
 
@@ -620,7 +678,42 @@ rn_status gated_norm_bwd(int64_t rows, int32_t width, float eps, rn_dtype dt, co
                    dx, dz, dw, ws, ws_bytes, stream);
 }
 
+int64_t rmsnorm_bwd_chunk_count(int64_t rows) {
+  return rows < 0 || rows > kMaxRows ? 0 : n_chunks_of(rows);
+}
+
+rn_status rmsnorm_bwd_chunks(int64_t rows, int32_t width, float eps, float weight_offset,
+                             rn_act act, rn_dtype dt, const void* x, const void* z,
+                             const float* w, const void* dy, const float* rstd,
+                             const uint8_t* row_mask, void* dx, void* dz, float* dw_chunks,
+                             void* ws, size_t ws_bytes, rn_stream stream) {
+  return bwd_entry(rows, width, eps, weight_offset, act, dt, x, z, w, dy, rstd, row_mask, nullptr,
+                   dx, dz, dw_chunks, ws, ws_bytes, stream, true);
+}
+
+size_t rn_fold_tree_workspace_bytes(int64_t n, int32_t width) { return fold_ws_bytes_of(n, width); }
+
+rn_status rn_fold_tree(int64_t n, int32_t width, const float* in, float* out, void* ws,
+                       size_t ws_bytes, rn_stream stream) {
+  t_launches = 0;
+  if (n < 1 || n > kMaxRows) return RN_E_ARG;
+  if (!width_ok(width)) return RN_E_WIDTH;
+  if (!in || !out) return RN_E_ARG;
+  if (!aligned16(in) || !aligned16(out)) return RN_E_ALIGN;
+  const size_t need = fold_ws_bytes_of(n, width);
+  if (!ws || ws_bytes < need) return RN_E_WORKSPACE;
+  if (!aligned16(ws)) return RN_E_ALIGN;
+  const Range rin[] = {{in, size_t(n) * width * sizeof(float)}};
+  const Range rout[] = {{out, size_t(width) * sizeof(float)}, {ws, need}};
+  const rn_status e = check_ranges(rin, 1, rout, 2);
+  if (e != RN_OK || g_validate_only.load()) return e;
+  float* r1 = static_cast<float*>(ws);
+  float* r2 = r1 + size_t((n + kFoldRG - 1) / kFoldRG) * width;
+  return run_fold(in, r2, r1, n, width, out, static_cast<cudaStream_t>(stream));
+}
+
 rn_status rn_fold_rows(int64_t n, int32_t width, const float* in, float* out, rn_stream stream) {
+  t_launches = 0;
   if (n < 1 || n > 256) return RN_E_ARG;
   if (!width_ok(width)) return RN_E_WIDTH;
   if (!in || !out) return RN_E_ARG;
@@ -678,6 +771,8 @@ const char* rn_status_string(rn_status s) {
 }
 
 int rn_last_cuda_error(void) { return t_last_cuda; }
+
+int32_t rn_last_launches(void) { return t_launches; }
 
 rn_status rn_test_set_geometry(int32_t max_ctas, int32_t leaves_per_cta_req, int32_t fold_rows) {
   auto pow2 = [](int v) { return v > 0 && (v & (v - 1)) == 0; };

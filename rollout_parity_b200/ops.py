@@ -319,6 +319,69 @@ def gated_norm_bwd(x: torch.Tensor, z: torch.Tensor, w: torch.Tensor, dy: torch.
     return dx, dz, dw
 
 
+def rmsnorm_bwd_chunks(x: torch.Tensor, w: torch.Tensor, dy: torch.Tensor,
+                       rstd: Optional[torch.Tensor] = None, eps: float = 1e-6,
+                       weight_offset: float = 1.0, z: Optional[torch.Tensor] = None, act=None, *,
+                       row_mask: Optional[torch.Tensor] = None,
+                       dx: Optional[torch.Tensor] = None, dz: Optional[torch.Tensor] = None,
+                       dw_chunks: Optional[torch.Tensor] = None,
+                       ws: Optional[torch.Tensor] = None, stream=None):
+    """rmsnorm_bwd returning dw's 256-row chunk partials [ceil(rows/256), width]
+    in place of dw (for the data-parallel fold).  Returns (dx, dz, dw_chunks)."""
+    rows, width = _rows_width(x)
+    a = act_code(act)
+    if a == Act.NONE:
+        if z is not None or dz is not None:
+            raise ValueError("z or dz given without a gate activation")
+    else:
+        _mat("z", z, x)
+        dz = torch.empty_like(x) if dz is None else _mat("dz", dz, x)
+    _vec("w", w, width, x.device)
+    _mat("dy", dy, x)
+    if rstd is not None:
+        _vec("rstd", rstd, rows, x.device)
+    if row_mask is not None:
+        if row_mask.dtype not in (torch.bool, torch.uint8) or tuple(row_mask.shape) != (rows,) \
+                or row_mask.device != x.device or not row_mask.is_contiguous():
+            raise ValueError(f"row_mask must be a contiguous bool/uint8 [{rows}] tensor on {x.device}")
+        row_mask = row_mask.view(torch.uint8)
+    nc = int(load().rmsnorm_bwd_chunk_count(rows))
+    dx = torch.empty_like(x) if dx is None else _mat("dx", dx, x)
+    if dw_chunks is None:
+        dw_chunks = torch.empty(nc, width, dtype=torch.float32, device=x.device)
+    elif (dw_chunks.device != x.device or dw_chunks.dtype != torch.float32
+          or tuple(dw_chunks.shape) != (nc, width) or not dw_chunks.is_contiguous()):
+        raise ValueError(f"dw_chunks must be a contiguous fp32 [{nc}, {width}] tensor on {x.device}")
+    ws, nws = _ws(rows, width, x.device, ws)
+    with torch.cuda.device(x.device):
+        check("rmsnorm_bwd_chunks",
+              load().rmsnorm_bwd_chunks(rows, width, eps, weight_offset, int(a), _dt(x), _ptr(x),
+                                        _ptr(z), _ptr(w), _ptr(dy), _ptr(rstd), _ptr(row_mask),
+                                        _ptr(dx), _ptr(dz), _ptr(dw_chunks), _ptr(ws), nws,
+                                        _stream(x, stream)))
+    return dx, dz, dw_chunks
+
+
+def rn_fold_tree(partials: torch.Tensor, *, out: Optional[torch.Tensor] = None,
+                 ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The level-by-level pairwise tree over the rows of a [n, width] fp32 CUDA
+    tensor (any n >= 1); returns the [width] result."""
+    if partials.dim() != 2 or partials.dtype != torch.float32 or not partials.is_cuda \
+            or not partials.is_contiguous():
+        raise ValueError("partials must be a contiguous fp32 CUDA tensor [n, width]")
+    n, width = int(partials.shape[0]), int(partials.shape[1])
+    out = torch.empty(width, dtype=torch.float32, device=partials.device) if out is None else \
+        _vec("out", out, width, partials.device)
+    if ws is None:
+        nb = int(load().rn_fold_tree_workspace_bytes(n, width))
+        ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=partials.device)
+    with torch.cuda.device(partials.device):
+        check("rn_fold_tree", load().rn_fold_tree(n, width, _ptr(partials), _ptr(out), _ptr(ws),
+                                                  ws.numel() * ws.element_size(),
+                                                  _stream(partials, stream)))
+    return out
+
+
 def rn_fold_rows(partials: torch.Tensor, *, out: Optional[torch.Tensor] = None,
                  stream=None) -> torch.Tensor:
     """Joins the rows of a [n, width] fp32 CUDA tensor of dw partials with the

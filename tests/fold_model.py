@@ -66,3 +66,15 @@ def dw_tree(contribs: np.ndarray, add: Callable = _f32_add) -> np.ndarray:
 def tree_shape(n: int) -> str:
     """The tree over n nodes written out, e.g. tree_shape(5) == '(((0+1)+(2+3))+4)'."""
     return pairwise_tree([str(i) for i in range(n)], lambda a, b: f"({a}+{b})")
+
+
+CHUNK_ROWS = 256
+
+
+def chunk_partials(contribs: np.ndarray, add: Callable = _f32_add) -> np.ndarray:
+    """contribs: [rows, width] fp32 one-row dws -> the 256-row chunk partials
+    [ceil(rows/256), width]: chunk c is the declared tree over the leaves of
+    rows [256 c, 256 c + 256) (fewer in a ragged last chunk)."""
+    contribs = np.asarray(contribs, dtype=np.float32)
+    return np.stack([dw_tree(contribs[s:s + CHUNK_ROWS], add)
+                     for s in range(0, contribs.shape[0], CHUNK_ROWS)])

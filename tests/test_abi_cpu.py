@@ -21,7 +21,7 @@ def header_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(
-        r"^(?:rn_status|size_t|const char\s*\*|int32_t|int|void)\s+(\w+)\s*\(", text,
+        r"^(?:rn_status|size_t|const char\s*\*|int64_t|int32_t|int|void)\s+(\w+)\s*\(", text,
         flags=re.M)))
 
 
@@ -412,3 +412,55 @@ def test_binding_rejects_host_tensors(lib):
     w = torch.zeros(128)
     with pytest.raises(ValueError):
         rn.norm_fwd(x, w)
+
+
+def cbwd(lib, rows=R, width=H, act=Act.SILU, woff=0.0, dt=DType.BF16, **kw):
+    ptr = dict(x=P(X), z=P(Z), w=P(W), dy=P(DY), rstd=P(RS), dx=P(DX), dz=P(DZ), dw=P(DW),
+               ws=P(WS))
+    ptr.update(kw)
+    nws = kw.get("ws_bytes", lib.norm_bwd_workspace_bytes(rows, width))
+    return lib.rmsnorm_bwd_chunks(rows, width, 1e-6, woff, act, dt, ptr["x"], ptr["z"], ptr["w"],
+                                  ptr["dy"], ptr["rstd"], ptr.get("mask"), ptr["dx"], ptr["dz"],
+                                  ptr["dw"], ptr["ws"], nws, None)
+
+
+def test_chunk_count(lib):
+    for rows, want in ((0, 0), (1, 1), (256, 1), (257, 2), (262144, 1024), (-1, 0),
+                       ((1 << 36) + 1, 0)):
+        assert lib.rmsnorm_bwd_chunk_count(rows) == want, rows
+
+
+def test_chunk_backward_checks(lib):
+    with validate_only(lib):
+        assert cbwd(lib) == Status.OK
+        assert cbwd(lib, act=Act.NONE, woff=1.0, z=0, dz=0) == Status.OK
+        assert cbwd(lib, rows=0, x=0, z=0, dy=0, dx=0, dz=0, ws=0, rstd=0) == Status.OK
+        assert cbwd(lib, rows=0, x=0, z=0, dy=0, dx=0, dz=0, ws=0, rstd=0, dw=0) == Status.OK
+        assert cbwd(lib, ws=0) == Status.E_WORKSPACE
+        assert cbwd(lib, dw=0) == Status.E_ARG
+        assert cbwd(lib, width=20) == Status.E_WIDTH
+        # the chunk partials span ceil(R/256) rows of width floats: an output
+        # that starts inside them overlaps (a [width] dw would not reach it)
+        nc = lib.rmsnorm_bwd_chunk_count(1000)
+        assert nc == 4
+        assert cbwd(lib, rows=1000, dx=P(DW, H * 4 * (nc - 1))) == Status.E_ARG
+        assert rbwd(lib, rows=1000, act=Act.SILU, woff=0.0, dx=P(DW, H * 4 * (nc - 1))) == \
+            Status.OK
+
+
+def test_fold_tree_checks(lib):
+    need = lib.rn_fold_tree_workspace_bytes(3000, 128)
+    assert need == (375 + 47) * 128 * 4
+    assert lib.rn_fold_tree_workspace_bytes(0, 128) == 0
+    assert lib.rn_fold_tree_workspace_bytes(8, 12) == 0
+    with validate_only(lib):
+        assert lib.rn_fold_tree(3000, 128, P(X), P(Y), P(WS), need, None) == Status.OK
+        assert lib.rn_fold_tree(1, 128, P(X), P(Y), P(WS), 1024, None) == Status.OK
+        assert lib.rn_fold_tree(0, 128, P(X), P(Y), P(WS), need, None) == Status.E_ARG
+        assert lib.rn_fold_tree(3000, 128, P(X), P(Y), P(WS), need - 1, None) == Status.E_WORKSPACE
+        assert lib.rn_fold_tree(3000, 128, P(X), P(Y), 0, need, None) == Status.E_WORKSPACE
+        assert lib.rn_fold_tree(3000, 12, P(X), P(Y), P(WS), need, None) == Status.E_WIDTH
+        assert lib.rn_fold_tree(3000, 128, P(X, 4), P(Y), P(WS), need, None) == Status.E_ALIGN
+        assert lib.rn_fold_tree(3000, 128, P(X), P(X, 512), P(WS), need, None) == Status.E_ARG
+        assert lib.rn_fold_tree(3000, 128, P(X), P(Y), P(X, 1024), need, None) == Status.E_ARG
+        assert lib.rn_fold_tree(3000, 128, P(X), P(Y), P(Y), need, None) == Status.E_ARG

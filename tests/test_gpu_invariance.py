@@ -230,3 +230,74 @@ def test_norm_input_sign_symmetry(cuda_lib):
     b = run(cuda_lib, workloads.Workload(**{**wl.__dict__, "x": -wl.x}))
     assert torch.equal(bits(b["y"]), bits(-a["y"])) and torch.equal(bits(b["dw"]), bits(-a["dw"]))
     assert torch.equal(bits(b["rstd"]), bits(a["rstd"])) and torch.equal(bits(b["dx"]), bits(a["dx"]))
+
+
+def _alone_and_shifted(cuda_lib, wl, full, rows, seed, keys):
+    """Each row in ``rows`` computed alone, and inside other data at a shifted
+    row offset, gives the bits it has in ``full``."""
+    rng = np.random.default_rng(seed)
+    for r in rows:
+        r = int(r)
+        one = run(cuda_lib, sub(wl, r, r + 1))
+        for k in keys:
+            assert torch.equal(bits(one[k]), bits(full[k][r:r + 1])), (k, r, "alone")
+        before, after = int(rng.integers(1, 40)), int(rng.integers(0, 9))
+        pad = workloads.make(wl.op, before + after, wl.width, wl.dtype, seed=r + 11,
+                             act=wl.act if wl.op == "general" else None,
+                             weight_offset=wl.weight_offset if wl.op == "general" else None
+                             ).to(DEV)
+        cat = lambda a, b: None if a is None else \
+            torch.cat([b[:before], a[r:r + 1], b[before:]]).contiguous()
+        moved = dataclasses.replace(wl, rows=before + 1 + after, x=cat(wl.x, pad.x),
+                                    z=cat(wl.z, pad.z), dy=cat(wl.dy, pad.dy), seq_lens=None)
+        out = run(cuda_lib, moved)
+        for k in keys:
+            assert torch.equal(bits(out[k][before:before + 1]), bits(full[k][r:r + 1])), \
+                (k, r, "shifted", before)
+
+
+def _prefix_sweep(cuda_lib, wl, prefixes, keys):
+    """Rows of each prefix batch equal the same rows of the full batch, and the
+    prefix's dw is the same across launch geometries and repeats."""
+    full = run(cuda_lib, wl)
+    for b in prefixes:
+        part = run(cuda_lib, sub(wl, 0, b)) if b < wl.rows else full
+        for k in keys:
+            assert torch.equal(bits(part[k]), bits(full[k][:b])), (k, b)
+        ref_dw = bits(part["dw"]).clone()
+        for geo in ((1, 1, 8), (7, 2, 64), (148, 0, 0), (0, 8, 256), (0, 0, 0)):
+            cuda_lib.rn_test_set_geometry(*geo)
+            again = run(cuda_lib, sub(wl, 0, b)) if b < wl.rows else run(cuda_lib, wl)
+            assert torch.equal(bits(again["dw"]), ref_dw), (b, geo)
+            for k in keys:
+                assert torch.equal(bits(again[k]), bits(full[k][:b])), (k, b, geo)
+        cuda_lib.rn_test_set_geometry(0, 0, 0)
+    return full
+
+
+@pytest.mark.slow
+def test_wide_8192_batch_size_sweep_bitwise(cuda_lib):
+    # the 32768 x 8192 bf16 workload: every row of the prefixes 1, 7, 128, 4096
+    # equals the same row of the full batch (512-thread teams, the shared-memory
+    # warp tree), dw is the same across geometries, and sampled rows alone and
+    # at shifted offsets keep their bits
+    wl = workloads.cfg_wide_8192().to(DEV)
+    full = _prefix_sweep(cuda_lib, wl, workloads.SWEEP_8192, ("y", "rstd", "dx"))
+    pick = np.random.default_rng(2).choice(wl.rows, 14, replace=False).tolist() + [0, wl.rows - 1]
+    _alone_and_shifted(cuda_lib, wl, full, pick, seed=3, keys=("y", "rstd", "dx"))
+
+
+@pytest.mark.parametrize("op,rows,width,dtype,act,off", [
+    ("general", 3000, 5120, "bf16", "none", 1.0),      # 128 x 5 teams
+    ("general", 1200, 5120, "bf16", "silu", 0.0),
+    ("gated", 600, 16384, "f32", None, None),          # 1024 x 4 teams
+    ("norm", 600, 16384, "bf16", None, None),          # 512 x 4 teams
+    ("gated", 2000, 4104, "bf16", None, None),         # 512 x 2, vector slots left idle
+])
+def test_multiwarp_batch_size_sweep_bitwise(cuda_lib, op, rows, width, dtype, act, off):
+    wl = workloads.make(op, rows, width, dtype, seed=width + rows, act=act,
+                        weight_offset=off, w_mean=1.0 if off in (None, 0.0) else 0.0).to(DEV)
+    keys = ("y", "rstd", "dx") + (("dz",) if wl.gated else ())
+    full = _prefix_sweep(cuda_lib, wl, (1, 7, 128, rows // 2 + 3, rows), keys)
+    pick = np.random.default_rng(rows).choice(rows, 6, replace=False).tolist() + [rows - 1]
+    _alone_and_shifted(cuda_lib, wl, full, pick, seed=width, keys=keys)

@@ -79,3 +79,63 @@ def test_unsupported_shards_are_refused_on_every_rank(tmp_path, rows):
     for r in range(2):
         assert (tmp_path / f"r{r}.err").exists(), r
         assert not (tmp_path / f"r{r}.npy").exists()
+
+
+# --- any split on 256-row chunk boundaries ------------------------------------
+def _contribs(rows, seed=1):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((rows, WIDTH)) * 10).astype(np.float32)
+
+
+def _chunk_worker(rank, world, port, split, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from rollout_parity_b200 import parallel
+        c = _contribs(sum(split))
+        s0 = sum(split[:rank])
+        mine = c[s0:s0 + split[rank]]
+        local = (torch.from_numpy(fold_model.chunk_partials(mine)) if split[rank]
+                 else torch.zeros(0, WIDTH))
+        try:
+            got = parallel.chunk_split_dw(local, split[rank], fold=_tree_fold)
+            np.save(os.path.join(out_dir, f"r{rank}.npy"), got.numpy())
+        except ValueError as e:
+            open(os.path.join(out_dir, f"r{rank}.err"), "w").write(str(e))
+    finally:
+        dist.destroy_process_group()
+
+
+def _run_chunks(tmp_path, split):
+    mp.spawn(_chunk_worker, args=(len(split), _free_port(), split, str(tmp_path)),
+             nprocs=len(split), join=True)
+
+
+@pytest.mark.parametrize("split", [[256, 256], [512, 300], [256, 1000], [0, 777], [768, 0],
+                                   [256, 512, 33], [1024, 256, 256]],
+                         ids=lambda s: "-".join(map(str, s)))
+def test_chunk_split_equals_whole_batch_tree(tmp_path, split):
+    _run_chunks(tmp_path, split)
+    whole = fold_model.dw_tree(_contribs(sum(split)))
+    for r in range(len(split)):
+        got = np.load(tmp_path / f"r{r}.npy")
+        assert np.array_equal(got.view(np.uint32), whole.view(np.uint32)), (split, r)
+
+
+@pytest.mark.parametrize("split", [[300, 256], [255, 1], [256, 100, 256]],
+                         ids=lambda s: "-".join(map(str, s)))
+def test_chunk_split_off_boundaries_is_refused_on_every_rank(tmp_path, split):
+    _run_chunks(tmp_path, split)
+    for r in range(len(split)):
+        assert (tmp_path / f"r{r}.err").exists(), r
+        assert not (tmp_path / f"r{r}.npy").exists()
+
+
+def test_chunk_model_is_the_leaf_tree_from_its_third_level():
+    # the model's own claim, checked on ragged row counts: the tree over chunk
+    # partials is the declared tree over leaves
+    for rows in (1, 31, 256, 257, 1000, 2048, 4100):
+        c = _contribs(rows, seed=rows)
+        got = fold_model.pairwise_tree(list(fold_model.chunk_partials(c)), fold_model._f32_add)
+        assert np.array_equal(np.asarray(got).view(np.uint32), fold_model.dw_tree(c).view(np.uint32))

@@ -64,3 +64,32 @@ def test_static_scratch_backward_rejects_shapes_beyond_its_scratch():
     st = lib.gated_norm_bwd_static_ws(rows, 128, 1e-6, int(DType.BF16), fake, fake, fake, fake,
                                       None, fake, fake, fake, None)
     assert st == Status.E_WORKSPACE
+
+
+@pytest.mark.gpu
+def test_static_scratch_backward_writes_only_its_outputs(cuda_lib):
+    # dx, dz and dw sit between 256-byte guards of a sentinel pattern; a ragged
+    # width (1032) and row count (3001) must leave the guards unchanged
+    lib = cuda_lib.load()
+    dev = torch.device("cuda:0")
+    rows, width, guard = 3001, 1032, 256
+    wl = workloads.make("gated", rows, width, "bf16", seed=9).to(dev)
+    bufs = []
+
+    def guarded(n_elems, dtype):
+        nbytes = n_elems * torch.empty(0, dtype=dtype).element_size()
+        raw = torch.full((2 * guard + nbytes,), 0x5A, dtype=torch.uint8, device=dev)
+        bufs.append((raw, nbytes))
+        return raw[guard:guard + nbytes].view(dtype)
+
+    dx = guarded(rows * width, torch.bfloat16).view(rows, width)
+    dz = guarded(rows * width, torch.bfloat16).view(rows, width)
+    dw = guarded(width, torch.float32)
+    _, rstd = cuda_lib.gated_norm_fwd(wl.x, wl.z, wl.w, wl.eps)
+    assert _static_bwd(lib, wl, rstd, dx, dz, dw) == Status.OK
+    torch.cuda.synchronize()
+    for raw, nbytes in bufs:
+        assert bool((raw[:guard] == 0x5A).all()) and bool((raw[guard + nbytes:] == 0x5A).all())
+    ref_dx, ref_dz, ref_dw = cuda_lib.gated_norm_bwd(wl.x, wl.z, wl.w, wl.dy, rstd, wl.eps)
+    for got, want in ((dx, ref_dx), (dz, ref_dz), (dw, ref_dw)):
+        assert torch.equal(_bits(got), _bits(want))
