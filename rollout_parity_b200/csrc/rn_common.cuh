@@ -89,6 +89,17 @@ __host__ __device__ constexpr int bwd_stages_of(int T, int K) {
   return T <= 16 ? 3 : (T <= 128 ? 4 : (T <= 512 ? (K <= 2 ? 3 : 2) : 1));
 }
 
+// k_bwd shapes that run the lean row (bwd_row_lean): wide teams holding at
+// least 16 elements a thread whose pass-1 state (xh, g*dy and, with a gate,
+// the sigmoid) does not fit the register file of their launch shape -- every
+// gated one, and the ungated 512- and 1024-thread teams with K >= 3.  The
+// others keep the state in registers (bwd_row), which measured faster where it
+// fits (16384 x 5120 and 32768 x 8192 bf16 without a gate); with a gate the
+// lean row measured 17-34% faster (widths 512, 2048, 5120, 8192 in bf16).
+__host__ __device__ constexpr bool lean_bwd(int T, int K, int VE, bool gated) {
+  return T >= 32 && K * VE >= 16 && (gated || (T >= 512 && K >= 3));
+}
+
 // Where a thread's gain (w, or w + offset) comes from: shared memory
 // (thread-major) for sub-warp teams, registers when K*VE <= 16, else global
 // memory through L1.

@@ -637,6 +637,121 @@ __device__ __forceinline__ void bwd_row(const BwdArgs& a, const G& gain, const u
   }
 }
 
+// The same row as bwd_row, for wide rows in k_bwd, holding fewer registers:
+// the staged row stays in shared memory (its slot is not reused before the
+// next row starts), pass 1 keeps only the sigmoid of each element, and pass 2
+// reads x, dy (and z) again and recomputes xh and g*dy -- the same
+// operations on the same values, so the same bits as bwd_row.  Pass 2 adds
+// the row's dw contributions dy*xh*a(z) to acc when add_dw.  `stg(ten, k)`
+// is this thread's staged vector k of tensor ten (0 x, 1 dy, 2 z).
+template <int DT, int T, int K, int ACT, bool EXACT, bool RESID, typename G, typename Stg>
+__device__ __forceinline__ void bwd_row_lean(const BwdArgs& a, const G& gain, Stg stg,
+                                             float rs_staged, bool have_rstd, int64_t row,
+                                             bool act, bool add_dw, int t, float* red,
+                                             int& phase, int team, int NT, unsigned mask,
+                                             float2 (&acc)[K][Fmt<DT>::VE / 2]) {
+  using F = Fmt<DT>;
+  constexpr bool GATED = ACT != kActNone;
+  constexpr int VE = F::VE;
+  const int nv = a.nv;
+  float rs = rs_staged;
+  if (!have_rstd) {   // uniform branch
+    uint4 xr[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) xr[k] = *stg(0, k);
+    float ss[1] = {thread_sumsq<DT, T, K, EXACT>(xr, nv, t)};
+    team_sum<T, 1>(ss, red, phase, team, NT, mask);
+    rs = rsqrtf(__fadd_rn(mean_of(ss[0], a.H, a.inv_h, a.h_pow2), a.eps));
+  }
+  const float2 rs2 = bc2(rs);
+  float2 sg[K][GATED ? VE / 2 : 1];
+  // g*dy and xh of vector k (recomputed in both passes from the staged row)
+  auto terms = [&](int k, float2 (&gd)[VE / 2], float2 (&xh)[VE / 2], float2 (&df)[VE / 2],
+                   float2 (&zf)[VE / 2], float2 (&gk)[VE / 2], bool first) {
+    float2 xf[VE / 2];
+    F::unpack2(*stg(0, k), xf);
+    F::unpack2(*stg(1, k), df);
+    if constexpr (GATED) F::unpack2(*stg(2, k), zf);
+    gain.get2(k, gk);
+#pragma unroll
+    for (int q = 0; q < VE / 2; ++q) {
+      xh[q] = mul2(xf[q], rs2);
+      float2 g;
+      if constexpr (GATED) {
+        if (first) sg[k][q] = sigmoid2(zf[q]);
+        g = mul2(gk[q], gate2<ACT>(zf[q], sg[k][q]));   // u * a(z)
+      } else {
+        g = gk[q];                                      // u
+      }
+      gd[q] = mul2(g, df[q]);
+    }
+  };
+  // pass 1: per-vector dot chains (two vectors per pair instruction, each lane
+  // its own ascending chain, as vector_dots), then the pairwise tree
+  float dp[K];
+#pragma unroll
+  for (int k = 0; k < K; k += 2) {
+    float2 gd0[VE / 2], xh0[VE / 2], df0[VE / 2], zf0[VE / 2], gk0[VE / 2];
+    terms(k, gd0, xh0, df0, zf0, gk0, true);
+    if (k + 1 < K) {
+      float2 gd1[VE / 2], xh1[VE / 2], df1[VE / 2], zf1[VE / 2], gk1[VE / 2];
+      terms(k + 1, gd1, xh1, df1, zf1, gk1, true);
+      float2 c = bc2(-0.0f);
+#pragma unroll
+      for (int q = 0; q < VE / 2; ++q) {
+        c = fma2(make_float2(gd0[q].x, gd1[q].x), make_float2(xh0[q].x, xh1[q].x), c);
+        c = fma2(make_float2(gd0[q].y, gd1[q].y), make_float2(xh0[q].y, xh1[q].y), c);
+      }
+      dp[k] = (EXACT || k * T + t < nv) ? c.x : -0.0f;
+      dp[k + 1] = (EXACT || (k + 1) * T + t < nv) ? c.y : -0.0f;
+    } else {
+      float c = -0.0f;
+#pragma unroll
+      for (int q = 0; q < VE / 2; ++q) {
+        c = __fmaf_rn(gd0[q].x, xh0[q].x, c);
+        c = __fmaf_rn(gd0[q].y, xh0[q].y, c);
+      }
+      dp[k] = (EXACT || k * T + t < nv) ? c : -0.0f;
+    }
+  }
+  float dot[1] = {pairwise_tree<K>(dp)};
+  team_sum<T, 1>(dot, red, phase, team, NT, mask);
+  const float2 m2 = bc2(mean_of(dot[0], a.H, a.inv_h, a.h_pow2));
+  // pass 2: dx, dz stores and the dw contributions
+  const int64_t off = row * nv + t;
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    if (act && (EXACT || k * T + t < nv)) {
+      float2 gd[VE / 2], xh[VE / 2], df[VE / 2], zf[VE / 2], gk[VE / 2];
+      terms(k, gd, xh, df, zf, gk, false);
+      float2 dxv[VE / 2], dzv[VE / 2];
+#pragma unroll
+      for (int q = 0; q < VE / 2; ++q) {
+        dxv[q] = mul2(rs2, fma2(neg2(xh[q]), m2, gd[q]));        // rstd*(g*dy - xh*m)
+        const float2 qv = mul2(df[q], xh[q]);                    // dy * xh
+        float2 d;
+        if constexpr (GATED) {
+          const float2 sv = sg[k][q];
+          const float2 c = gate_slope_over_s2<ACT>(zf[q], sv);
+          dzv[q] = mul2(mul2(mul2(qv, gk[q]), sv), c);           // dy*xh*u*a'(z)
+          d = mul2(qv, gate2<ACT>(zf[q], sv));                   // dy*xh*a(z)
+        } else {
+          d = qv;
+        }
+        if (add_dw) acc[k][q] = add2(acc[k][q], d);
+      }
+      if constexpr (RESID) {   // dx = dnorm + dres, rounded once
+        float2 rf[VE / 2];
+        F::unpack2(__ldcs(a.dres + off + k * T), rf);
+#pragma unroll
+        for (int q = 0; q < VE / 2; ++q) dxv[q] = add2(dxv[q], rf[q]);
+      }
+      st_stream(a.dx + off + k * T, F::pack2v(dxv));
+      if constexpr (GATED) st_stream(a.dz + off + k * T, F::pack2v(dzv));
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Backward: one team per 32-row leaf, rows in ascending order.  x, dy (z) and
 // rstd are staged S-1 rows ahead; pass 1 keeps xh, g*dy and s in registers for
@@ -719,23 +834,32 @@ k_bwd(const BwdArgs a) {
         issue(r0 + ahead, ahead < kLeafRows && r0 + ahead < a.rows, sa);
       }
       cp_async_wait<S - 1>();
-      uint4 xr[K], dr[K], zr[K];
-#pragma unroll
-      for (int k = 0; k < K; ++k) {
-        xr[k] = *slot(sl, 0, k);
-        dr[k] = *slot(sl, 1, k);
-        if constexpr (GATED) zr[k] = *slot(sl, 2, k);
-      }
-      float2 d[K][VE / 2];
-      bwd_row<DT, T, K, ACT, EXACT, RESID, false>(a, gain, xr, dr, zr,
-                                                 have_rstd ? rsm[sl * bd + tid] : 0.0f,
-                                   have_rstd, row, act, t, red, phase, team, NT, mask, d);
-      if (act && (a.mask == nullptr || __ldg(a.mask + row) != 0)) {   // masked rows add nothing
+      const bool add_dw = act && (a.mask == nullptr || __ldg(a.mask + row) != 0);
+      if constexpr (lean_bwd(T, K, VE, GATED)) {
+        const int slc = sl;
+        bwd_row_lean<DT, T, K, ACT, EXACT, RESID>(
+            a, gain, [&](int ten, int k) -> const uint4* { return slot(slc, ten, k); },
+            have_rstd ? rsm[sl * bd + tid] : 0.0f, have_rstd, row, act, add_dw, t, red, phase,
+            team, NT, mask, acc);
+      } else {
+        uint4 xr[K], dr[K], zr[K];
 #pragma unroll
         for (int k = 0; k < K; ++k) {
-          if (EXACT || k * T + t < nv) {
+          xr[k] = *slot(sl, 0, k);
+          dr[k] = *slot(sl, 1, k);
+          if constexpr (GATED) zr[k] = *slot(sl, 2, k);
+        }
+        float2 d[K][VE / 2];
+        bwd_row<DT, T, K, ACT, EXACT, RESID, false>(a, gain, xr, dr, zr,
+                                                   have_rstd ? rsm[sl * bd + tid] : 0.0f,
+                                     have_rstd, row, act, t, red, phase, team, NT, mask, d);
+        if (add_dw) {   // masked rows add nothing
 #pragma unroll
-            for (int q = 0; q < VE / 2; ++q) acc[k][q] = add2(acc[k][q], d[k][q]);
+          for (int k = 0; k < K; ++k) {
+            if (EXACT || k * T + t < nv) {
+#pragma unroll
+              for (int q = 0; q < VE / 2; ++q) acc[k][q] = add2(acc[k][q], d[k][q]);
+            }
           }
         }
       }
