@@ -834,8 +834,8 @@ k_bwd(const BwdArgs a) {
         issue(r0 + ahead, ahead < kLeafRows && r0 + ahead < a.rows, sa);
       }
       cp_async_wait<S - 1>();
-      const bool add_dw = act && (a.mask == nullptr || __ldg(a.mask + row) != 0);
       if constexpr (lean_bwd(T, K, VE, GATED)) {
+        const bool add_dw = act && (a.mask == nullptr || __ldg(a.mask + row) != 0);
         const int slc = sl;
         bwd_row_lean<DT, T, K, ACT, EXACT, RESID>(
             a, gain, [&](int ten, int k) -> const uint4* { return slot(slc, ten, k); },
@@ -853,7 +853,7 @@ k_bwd(const BwdArgs a) {
         bwd_row<DT, T, K, ACT, EXACT, RESID, false>(a, gain, xr, dr, zr,
                                                    have_rstd ? rsm[sl * bd + tid] : 0.0f,
                                      have_rstd, row, act, t, red, phase, team, NT, mask, d);
-        if (add_dw) {   // masked rows add nothing
+        if (act && (a.mask == nullptr || __ldg(a.mask + row) != 0)) {   // masked rows add nothing
 #pragma unroll
           for (int k = 0; k < K; ++k) {
             if (EXACT || k * T + t < nv) {
