@@ -212,6 +212,13 @@ def cfg_qk_norm(width: int, rows: int, seed: int = 0) -> Workload:
                 weight_offset=1.0, name=f"qk_norm_{rows}x{width}_bf16")
 
 
+def cfg_gated_wide(width: int, seed: int = 0) -> Workload:
+    """The gated operator (silu, offset 0) on 16384 rows at a model width, bf16,
+    w ~ N(1, 0.1): the pages' rstd matrix widths 2048 and 5120 with the gate."""
+    return make("general", 16384, width, "bf16", seed=seed, w_mean=1.0, w_std=0.1, act="silu",
+                weight_offset=0.0, name=f"silu_16384x{width}_bf16")
+
+
 VARIANTS = {
     "sigmoid_262144x128_bf16_outliers": cfg_sigmoid_heads,
     "silu_262144x128_f16_outliers": cfg_f16_heads,
@@ -219,6 +226,8 @@ VARIANTS = {
     "sigmoid_off1_16384x2048_f32": cfg_sigmoid_f32_2048,
     "qk_norm_131072x256_bf16": lambda seed=0: cfg_qk_norm(256, 131072, seed),
     "qk_norm_65536x512_bf16": lambda seed=0: cfg_qk_norm(512, 65536, seed),
+    "silu_16384x2048_bf16": lambda seed=0: cfg_gated_wide(2048, seed),
+    "silu_16384x5120_bf16": lambda seed=0: cfg_gated_wide(5120, seed),
 }
 ALL = {**CONFIGS, **VARIANTS}
 
