@@ -583,7 +583,7 @@ size_t bwd_smem_bytes(const Sched& s, int lpc, int width, bool gated, rn_dtype d
   const size_t bd = size_t(lpc) * s.T;
   const size_t W = s.T > 32 ? s.T / 32 : 1;
   const size_t red = s.T > 32 ? 2 * size_t(lpc) * W * sizeof(float) : 0;
-  const size_t gain = s.T <= 16 ? size_t(s.K) * s.T * VE * sizeof(float) : 0;
+  const size_t gain = gain_src_of(s.T, s.K, int(VE)) == kGainSmem ? size_t(s.K) * s.T * VE * sizeof(float) : 0;
   const size_t stages = size_t(bwd_stages_of(s.T, s.K)) * (gated ? 3 : 2) * s.K * bd * 16;
   const size_t leaves = lpc > 1 ? size_t(lpc) * width * sizeof(float) : 0;
   return red + gain + stages + leaves + size_t(bwd_stages_of(s.T, s.K)) * bd * sizeof(float);
@@ -607,7 +607,7 @@ size_t fwd_smem_bytes(const Sched& s, bool gated, bool resid, rn_dtype dt) {
   const size_t B = fwd_block_of(s.T, s.K), NT = B / s.T;
   const size_t W = s.T > 32 ? s.T / 32 : 1;
   const size_t red = s.T > 32 ? 2 * NT * W * sizeof(float) : 0;
-  const size_t gain = s.T <= 16 ? size_t(s.K) * s.T * VE * sizeof(float) : 0;
+  const size_t gain = gain_src_of(s.T, s.K, int(VE)) == kGainSmem ? size_t(s.K) * s.T * VE * sizeof(float) : 0;
   return red + gain + size_t(fwd_stages_of(s.T)) * (1 + gated + resid) * s.K * B * 16;
 }
 

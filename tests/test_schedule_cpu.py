@@ -114,18 +114,24 @@ def bwd_stages(t, k):
     return 3 if t <= 16 else (4 if t <= 128 else ((3 if k <= 2 else 2) if t <= 512 else 1))
 
 
+def gain_in_smem(t, k, ve):
+    """The gain is staged in shared memory for sub-warp teams and for threads
+    of more than 16 elements in rows of at most 8192 elements."""
+    return t <= 16 or (k * ve > 16 and t * k * ve <= 8192)
+
+
 def fwd_smem(t, k, ve, tensors):
     b = fwd_block(t, k)
     nt, w = b // t, (t // 32 if t > 32 else 1)
     red = 2 * nt * w * 4 if t > 32 else 0
-    gain = k * t * ve * 4 if t <= 16 else 0
+    gain = k * t * ve * 4 if gain_in_smem(t, k, ve) else 0
     return red + gain + fwd_stages(t) * tensors * k * b * 16
 
 
 def bwd_smem(t, k, ve, lpc, width, tensors):
     bd, w = lpc * t, (t // 32 if t > 32 else 1)
     red = 2 * lpc * w * 4 if t > 32 else 0
-    gain = k * t * ve * 4 if t <= 16 else 0
+    gain = k * t * ve * 4 if gain_in_smem(t, k, ve) else 0
     stages = bwd_stages(t, k) * tensors * k * bd * 16
     leaves = lpc * width * 4 if lpc > 1 else 0
     return red + gain + stages + leaves + bwd_stages(t, k) * bd * 4
