@@ -84,9 +84,15 @@ __host__ __device__ constexpr int bwd_min_blocks_of(int T, int K) {
 }
 // Backward staging depth (rows in flight per team): deeper for the wide teams,
 // whose few leaves (one per 32 rows) must each keep more bytes in flight,
-// within 227 KB of shared memory per CTA at the widest rows.
-__host__ __device__ constexpr int bwd_stages_of(int T, int K) {
-  return T <= 16 ? 3 : (T <= 128 ? 4 : (T <= 512 ? (K <= 2 ? 3 : 2) : 1));
+// within 227 KB of shared memory per CTA at the widest rows.  With a gate a
+// third tensor is staged, and where four stages held the CTAs to one per SM
+// fewer stages measured faster: two for 32-thread teams (65536 x 512 bf16
+// silu: 80.3 -> 72.2 us) and three for 128-thread teams with K >= 3 (16384 x
+// 5120: 252.4 -> 195.1 us); at 128 x 2 (width 2048) four stages stay faster.
+__host__ __device__ constexpr int bwd_stages_of(int T, int K, bool gated) {
+  return T <= 16 ? 3
+                 : (T <= 128 ? (gated && T == 32 ? 2 : (gated && T == 128 && K >= 3 ? 3 : 4))
+                             : (T <= 512 ? (K <= 2 ? 3 : 2) : 1));
 }
 
 // k_bwd shapes that run the lean row (bwd_row_lean): wide teams holding at

@@ -110,8 +110,12 @@ def fwd_stages(t):
     return 3 if t <= 32 else (2 if t <= 512 else 1)
 
 
-def bwd_stages(t, k):
-    return 3 if t <= 16 else (4 if t <= 128 else ((3 if k <= 2 else 2) if t <= 512 else 1))
+def bwd_stages(t, k, gated=True):
+    if t <= 16:
+        return 3
+    if t <= 128:
+        return 2 if gated and t == 32 else (3 if gated and t == 128 and k >= 3 else 4)
+    return (3 if k <= 2 else 2) if t <= 512 else 1
 
 
 def gain_in_smem(t, k, ve):
@@ -132,9 +136,10 @@ def bwd_smem(t, k, ve, lpc, width, tensors):
     bd, w = lpc * t, (t // 32 if t > 32 else 1)
     red = 2 * lpc * w * 4 if t > 32 else 0
     gain = k * t * ve * 4 if gain_in_smem(t, k, ve) else 0
-    stages = bwd_stages(t, k) * tensors * k * bd * 16
+    gated = tensors == 3
+    stages = bwd_stages(t, k, gated) * tensors * k * bd * 16
     leaves = lpc * width * 4 if lpc > 1 else 0
-    return red + gain + stages + leaves + bwd_stages(t, k) * bd * 4
+    return red + gain + stages + leaves + bwd_stages(t, k, gated) * bd * 4
 
 
 def bwd_lpc(t, k, ve, width):
@@ -159,6 +164,7 @@ def test_every_shape_fits_shared_memory(ve):
         if stripe:                            # gain, stages, rstd stages, transpose buffer
             s = kb * tb * ve * 4 + 3 * 3 * kb * 32 * 16 + 3 * 32 * 4 + (32 // tb) * (width + 4) * 4
         else:                                 # dh is read into registers, not staged
-            s = bwd_smem(tb, kb, ve, bwd_lpc(tb, kb, ve, width), width, 3)
+            lpc = bwd_lpc(tb, kb, ve, width)
+            s = max(bwd_smem(tb, kb, ve, lpc, width, 3), bwd_smem(tb, kb, ve, lpc, width, 2))
         worst = max(worst, s)
     assert worst <= SMEM_LIMIT, worst
