@@ -584,16 +584,16 @@ size_t bwd_smem_bytes(const Sched& s, int lpc, int width, bool gated, rn_dtype d
   const size_t W = s.T > 32 ? s.T / 32 : 1;
   const size_t red = s.T > 32 ? 2 * size_t(lpc) * W * sizeof(float) : 0;
   const size_t gain = gain_src_of(s.T, s.K, int(VE)) == kGainSmem ? size_t(s.K) * s.T * VE * sizeof(float) : 0;
-  const size_t stages = size_t(bwd_stages_of(s.T, s.K)) * (gated ? 3 : 2) * s.K * bd * 16;
+  const size_t stages = size_t(bwd_stages_of(s.T, s.K, gated)) * (gated ? 3 : 2) * s.K * bd * 16;
   const size_t leaves = lpc > 1 ? size_t(lpc) * width * sizeof(float) : 0;
-  return red + gain + stages + leaves + size_t(bwd_stages_of(s.T, s.K)) * bd * sizeof(float);
+  return red + gain + stages + leaves + size_t(bwd_stages_of(s.T, s.K, gated)) * bd * sizeof(float);
 }
 
 // Dynamic shared memory of k_bwd_stripe: gain, staged rows, staged rstd, the
 // transpose buffer (the kernel's layout).
 size_t bwd_stripe_smem_bytes(const Sched& s, int width, bool gated, rn_dtype dt) {
   const size_t VE = size_t(vec_elems(dt));
-  const size_t S = size_t(bwd_stages_of(s.T, s.K));
+  const size_t S = size_t(bwd_stages_of(s.T, s.K, gated));
   const size_t gain = size_t(s.K) * s.T * VE * sizeof(float);
   const size_t stages = S * (gated ? 3 : 2) * s.K * 32 * 16;
   const size_t rstd = S * 32 * sizeof(float);

@@ -573,9 +573,9 @@ __device__ __forceinline__ void bwd_row(const BwdArgs& a, const G& gain, const u
     team_sum<T, 1>(ss, red, phase, team, NT, mask);
     rs = rsqrtf(__fadd_rn(mean_of(ss[0], a.H, a.inv_h, a.h_pow2), a.eps));
   }
-  // pass 1: keep xh, g*dy and s for pass 2 (element pairs)
+  // pass 1: keep xh, g*dy, a(z) and u*a'(z) for pass 2 (element pairs)
   const float2 rs2 = bc2(rs);
-  float2 xh[K][VE / 2], gd[K][VE / 2], sg[K][GATED ? VE / 2 : 1];
+  float2 xh[K][VE / 2], gd[K][VE / 2], ga[K][GATED ? VE / 2 : 1], uap[K][GATED ? VE / 2 : 1];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     float2 xf[VE / 2], df[VE / 2], zf[VE / 2], gk[VE / 2];
@@ -588,10 +588,12 @@ __device__ __forceinline__ void bwd_row(const BwdArgs& a, const G& gain, const u
       xh[k][q] = mul2(xf[q], rs2);
       float2 g;
       if constexpr (GATED) {
-        sg[k][q] = sigmoid2(zf[q]);
-        g = mul2(gk[q], gate2<ACT>(zf[q], sg[k][q]));   // u * a(z)
+        const float2 sv = sigmoid2(zf[q]);
+        ga[k][q] = gate2<ACT>(zf[q], sv);                            // a(z)
+        uap[k][q] = mul2(gk[q], mul2(sv, gate_slope_over_s2<ACT>(zf[q], sv)));   // u * a'(z)
+        g = mul2(gk[q], ga[k][q]);                                   // u * a(z)
       } else {
-        g = gk[q];                                      // u
+        g = gk[q];                                                   // u
       }
       gd[k][q] = mul2(g, df[q]);
     }
@@ -606,21 +608,15 @@ __device__ __forceinline__ void bwd_row(const BwdArgs& a, const G& gain, const u
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     if (act && (EXACT || k * T + t < nv)) {
-      float2 df[VE / 2], zf[VE / 2], dxv[VE / 2], dzv[VE / 2], gk[VE / 2];
+      float2 df[VE / 2], dxv[VE / 2], dzv[VE / 2];
       F::unpack2(dr[k], df);
-      if constexpr (GATED) {
-        F::unpack2(zr[k], zf);
-        gain.get2(k, gk);
-      }
 #pragma unroll
       for (int q = 0; q < VE / 2; ++q) {
         dxv[q] = mul2(rs2, fma2(neg2(xh[k][q]), m2, gd[k][q]));   // rstd*(g*dy - xh*m)
         const float2 qv = mul2(df[q], xh[k][q]);                  // dy * xh
         if constexpr (GATED) {
-          const float2 sv = sg[k][q];
-          const float2 c = gate_slope_over_s2<ACT>(zf[q], sv);
-          dzv[q] = mul2(mul2(mul2(qv, gk[q]), sv), c);            // dy*xh*u*a'(z)
-          d[k][q] = mul2(qv, gate2<ACT>(zf[q], sv));              // dy*xh*a(z)
+          dzv[q] = mul2(qv, uap[k][q]);                           // dy*xh*(u*a'(z))
+          d[k][q] = mul2(qv, ga[k][q]);                           // dy*xh*a(z)
         } else {
           d[k][q] = qv;
         }
@@ -732,8 +728,8 @@ __device__ __forceinline__ void bwd_row_lean(const BwdArgs& a, const G& gain, St
         float2 d;
         if constexpr (GATED) {
           const float2 sv = sg[k][q];
-          const float2 c = gate_slope_over_s2<ACT>(zf[q], sv);
-          dzv[q] = mul2(mul2(mul2(qv, gk[q]), sv), c);           // dy*xh*u*a'(z)
+          const float2 uap = mul2(gk[q], mul2(sv, gate_slope_over_s2<ACT>(zf[q], sv)));
+          dzv[q] = mul2(qv, uap);                                // dy*xh*(u*a'(z))
           d = mul2(qv, gate2<ACT>(zf[q], sv));                   // dy*xh*a(z)
         } else {
           d = qv;
@@ -766,7 +762,7 @@ k_bwd(const BwdArgs a) {
   using F = Fmt<DT>;
   constexpr bool GATED = ACT != kActNone;
   constexpr int VE = F::VE;
-  constexpr int S = bwd_stages_of(T, K);
+  constexpr int S = bwd_stages_of(T, K, GATED);
   constexpr int NTEN = GATED ? 3 : 2;   // staged tensors: x, dy (, z)
   constexpr int W = T > 32 ? T / 32 : 1;
   constexpr int GS = gain_src_of(T, K, VE);
@@ -893,7 +889,7 @@ k_bwd_stripe(const BwdArgs a, int lpc) {
   using F = Fmt<DT>;
   constexpr bool GATED = ACT != kActNone;
   constexpr int VE = F::VE;
-  constexpr int S = bwd_stages_of(T, K);
+  constexpr int S = bwd_stages_of(T, K, GATED);
   constexpr int NTEN = GATED ? 3 : 2;     // staged tensors: x, dy (, z)
   constexpr int GS = gain_src_of(T, K, VE);
   constexpr int RPS = 32 / T;             // rows per step
