@@ -511,7 +511,25 @@ k_fwd(const FwdArgs a) {
         if (act && (EXACT || k * T + t < nv)) st_stream(a.h + row * nv + t + k * T, xr[k]);
       }
     }
-    float ss[1] = {thread_sumsq<DT, T, K, EXACT>(xr, nv, t)};
+    // x unpacked once: for the sum of squares and the epilogue; the gate a(z)
+    // does not depend on rstd, so it is formed before the row reduction
+    float2 xf[K][VE / 2], az[K][GATED ? VE / 2 : 1];
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      F::unpack2(xr[k], xf[k]);
+      if constexpr (GATED) {
+        float2 zf[VE / 2];
+        F::unpack2(zr[k], zf);
+#pragma unroll
+        for (int q = 0; q < VE / 2; ++q) az[k][q] = gate2<ACT>(zf[q], sigmoid2(zf[q]));
+      }
+    }
+    float ss[1];
+    {
+      float p[K];
+      vector_dots<VE, T, K, EXACT>(xf, xf, nv, t, p);
+      ss[0] = pairwise_tree<K>(p);
+    }
     team_sum<T, 1>(ss, red, phase, team, NT, mask);
     const float r = rsqrtf(__fadd_rn(mean_of(ss[0], a.H, a.inv_h, a.h_pow2), a.eps));
     const int64_t off = row * nv + t;
@@ -519,20 +537,15 @@ k_fwd(const FwdArgs a) {
 #pragma unroll
     for (int k = 0; k < K; ++k) {
       if (act && (EXACT || k * T + t < nv)) {
-        float2 f[VE / 2], yv[VE / 2], gk[VE / 2];
-        F::unpack2(xr[k], f);
+        float2 yv[VE / 2], gk[VE / 2];
         gain.get2(k, gk);
         if constexpr (GATED) {
-          float2 zf[VE / 2];
-          F::unpack2(zr[k], zf);
 #pragma unroll
-          for (int q = 0; q < VE / 2; ++q) {
-            const float2 az = gate2<ACT>(zf[q], sigmoid2(zf[q]));
-            yv[q] = mul2(mul2(mul2(f[q], r2), gk[q]), az);   // x*rstd*u*a(z)
-          }
+          for (int q = 0; q < VE / 2; ++q)
+            yv[q] = mul2(mul2(mul2(xf[k][q], r2), gk[q]), az[k][q]);   // x*rstd*u*a(z)
         } else {
 #pragma unroll
-          for (int q = 0; q < VE / 2; ++q) yv[q] = mul2(mul2(f[q], r2), gk[q]);
+          for (int q = 0; q < VE / 2; ++q) yv[q] = mul2(mul2(xf[k][q], r2), gk[q]);
         }
         st_stream(a.y + off + k * T, F::pack2v(yv));
       }
