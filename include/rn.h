@@ -388,6 +388,15 @@ void rn_test_set_validate_only(int32_t on);
 rn_status rn_test_rcp_1to2(int64_t n, const float* d, float* out, int32_t steps,
                            rn_stream stream);
 
+/*
+ * Test entry point: out[i] = the gate's sigmoid 1 / (1 + e^{-z[i]}) as the
+ * row kernels evaluate it (n floats, device pointers; e^{-|z|} from CUDA's
+ * expf, the reciprocal of rn_test_rcp_1to2 with one step); RN_E_ARG for n < 0
+ * or a NULL pointer with n > 0.  Lets a test bound it against the exact
+ * function, subnormal tail included.
+ */
+rn_status rn_test_sigmoid(int64_t n, const float* z, float* out, rn_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

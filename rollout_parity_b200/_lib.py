@@ -77,6 +77,7 @@ SIGNATURES = {
     "rn_test_set_geometry": (c_i32, [c_i32, c_i32, c_i32]),
     "rn_test_set_validate_only": (None, [c_i32]),
     "rn_test_rcp_1to2": (c_i32, [c_i64, c_vp, c_vp, c_i32, c_vp]),
+    "rn_test_sigmoid": (c_i32, [c_i64, c_vp, c_vp, c_vp]),
 }
 
 _lib = None

@@ -21,6 +21,7 @@
 
 #include "rn.h"
 #include "rn_common.cuh"
+#include "rn_gate.cuh"
 
 namespace {
 
@@ -167,6 +168,14 @@ k_fold1(const float* __restrict__ in, int64_t n, int H, float* __restrict__ out)
 __global__ void k_fill_neg_zero(float* __restrict__ out, int n) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) out[i] = -0.0f;
+}
+
+// Test kernel: the gate's sigmoid as the row kernels evaluate it, for checking
+// against the exact function.
+__global__ void k_test_sigmoid(const float* __restrict__ z, float* __restrict__ out, int64_t n) {
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n;
+       i += int64_t(gridDim.x) * blockDim.x)
+    out[i] = sigmoid2(make_float2(z[i], z[i])).x;
 }
 
 // Test kernel: the reciprocal used by the sigmoid, for checking against IEEE
@@ -794,6 +803,15 @@ rn_status rn_test_rcp_1to2(int64_t n, const float* d, float* out, int32_t steps,
   const int64_t blocks = (n + 255) / 256;
   k_test_rcp<<<int(blocks < 4096 ? blocks : 4096), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       d, out, n, steps);
+  return launch_status();
+}
+
+rn_status rn_test_sigmoid(int64_t n, const float* z, float* out, rn_stream stream) {
+  if (n < 0 || (n > 0 && (!z || !out))) return RN_E_ARG;
+  if (n == 0 || g_validate_only.load()) return RN_OK;
+  const int64_t blocks = (n + 255) / 256;
+  k_test_sigmoid<<<int(blocks < 4096 ? blocks : 4096), 256, 0,
+                   static_cast<cudaStream_t>(stream)>>>(z, out, n);
   return launch_status();
 }
 

@@ -47,6 +47,7 @@
 #include <cuda_fp16.h>
 
 #include "rn_common.cuh"
+#include "rn_gate.cuh"
 
 namespace rn_detail {
 
@@ -110,54 +111,6 @@ struct Fmt<RN_F32> {
 };
 
 __device__ __forceinline__ void st_stream(uint4* p, const uint4& v) { __stcs(p, v); }
-
-// ---------------------------------------------------------------------------
-// arithmetic of element pairs, written with explicit roundings
-// ---------------------------------------------------------------------------
-// Packed fp32 pairs (sm_100's two-lane fp32 instructions): each lane is the
-// IEEE fp32 operation rounded to nearest even, so a pair op gives the bits of
-// the two scalar ops it replaces and halves the instructions issued.  Adds
-// stay scalar __fadd_rn: a product followed by a packed add was observed to
-// come out fused (one rounding instead of two), which changed dw's bits, while
-// __fadd_rn is never merged into a multiply-add.
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-  return make_float2(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y));
-}
-__device__ __forceinline__ float2 bc2(float a) { return make_float2(a, a); }
-__device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
-
-// s(z) = 1 / (1 + exp(-z)) of both lanes   (PR #468 Summary, "Activation" bullet)
-// Evaluated as 1/(1+e) for z >= 0 and e/(1+e) for z < 0 with e = exp(-|z|) in
-// (0, 1]: the same function, but exp never overflows, so for z < -88.7 the
-// sigmoid is the fp32 subnormal e^z rather than 1/inf = 0 (outlier gates reach
-// there, and x*rstd*w*z*s(z) can still be a normal bf16 number).  1/(1+e) is
-// rcp.approx refined by kRcpSteps Newton steps (rcp_1to2's operations).
-__device__ __forceinline__ float2 sigmoid2(float2 z) {
-  const float2 e = make_float2(expf(-fabsf(z.x)), expf(-fabsf(z.y)));
-  const float2 d = add2(bc2(1.0f), e);
-  float2 y;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y.x) : "f"(d.x));
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y.y) : "f"(d.y));
-#pragma unroll
-  for (int i = 0; i < kRcpSteps; ++i) y = fma2(y, fma2(neg2(d), y, bc2(1.0f)), y);
-  const float2 er = mul2(e, y);
-  return make_float2(z.x >= 0.0f ? y.x : er.x, z.y >= 0.0f ? y.y : er.y);
-}
-
-// a(z) from z and s = s(z): silu(z) = z * s(z), or the sigmoid itself
-template <int ACT>
-__device__ __forceinline__ float2 gate2(float2 z, float2 s) {
-  return ACT == kActSilu ? mul2(z, s) : s;
-}
-// a'(z) / s(z): 1 + z * (1 - s) for silu, 1 - s for the sigmoid (1 + (-s)
-// is the IEEE difference 1 - s exactly)
-template <int ACT>
-__device__ __forceinline__ float2 gate_slope_over_s2(float2 z, float2 s) {
-  const float2 one_minus_s = add2(bc2(1.0f), neg2(s));
-  return ACT == kActSilu ? fma2(z, one_minus_s, bc2(1.0f)) : one_minus_s;
-}
 
 // u = w + offset, the offset added only when it is nonzero, so that with
 // offset 0 a -0.0 weight stays -0.0 (PR #468, "Changes to existing code, in
@@ -557,8 +510,9 @@ k_fwd(const FwdArgs a) {
 }
 
 // One row of the backward for this thread's K vectors: rstd (staged, or
-// recomputed exactly as the forward does), pass 1 (xh, g*dy, s and the
-// per-vector dot partials), the team's dot product, pass 2 (dx and dz
+// recomputed exactly as the forward does), pass 1 (xh and g*dy kept, the dz
+// stores and the dw contributions, which need no row statistic but rstd),
+// the per-vector dot partials and the team's dot product, pass 2 (the dx
 // stores).  d receives the row's dw contributions dy*xh*a(z) of this thread's
 // elements (meaningful only when act).  For T > 32 every team of the CTA must
 // call it in lockstep.
@@ -574,24 +528,20 @@ __device__ __forceinline__ void bwd_row(const BwdArgs& a, const G& gain, const u
   constexpr bool GATED = ACT != kActNone;
   constexpr int VE = F::VE;
   const int nv = a.nv;
-  uint4 rv[RESID ? K : 1];   // dres of this row, loaded early to hide its latency
-  if constexpr (RESID) {
-#pragma unroll
-    for (int k = 0; k < K; ++k)
-      if (act && (EXACT || k * T + t < nv)) rv[k] = __ldcs(a.dres + row * nv + t + k * T);
-  }
   float rs = rs_staged;
   if (!have_rstd) {   // uniform branch
     float ss[1] = {thread_sumsq<DT, T, K, EXACT, XJ>(xr, nv, t)};
     team_sum<T, 1>(ss, red, phase, team, NT, mask);
     rs = rsqrtf(__fadd_rn(mean_of(ss[0], a.H, a.inv_h, a.h_pow2), a.eps));
   }
-  // pass 1: keep xh, g*dy, a(z) and u*a'(z) for pass 2 (element pairs)
+  // pass 1: xh and g*dy kept for pass 2; dz stored and the dw contributions
+  // dy*xh*a(z) formed (neither depends on the row's dot product)
   const float2 rs2 = bc2(rs);
-  float2 xh[K][VE / 2], gd[K][VE / 2], ga[K][GATED ? VE / 2 : 1], uap[K][GATED ? VE / 2 : 1];
+  const int64_t off = row * nv + t;
+  float2 xh[K][VE / 2], gd[K][VE / 2];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
-    float2 xf[VE / 2], df[VE / 2], zf[VE / 2], gk[VE / 2];
+    float2 xf[VE / 2], df[VE / 2], zf[VE / 2], gk[VE / 2], dzv[VE / 2];
     F::unpack2(xr[k], xf);
     F::unpack2(dr[k], df);
     if constexpr (GATED) F::unpack2(zr[k], zf);
@@ -599,41 +549,42 @@ __device__ __forceinline__ void bwd_row(const BwdArgs& a, const G& gain, const u
 #pragma unroll
     for (int q = 0; q < VE / 2; ++q) {
       xh[k][q] = mul2(xf[q], rs2);
-      float2 g;
+      const float2 qv = mul2(df[q], xh[k][q]);                      // dy * xh
       if constexpr (GATED) {
         const float2 sv = sigmoid2(zf[q]);
-        ga[k][q] = gate2<ACT>(zf[q], sv);                            // a(z)
-        uap[k][q] = mul2(gk[q], mul2(sv, gate_slope_over_s2<ACT>(zf[q], sv)));   // u * a'(z)
-        g = mul2(gk[q], ga[k][q]);                                   // u * a(z)
+        const float2 ga = gate2<ACT>(zf[q], sv);                     // a(z)
+        const float2 uap = mul2(gk[q], mul2(sv, gate_slope_over_s2<ACT>(zf[q], sv)));   // u * a'(z)
+        gd[k][q] = mul2(mul2(gk[q], ga), df[q]);                     // u * a(z) * dy
+        dzv[q] = mul2(qv, uap);                                      // dy*xh*(u*a'(z))
+        d[k][q] = mul2(qv, ga);                                      // dy*xh*a(z)
       } else {
-        g = gk[q];                                                   // u
+        gd[k][q] = mul2(gk[q], df[q]);                               // u * dy
+        d[k][q] = qv;
       }
-      gd[k][q] = mul2(g, df[q]);
     }
+    if constexpr (GATED) {
+      if (act && (EXACT || k * T + t < nv)) st_stream(a.dz + off + k * T, F::pack2v(dzv));
+    }
+  }
+  uint4 rv[RESID ? K : 1];   // dres of this row, loaded before the reduction to hide its latency
+  if constexpr (RESID) {
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+      if (act && (EXACT || k * T + t < nv)) rv[k] = __ldcs(a.dres + off + k * T);
   }
   float dp[K];   // per-vector dot partials, joined by the pairwise tree
   vector_dots<VE, T, K, EXACT>(gd, xh, nv, t, dp);
   float dot[1] = {pairwise_tree<K>(dp)};
   team_sum<T, 1>(dot, red, phase, team, NT, mask);
   const float2 m2 = bc2(mean_of(dot[0], a.H, a.inv_h, a.h_pow2));
-  // pass 2: dx, dz and the dw contributions
-  const int64_t off = row * nv + t;
+  // pass 2: dx
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     if (act && (EXACT || k * T + t < nv)) {
-      float2 df[VE / 2], dxv[VE / 2], dzv[VE / 2];
-      F::unpack2(dr[k], df);
+      float2 dxv[VE / 2];
 #pragma unroll
-      for (int q = 0; q < VE / 2; ++q) {
+      for (int q = 0; q < VE / 2; ++q)
         dxv[q] = mul2(rs2, fma2(neg2(xh[k][q]), m2, gd[k][q]));   // rstd*(g*dy - xh*m)
-        const float2 qv = mul2(df[q], xh[k][q]);                  // dy * xh
-        if constexpr (GATED) {
-          dzv[q] = mul2(qv, uap[k][q]);                           // dy*xh*(u*a'(z))
-          d[k][q] = mul2(qv, ga[k][q]);                           // dy*xh*a(z)
-        } else {
-          d[k][q] = qv;
-        }
-      }
       if constexpr (RESID) {   // dx = dnorm + dres, rounded once
         float2 rf[VE / 2];
         F::unpack2(rv[k], rf);
@@ -641,18 +592,17 @@ __device__ __forceinline__ void bwd_row(const BwdArgs& a, const G& gain, const u
         for (int q = 0; q < VE / 2; ++q) dxv[q] = add2(dxv[q], rf[q]);
       }
       st_stream(a.dx + off + k * T, F::pack2v(dxv));
-      if constexpr (GATED) st_stream(a.dz + off + k * T, F::pack2v(dzv));
     }
   }
 }
 
 // The same row as bwd_row, for wide rows in k_bwd, holding fewer registers:
 // the staged row stays in shared memory (its slot is not reused before the
-// next row starts), pass 1 keeps only the sigmoid of each element, and pass 2
-// reads x, dy (and z) again and recomputes xh and g*dy -- the same
-// operations on the same values, so the same bits as bwd_row.  Pass 2 adds
-// the row's dw contributions dy*xh*a(z) to acc when add_dw.  `stg(ten, k)`
-// is this thread's staged vector k of tensor ten (0 x, 1 dy, 2 z).
+// next row starts), pass 1 stores dz, adds the row's dw contributions
+// dy*xh*a(z) to acc when add_dw and keeps only g*dy of each element, and
+// pass 2 reads x again and recomputes xh -- the same operations on the same
+// values, so the same bits as bwd_row.  `stg(ten, k)` is this thread's staged
+// vector k of tensor ten (0 x, 1 dy, 2 z).
 template <int DT, int T, int K, int ACT, bool EXACT, bool RESID, typename G, typename Stg>
 __device__ __forceinline__ void bwd_row_lean(const BwdArgs& a, const G& gain, Stg stg,
                                              float rs_staged, bool have_rstd, int64_t row,
@@ -673,11 +623,12 @@ __device__ __forceinline__ void bwd_row_lean(const BwdArgs& a, const G& gain, St
     rs = rsqrtf(__fadd_rn(mean_of(ss[0], a.H, a.inv_h, a.h_pow2), a.eps));
   }
   const float2 rs2 = bc2(rs);
-  float2 sg[K][GATED ? VE / 2 : 1];
-  // g*dy and xh of vector k (recomputed in both passes from the staged row)
-  auto terms = [&](int k, float2 (&gd)[VE / 2], float2 (&xh)[VE / 2], float2 (&df)[VE / 2],
-                   float2 (&zf)[VE / 2], float2 (&gk)[VE / 2], bool first) {
-    float2 xf[VE / 2];
+  const int64_t off = row * nv + t;
+  float2 gdk[K][VE / 2];   // g*dy, kept for pass 2
+  // pass 1 for vector k: xh, g*dy (kept); dz stored and the dw contribution
+  // dy*xh*a(z) added to acc (neither depends on the row's dot product)
+  auto terms = [&](int k, float2 (&xh)[VE / 2]) {
+    float2 xf[VE / 2], df[VE / 2], zf[VE / 2], gk[VE / 2], dzv[VE / 2];
     F::unpack2(*stg(0, k), xf);
     F::unpack2(*stg(1, k), df);
     if constexpr (GATED) F::unpack2(*stg(2, k), zf);
@@ -685,31 +636,40 @@ __device__ __forceinline__ void bwd_row_lean(const BwdArgs& a, const G& gain, St
 #pragma unroll
     for (int q = 0; q < VE / 2; ++q) {
       xh[q] = mul2(xf[q], rs2);
-      float2 g;
+      const float2 qv = mul2(df[q], xh[q]);                          // dy * xh
+      float2 d;
       if constexpr (GATED) {
-        if (first) sg[k][q] = sigmoid2(zf[q]);
-        g = mul2(gk[q], gate2<ACT>(zf[q], sg[k][q]));   // u * a(z)
+        const float2 sv = sigmoid2(zf[q]);
+        const float2 ga = gate2<ACT>(zf[q], sv);                     // a(z)
+        const float2 uap = mul2(gk[q], mul2(sv, gate_slope_over_s2<ACT>(zf[q], sv)));   // u * a'(z)
+        gdk[k][q] = mul2(mul2(gk[q], ga), df[q]);                    // u * a(z) * dy
+        dzv[q] = mul2(qv, uap);                                      // dy*xh*(u*a'(z))
+        d = mul2(qv, ga);                                            // dy*xh*a(z)
       } else {
-        g = gk[q];                                      // u
+        gdk[k][q] = mul2(gk[q], df[q]);                              // u * dy
+        d = qv;
       }
-      gd[q] = mul2(g, df[q]);
+      if (add_dw && (EXACT || k * T + t < nv)) acc[k][q] = add2(acc[k][q], d);
+    }
+    if constexpr (GATED) {
+      if (act && (EXACT || k * T + t < nv)) st_stream(a.dz + off + k * T, F::pack2v(dzv));
     }
   };
-  // pass 1: per-vector dot chains (two vectors per pair instruction, each lane
-  // its own ascending chain, as vector_dots), then the pairwise tree
+  // per-vector dot chains (two vectors per pair instruction, each lane its own
+  // ascending chain, as vector_dots), then the pairwise tree
   float dp[K];
 #pragma unroll
   for (int k = 0; k < K; k += 2) {
-    float2 gd0[VE / 2], xh0[VE / 2], df0[VE / 2], zf0[VE / 2], gk0[VE / 2];
-    terms(k, gd0, xh0, df0, zf0, gk0, true);
+    float2 xh0[VE / 2];
+    terms(k, xh0);
     if (k + 1 < K) {
-      float2 gd1[VE / 2], xh1[VE / 2], df1[VE / 2], zf1[VE / 2], gk1[VE / 2];
-      terms(k + 1, gd1, xh1, df1, zf1, gk1, true);
+      float2 xh1[VE / 2];
+      terms(k + 1, xh1);
       float2 c = bc2(-0.0f);
 #pragma unroll
       for (int q = 0; q < VE / 2; ++q) {
-        c = fma2(make_float2(gd0[q].x, gd1[q].x), make_float2(xh0[q].x, xh1[q].x), c);
-        c = fma2(make_float2(gd0[q].y, gd1[q].y), make_float2(xh0[q].y, xh1[q].y), c);
+        c = fma2(make_float2(gdk[k][q].x, gdk[k + 1][q].x), make_float2(xh0[q].x, xh1[q].x), c);
+        c = fma2(make_float2(gdk[k][q].y, gdk[k + 1][q].y), make_float2(xh0[q].y, xh1[q].y), c);
       }
       dp[k] = (EXACT || k * T + t < nv) ? c.x : -0.0f;
       dp[k + 1] = (EXACT || (k + 1) * T + t < nv) ? c.y : -0.0f;
@@ -717,8 +677,8 @@ __device__ __forceinline__ void bwd_row_lean(const BwdArgs& a, const G& gain, St
       float c = -0.0f;
 #pragma unroll
       for (int q = 0; q < VE / 2; ++q) {
-        c = __fmaf_rn(gd0[q].x, xh0[q].x, c);
-        c = __fmaf_rn(gd0[q].y, xh0[q].y, c);
+        c = __fmaf_rn(gdk[k][q].x, xh0[q].x, c);
+        c = __fmaf_rn(gdk[k][q].y, xh0[q].y, c);
       }
       dp[k] = (EXACT || k * T + t < nv) ? c : -0.0f;
     }
@@ -726,29 +686,15 @@ __device__ __forceinline__ void bwd_row_lean(const BwdArgs& a, const G& gain, St
   float dot[1] = {pairwise_tree<K>(dp)};
   team_sum<T, 1>(dot, red, phase, team, NT, mask);
   const float2 m2 = bc2(mean_of(dot[0], a.H, a.inv_h, a.h_pow2));
-  // pass 2: dx, dz stores and the dw contributions
-  const int64_t off = row * nv + t;
+  // pass 2: dx, with xh recomputed from the staged x
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     if (act && (EXACT || k * T + t < nv)) {
-      float2 gd[VE / 2], xh[VE / 2], df[VE / 2], zf[VE / 2], gk[VE / 2];
-      terms(k, gd, xh, df, zf, gk, false);
-      float2 dxv[VE / 2], dzv[VE / 2];
+      float2 xf[VE / 2], dxv[VE / 2];
+      F::unpack2(*stg(0, k), xf);
 #pragma unroll
-      for (int q = 0; q < VE / 2; ++q) {
-        dxv[q] = mul2(rs2, fma2(neg2(xh[q]), m2, gd[q]));        // rstd*(g*dy - xh*m)
-        const float2 qv = mul2(df[q], xh[q]);                    // dy * xh
-        float2 d;
-        if constexpr (GATED) {
-          const float2 sv = sg[k][q];
-          const float2 uap = mul2(gk[q], mul2(sv, gate_slope_over_s2<ACT>(zf[q], sv)));
-          dzv[q] = mul2(qv, uap);                                // dy*xh*(u*a'(z))
-          d = mul2(qv, gate2<ACT>(zf[q], sv));                   // dy*xh*a(z)
-        } else {
-          d = qv;
-        }
-        if (add_dw) acc[k][q] = add2(acc[k][q], d);
-      }
+      for (int q = 0; q < VE / 2; ++q)
+        dxv[q] = mul2(rs2, fma2(neg2(mul2(xf[q], rs2)), m2, gdk[k][q]));   // rstd*(g*dy - xh*m)
       if constexpr (RESID) {   // dx = dnorm + dres, rounded once
         float2 rf[VE / 2];
         F::unpack2(__ldcs(a.dres + off + k * T), rf);
@@ -756,15 +702,15 @@ __device__ __forceinline__ void bwd_row_lean(const BwdArgs& a, const G& gain, St
         for (int q = 0; q < VE / 2; ++q) dxv[q] = add2(dxv[q], rf[q]);
       }
       st_stream(a.dx + off + k * T, F::pack2v(dxv));
-      if constexpr (GATED) st_stream(a.dz + off + k * T, F::pack2v(dzv));
     }
   }
 }
 
 // ---------------------------------------------------------------------------
 // Backward: one team per 32-row leaf, rows in ascending order.  x, dy (z) and
-// rstd are staged S-1 rows ahead; pass 1 keeps xh, g*dy and s in registers for
-// pass 2 (dx, dz stores and the leaf's dw fold).  The CTA's leaves (an aligned
+// rstd are staged S-1 rows ahead; pass 1 stores dz and forms the dw
+// contributions, pass 2 the dx (bwd_row, or bwd_row_lean for the wide teams
+// lean_bwd picks), and the leaf's dw fold follows the row.  The CTA's leaves (an aligned
 // power-of-two group) are joined by the pairwise tree; one partial per CTA.
 //   g = u * a(z);  m = mean(g * dy * xh);  dx = rstd * (g*dy - xh*m)
 //   dz = dy * xh * u * a'(z);  dw leaf += dy * xh * a(z)
