@@ -297,7 +297,7 @@ def run_ours(a):
     # without graphs, every step of the timed loop)
     ev = [[torch.cuda.Event(enable_timing=True, external=not a.no_graph) for _ in range(3)]
           for _ in range(G)]
-    graph = graph_ev = None
+    graph = graph_ev = graph_fwd_only = graph_bwd_only = None
     if not a.no_graph:
         # graph: G steps of calls only; it is what the timed region replays K / G times.
         # graph_ev: the same G steps with event records between the calls.
@@ -324,6 +324,21 @@ def run_ours(a):
 
         graph = capture(False)
         graph_ev = capture(True)
+
+        def capture_one(call, off):
+            # G calls of one direction back to back, buffer sets rotating
+            g = torch.cuda.CUDAGraph()
+            cap.wait_stream(stream)
+            with torch.cuda.graph(g, stream=cap):
+                for j in range(G):
+                    st_ = call(P[(j + off) % nsets], cap.cuda_stream)
+                    if st_:
+                        raise RuntimeError(f"capture failed: status {st_}")
+            stream.wait_stream(cap)
+            return g
+
+        graph_fwd_only = capture_one(fwd, 0)
+        graph_bwd_only = capture_one(bwd, 2)
         for _ in range(max(1, a.warmup // G)):
             graph.replay()
         torch.cuda.synchronize()
@@ -364,6 +379,19 @@ def run_ours(a):
         torch.cuda.synchronize()
     fwd_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(G)]
     bwd_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(G)]
+    # each direction alone, G calls back to back (launches overlap as in the
+    # step): mean time per call without an event between calls
+    streamed = {}
+    for name, g in (("fwd", graph_fwd_only), ("bwd", graph_bwd_only)):
+        if g is None:
+            continue
+        g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        streamed[name] = e0.elapsed_time(e1) / G
     if dist is not None:
         t = torch.tensor([ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -422,6 +450,13 @@ def run_ours(a):
             "fwd_us": round(1e3 * fwd_mean, 2), "bwd_us": round(1e3 * bwd_mean, 2),
             "fwd_gbs": round(fwd_b / (fwd_mean / 1e3) / 1e9, 1),
             "bwd_gbs": round(achieved, 1),
+            "back_to_back": ({"fwd_us": round(1e3 * streamed["fwd"], 2),
+                              "bwd_us": round(1e3 * streamed["bwd"], 2),
+                              "fwd_gbs": round(fwd_b / streamed["fwd"] / 1e6, 1),
+                              "bwd_gbs": round(bwd_b / streamed["bwd"] / 1e6, 1),
+                              "timing": f"{G} calls of one direction in one graph, buffer sets "
+                                        "rotating, one event pair around the replay"}
+                             if streamed else None),
             "invariance": inv,
             "roofline": {"bound": "hbm",
                          "kernel": "rmsnorm_bwd call (backward kernel + dw fold pass)",

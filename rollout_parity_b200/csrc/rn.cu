@@ -111,56 +111,76 @@ k_fold(const float* __restrict__ in, int64_t n, int H, float* __restrict__ out) 
 }
 
 // The last fold pass when at most kFold1Rows = 1024 partial rows remain: a CTA
-// of 32 warps covers 8 columns.  Warp w takes rows [32w, 32w + 32); its lane
-// (g, c) streams rows [32w + 8g, 32w + 8g + 8) of column c through the binary
-// counter of pending subtrees, the four 8-row subtrees of a warp are joined by
-// shuffles (g with g+1, then the pairs), and the 32 warp results (aligned
-// blocks of 32 rows: perfect subtrees) by the pairwise tree in shared memory.
-// Absent nodes are skipped, never added as zeros.  One launch where k_fold
-// would need two, spread over H/8 CTAs.
+// of W warps covers 8 columns and all the rows.  Warp w takes rows
+// [4Lw, 4Lw + 4L) with L = 256 / W; its lane (g, c) streams rows
+// [4Lw + Lg, 4Lw + Lg + L) of column c through the binary counter of pending
+// subtrees, the four L-row subtrees of a warp are joined by shuffles (g with
+// g+1, then the pairs), and the W warp results (aligned blocks of 4L rows:
+// perfect subtrees) by the pairwise tree in shared memory.  Absent nodes are
+// skipped, never added as zeros.  One launch where k_fold would need two, over
+// H/8 CTAs; W only sets how many lanes share the rows (32 warps of 8 rows a
+// lane when the H/8 CTAs fit one per SM, fewer and longer lanes for wider rows,
+// so the CTAs still fit in one wave), never the tree.
 constexpr int kFold1Rows = 1024;
-__global__ void __launch_bounds__(1024)
+template <int W>
+__global__ void __launch_bounds__(32 * W)
 k_fold1(const float* __restrict__ in, int64_t n, int H, float* __restrict__ out) {
+  constexpr int L = 256 / W;                // rows a lane streams
+  constexpr int LB = L == 8 ? 3 : (L == 16 ? 4 : 5);
+  static_assert(W * 4 * L == kFold1Rows && (1 << LB) == L, "W in {32, 16, 8}");
   griddep_trigger();
   griddep_wait();      // the partials of the previous kernel are complete and visible
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int cl = lane & 7, g = lane >> 3;
   const int c = blockIdx.x * 8 + cl;
   const bool col_ok = c < H;
-  const int64_t start = int64_t(w) * 32 + int64_t(g) * 8;
+  const int64_t start = (int64_t(w) * 4 + g) * L;
   const int64_t left = n - start;
-  const int cnt = left <= 0 ? 0 : (left >= 8 ? 8 : int(left));
-  float v[8];
+  const int cnt = left <= 0 ? 0 : (left >= L ? L : int(left));
+  float v[L];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = (col_ok && i < cnt) ? __ldcg(in + (start + i) * H + c) : 0.0f;
-  TreeCounter<3, float> tc;
+  for (int i = 0; i < L; ++i) v[i] = (col_ok && i < cnt) ? __ldcg(in + (start + i) * H + c) : 0.0f;
+  TreeCounter<LB, float> tc;
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < L; ++i)
     if (i < cnt) tc.push(i, v[i]);
   float r = cnt > 0 ? tc.finish(cnt) : 0.0f;
-  // the warp's four 8-row subtrees: (g0 + g1), (g2 + g3), then the pairs
-  const int64_t wleft = n - int64_t(w) * 32;
-  const int ng8 = wleft <= 0 ? 0 : (wleft >= 32 ? 4 : int((wleft + 7) / 8));   // present subtrees
+  // the warp's four L-row subtrees: (g0 + g1), (g2 + g3), then the pairs
+  const int64_t wleft = n - int64_t(w) * 4 * L;
+  const int ng = wleft <= 0 ? 0 : (wleft >= 4 * L ? 4 : int((wleft + L - 1) / L));   // present
   const float r1 = __shfl_down_sync(0xffffffffu, r, 8);
-  if ((g & 1) == 0 && g + 1 < ng8) r = __fadd_rn(r, r1);
+  if ((g & 1) == 0 && g + 1 < ng) r = __fadd_rn(r, r1);
   const float r2 = __shfl_down_sync(0xffffffffu, r, 16);
-  if (g == 0 && 2 < ng8) r = __fadd_rn(r, r2);
-  __shared__ float sm[32][8];
+  if (g == 0 && 2 < ng) r = __fadd_rn(r, r2);
+  __shared__ float sm[W][8];
   if (g == 0) sm[w][cl] = r;
   __syncthreads();
   if (w == 0 && g == 0 && col_ok) {
-    const int nw = int((n + 31) / 32);
-    float p[32];
+    const int nw = int((n + 4 * L - 1) / (4 * L));
+    float p[W];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) p[i] = sm[i][cl];
+    for (int i = 0; i < W; ++i) p[i] = sm[i][cl];
 #pragma unroll
-    for (int sft = 1; sft < 32; sft <<= 1) {
+    for (int sft = 1; sft < W; sft <<= 1) {
 #pragma unroll
-      for (int l = 0; l + sft < 32; l += 2 * sft)
+      for (int l = 0; l + sft < W; l += 2 * sft)
         if (l + sft < nw) p[l] = __fadd_rn(p[l], p[l + sft]);
     }
     out[c] = p[0];
   }
+}
+
+// k_fold1 for width H: the most warps per CTA (32, 16, 8) whose H/8 CTAs all
+// fit on the GPU at once.
+rn_status launch_fold1(const float* in, int64_t n, int H, float* out, cudaStream_t st) {
+  static KernelPrep p32, p16;
+  const int64_t ctas = (H + 7) / 8;
+  const dim3 grid{static_cast<unsigned>(ctas)};
+  if (ctas <= int64_t(prepare_kernel(k_fold1<32>, 1024, 0, p32)) * sm_count())
+    return launch_pdl(k_fold1<32>, grid, dim3(1024), 0, st, in, n, H, out);
+  if (ctas <= int64_t(prepare_kernel(k_fold1<16>, 512, 0, p16)) * sm_count())
+    return launch_pdl(k_fold1<16>, grid, dim3(512), 0, st, in, n, H, out);
+  return launch_pdl(k_fold1<8>, grid, dim3(256), 0, st, in, n, H, out);
 }
 
 // dw of a call with no rows: every column is the empty sum, -0.0 (the identity
@@ -374,7 +394,7 @@ rn_status run_fold(const float* src, float* a, float* b, int64_t n, int H, float
   while (n > 1) {
     int S = g_fold_rows.load();
     if (use_fold1(n))
-      return launch_pdl(k_fold1, dim3(unsigned((H + 7) / 8)), dim3(1024), 0, st, in, n, H, dw);
+      return launch_fold1(in, n, H, dw, st);
     if (S <= 0) S = fold_rows_default(n);
     const int B = S / kFoldRG;
     const int64_t nout = (n + S - 1) / S;

@@ -144,8 +144,8 @@ rn_status launch_bwd(int act, bool resid, const Sched& s, int lpc, const BwdArgs
                      int64_t groups, cudaStream_t st);
 
 // What prepare_kernel has done for one kernel, per device: the largest dynamic
-// shared-memory size it has allowed there and how many CTAs of that size fit
-// on one SM.  Both are properties of a device, so a process that drives
+// shared-memory size it has allowed there plus one (0: not prepared yet) and
+// how many CTAs of that size fit on one SM.  Both are properties of a device, so a process that drives
 // several GPUs prepares the kernel on each of them.
 constexpr int kMaxDevices = 64;
 struct KernelPrep {
@@ -165,7 +165,7 @@ int prepare_kernel(Kern kernel, int block, size_t smem, KernelPrep& prep) {
     dev = -1;
   }
   const bool cached = dev >= 0 && dev < kMaxDevices;
-  if (cached && smem <= prep.done[dev].load()) return prep.per_sm[dev].load();
+  if (cached && smem < prep.done[dev].load()) return prep.per_sm[dev].load();
   if (smem > 48 * 1024)
     (void)cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   int nb = 0;
@@ -176,7 +176,7 @@ int prepare_kernel(Kern kernel, int block, size_t smem, KernelPrep& prep) {
   }
   if (cached) {
     prep.per_sm[dev].store(nb);
-    prep.done[dev].store(smem);
+    prep.done[dev].store(smem + 1);
   }
   return nb;
 }

@@ -1000,8 +1000,13 @@ rn_status launch_stripe(const Sched& s, int lpc, const BwdArgs& a, int64_t group
   const size_t smem = bwd_stripe_smem_bytes(s, a.H, ACT != kActNone, rn_dtype(DT));
   static KernelPrep prep;
   (void)prepare_kernel(k_bwd_stripe<DT, T, K, ACT, RESID, XJ>, 32, smem, prep);
-  return launch_pdl(k_bwd_stripe<DT, T, K, ACT, RESID, XJ>, dim3(grid_cap(groups)), dim3(32),
-                    smem, st, a, lpc);
+  // An ordinary launch, not a programmatic dependent one: the grid is about one
+  // wave of single-warp CTAs (7 an SM at 262144 x 128), and CTAs started early
+  // pile onto the SMs with room while the previous kernel drains -- up to the
+  // register limit of 8 to 12 an SM -- so the most loaded SMs set the time.
+  // Started on an idle GPU they spread evenly.
+  k_bwd_stripe<DT, T, K, ACT, RESID, XJ><<<dim3(grid_cap(groups)), dim3(32), smem, st>>>(a, lpc);
+  return launch_status();
 }
 
 template <int DT, int T, int K, int ACT, bool EXACT, bool RESID>

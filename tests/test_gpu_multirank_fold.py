@@ -61,8 +61,10 @@ def test_fold_rows_rejects_bad_counts(cuda_lib):
 
 # --- any split on 256-row chunk boundaries ------------------------------------
 @pytest.mark.parametrize("n", [1, 2, 9, 256, 257, 1000, 1025, 2049, 3000, 70000])
-@pytest.mark.parametrize("width", [8, 128, 2056])
+@pytest.mark.parametrize("width", [8, 128, 2056, 4104, 5120])
 def test_fold_tree_is_the_declared_tree(cuda_lib, n, width):
+    # 257..1024 rows take the one-pass fold, whose CTAs have 32, 16 or 8 warps
+    # as the width needs (128, 2056: 32; 4104: 16; 5120: 8 on a 148-SM B200)
     if n * width > 70000 * 128:
         pytest.skip("kept to a few MB")
     rng = np.random.default_rng(n + width)
