@@ -506,6 +506,11 @@ def invariance_checks(rn, s, R, H, eps, wl):
 
 
 def run_e2e(rn, wl, dev, steps, step_b, world, dist):
+    """Steps through the public API with every step's inputs copied in from
+    pinned host memory and its results copied out, inside the timed region.
+    On one GPU two device buffer sets alternate, so step k's inputs go in (on
+    one stream) while step k-1's results come out (on another): the host link
+    carries both directions at once.  With N ranks each step runs in order."""
     R, H, eps = wl.rows, wl.width, wl.eps
     gated = wl.gated
     pin = lambda t: t.pin_memory()
@@ -514,55 +519,92 @@ def run_e2e(rn, wl, dev, steps, step_b, world, dist):
     oy, ors = torch.empty_like(hx).pin_memory(), torch.empty(R, dtype=torch.float32).pin_memory()
     odx, odz = torch.empty_like(hx).pin_memory(), torch.empty_like(hx).pin_memory()
     odw = torch.empty(H, dtype=torch.float32).pin_memory()
-    x = torch.empty_like(hx, device=dev)
-    z = torch.empty_like(hx, device=dev)
-    dy = torch.empty_like(hx, device=dev)
-    w = torch.empty_like(hw, device=dev)
-    y = torch.empty_like(x)
-    rstd = torch.empty(R, dtype=torch.float32, device=dev)
-    dx, dz = torch.empty_like(x), torch.empty_like(x)
-    dw = torch.empty(H, dtype=torch.float32, device=dev)
-    ws = rn.workspace(R, H, dev)
+    nbuf = 2 if dist is None else 1
+
+    def dev_set():
+        d = {"x": torch.empty_like(hx, device=dev), "dy": torch.empty_like(hx, device=dev),
+             "w": torch.empty_like(hw, device=dev), "rstd": torch.empty(R, dtype=torch.float32,
+                                                                        device=dev),
+             "dw": torch.empty(H, dtype=torch.float32, device=dev),
+             "z": torch.empty_like(hx, device=dev) if gated else None,
+             "ws": rn.workspace(R, H, dev)}
+        d["y"], d["dx"] = torch.empty_like(d["x"]), torch.empty_like(d["x"])
+        d["dz"] = torch.empty_like(d["x"]) if gated else None
+        return d
+
+    bufs = [dev_set() for _ in range(nbuf)]
     h2d = sum(t.numel() * t.element_size() for t in (hx, hz, hdy, hw) if t is not None)
     d2h = sum(t.numel() * t.element_size() for t in ((oy, ors, odx, odz, odw) if gated else
                                                      (oy, ors, odx, odw)))
-
-    def step():
-        x.copy_(hx, non_blocking=True)
-        if gated:
-            z.copy_(hz, non_blocking=True)
-        dy.copy_(hdy, non_blocking=True)
-        w.copy_(hw, non_blocking=True)
-        zz = z if gated else None
-        rn.rmsnorm_fwd(x, w, eps, wl.weight_offset, zz, wl.act, y=y, rstd=rstd)
-        if dist is None:
-            rn.rmsnorm_bwd(x, w, dy, rstd, eps, wl.weight_offset, zz, wl.act, dx=dx,
-                           dz=dz if gated else None, dw=dw, ws=ws)
-            odw.copy_(dw, non_blocking=True)
-        else:   # with N ranks the step's dw is the whole batch's (chunk partials folded)
-            _, _, ch = rn.rmsnorm_bwd_chunks(x, w, dy, rstd, eps, wl.weight_offset, zz, wl.act,
-                                             dx=dx, dz=dz if gated else None, ws=ws)
-            odw.copy_(chunk_split_dw(ch, R, rows_per_rank=rows_per_rank), non_blocking=True)
-        oy.copy_(y, non_blocking=True)
-        ors.copy_(rstd, non_blocking=True)
-        odx.copy_(dx, non_blocking=True)
-        if gated:
-            odz.copy_(dz, non_blocking=True)
-
     if dist is not None:
         from rollout_parity_b200.parallel import check_chunk_split, chunk_split_dw
         rows_per_rank = check_chunk_split(R, device=dev)
-    for _ in range(3):
-        step()
+    main = torch.cuda.current_stream(dev)
+    s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3)) if dist is None else \
+        (main, main, main)
+    ev = lambda: torch.cuda.Event()
+    computed = [ev() for _ in range(nbuf)]       # the set's compute is done (inputs free)
+    outputs_free = [ev() for _ in range(nbuf)]   # the copy-out that read the set is done
+    copied_in = [ev() for _ in range(nbuf)]
+    for e_ in computed + outputs_free:
+        e_.record(main)
+
+    def step(k):
+        b = k % nbuf
+        d = bufs[b]
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(computed[b])
+            d["x"].copy_(hx, non_blocking=True)
+            if gated:
+                d["z"].copy_(hz, non_blocking=True)
+            d["dy"].copy_(hdy, non_blocking=True)
+            d["w"].copy_(hw, non_blocking=True)
+            copied_in[b].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(copied_in[b])
+            s_cmp.wait_event(outputs_free[b])
+            zz = d["z"]
+            rn.rmsnorm_fwd(d["x"], d["w"], eps, wl.weight_offset, zz, wl.act, y=d["y"],
+                           rstd=d["rstd"])
+            if dist is None:
+                rn.rmsnorm_bwd(d["x"], d["w"], d["dy"], d["rstd"], eps, wl.weight_offset, zz,
+                               wl.act, dx=d["dx"], dz=d["dz"], dw=d["dw"], ws=d["ws"])
+                dw_out = d["dw"]
+            else:   # with N ranks the step's dw is the whole batch's (chunk partials folded)
+                _, _, ch = rn.rmsnorm_bwd_chunks(d["x"], d["w"], d["dy"], d["rstd"], eps,
+                                                 wl.weight_offset, zz, wl.act, dx=d["dx"],
+                                                 dz=d["dz"], ws=d["ws"])
+                dw_out = chunk_split_dw(ch, R, rows_per_rank=rows_per_rank)
+            computed[b].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(computed[b])
+            odw.copy_(dw_out, non_blocking=True)
+            oy.copy_(d["y"], non_blocking=True)
+            ors.copy_(d["rstd"], non_blocking=True)
+            odx.copy_(d["dx"], non_blocking=True)
+            if gated:
+                odz.copy_(d["dz"], non_blocking=True)
+            outputs_free[b].record(s_out)
+
+    def join():
+        for s_ in (s_in, s_cmp, s_out):
+            main.wait_stream(s_)
+
+    for k in range(3):
+        step(k)
+    join()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
         torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(steps):
-        step()
-    e.record()
+    s.record(main)
+    for s_ in (s_in, s_cmp, s_out):
+        s_.wait_stream(main)
+    for k in range(steps):
+        step(k)
+    join()
+    e.record(main)
     torch.cuda.synchronize()
     ms = s.elapsed_time(e)
     if dist is not None:
@@ -572,6 +614,9 @@ def run_e2e(rn, wl, dev, steps, step_b, world, dist):
     return {"value": round(world * step_b * steps / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 4),
+            "overlap": ("inputs of step k copied in while step k-1's results are copied out "
+                        "(two device buffer sets, three streams)" if dist is None else
+                        "none: copy in, compute, copy out in order"),
             "api": "rollout_parity_b200.rmsnorm_fwd/rmsnorm_bwd" if dist is None else
                    "rollout_parity_b200.rmsnorm_fwd/rmsnorm_bwd_chunks + parallel.chunk_split_dw"}
 
