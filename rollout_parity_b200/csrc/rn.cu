@@ -637,7 +637,7 @@ size_t fwd_smem_bytes(const Sched& s, bool gated, bool resid, rn_dtype dt) {
   const size_t W = s.T > 32 ? s.T / 32 : 1;
   const size_t red = s.T > 32 ? 2 * NT * W * sizeof(float) : 0;
   const size_t gain = gain_src_of(s.T, s.K, int(VE)) == kGainSmem ? size_t(s.K) * s.T * VE * sizeof(float) : 0;
-  return red + gain + size_t(fwd_stages_of(s.T)) * (1 + gated + resid) * s.K * B * 16;
+  return red + gain + size_t(fwd_stages_of(s.T, gated, resid, int(VE))) * (1 + gated + resid) * s.K * B * 16;
 }
 
 }  // namespace rn_detail

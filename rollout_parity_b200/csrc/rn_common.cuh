@@ -72,7 +72,15 @@ __host__ __device__ constexpr int fwd_block_of(int T, int K) {
 __host__ __device__ constexpr int fwd_min_blocks_of(int T, int K) {
   return T <= 16 ? (K <= 2 ? 4 : 8) : 1;
 }
-__host__ __device__ constexpr int fwd_stages_of(int T) { return T <= 32 ? 3 : (T <= 512 ? 2 : 1); }
+// Forward staging depth (rows in flight per team): three for sub-warp and
+// one-warp teams; three also for the gated 16-bit 128-thread teams without the
+// residual (H = 1032 to 8192 in bf16/fp16, x and z staged), where a third row
+// ahead measured faster (16384 x 2048 silu 41.4 -> 39.4 us, 16384 x 5120
+// 100.8 -> 86.5 us) while it slowed the ungated and fp32 rows of the same
+// teams; two up to 512 threads, else one.
+__host__ __device__ constexpr int fwd_stages_of(int T, bool gated, bool resid, int VE) {
+  return T <= 32 ? 3 : ((T == 128 && gated && !resid && VE == 8) ? 3 : (T <= 512 ? 2 : 1));
+}
 __host__ __device__ constexpr int bwd_max_block_of(int T) {
   return T <= 32 ? 8 * T : (T <= 128 ? 256 : T);
 }

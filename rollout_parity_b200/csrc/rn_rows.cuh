@@ -387,7 +387,7 @@ k_fwd(const FwdArgs a) {
   using F = Fmt<DT>;
   constexpr bool GATED = ACT != kActNone;
   constexpr int VE = F::VE;
-  constexpr int S = fwd_stages_of(T);
+  constexpr int S = fwd_stages_of(T, GATED, RESID, VE);
   constexpr int NTEN = 1 + GATED + RESID;   // staged tensors: x (, z) (, r)
   constexpr int TR = GATED ? 2 : 1;         // slot of r
   constexpr int B = fwd_block_of(T, K);

@@ -106,8 +106,10 @@ def fwd_block(t, k):
     return (128 if k <= 2 else 64) if t <= 16 else (128 if t == 32 else t)
 
 
-def fwd_stages(t):
-    return 3 if t <= 32 else (2 if t <= 512 else 1)
+def fwd_stages(t, gated, resid, ve):
+    if t <= 32 or (t == 128 and gated and not resid and ve == 8):
+        return 3
+    return 2 if t <= 512 else 1
 
 
 def bwd_stages(t, k, gated=True):
@@ -124,12 +126,12 @@ def gain_in_smem(t, k, ve):
     return t <= 16 or (k * ve > 16 and t * k * ve <= 8192)
 
 
-def fwd_smem(t, k, ve, tensors):
+def fwd_smem(t, k, ve, gated, resid):
     b = fwd_block(t, k)
     nt, w = b // t, (t // 32 if t > 32 else 1)
     red = 2 * nt * w * 4 if t > 32 else 0
     gain = k * t * ve * 4 if gain_in_smem(t, k, ve) else 0
-    return red + gain + fwd_stages(t) * tensors * k * b * 16
+    return red + gain + fwd_stages(t, gated, resid, ve) * (1 + gated + resid) * k * b * 16
 
 
 def bwd_smem(t, k, ve, lpc, width, tensors):
@@ -157,8 +159,9 @@ def test_every_shape_fits_shared_memory(ve):
     worst = 0
     for width in range(8, 16385, 8):
         t, k = fwd_shape(width, ve)
-        for tensors in (1, 2, 3):            # x; + z or r; + both
-            worst = max(worst, fwd_smem(t, k, ve, tensors))
+        for gated in (False, True):          # x; + z; + r; + both
+            for resid in (False, True):
+                worst = max(worst, fwd_smem(t, k, ve, gated, resid))
         tb, kb = bwd_shape(width, ve)
         stripe = width // ve == tb * kb and tb <= 8 and (tb * kb * ve) % 128 == 0
         if stripe:                            # gain, stages, rstd stages, transpose buffer
