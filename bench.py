@@ -417,6 +417,14 @@ def run_ours(a):
         bwd_mean = float(np.mean(bwd_ms))
         fwd_mean = float(np.mean(fwd_ms))
         achieved = bwd_b / (bwd_mean / 1e3) / 1e9
+        # the roofline's time per call: G calls back to back (as the timed
+        # region runs them: no event between calls), else the per-call events
+        if "bwd" in streamed:
+            rl_gbs = bwd_b / (streamed["bwd"] / 1e3) / 1e9
+            rl_timing = (f"{G} calls back to back in one graph, buffer sets rotating, one "
+                         "event pair around them")
+        else:
+            rl_gbs, rl_timing = achieved, "CUDA events around each call in the timed loop"
         traffic = profiled_traffic(a.workload)
         desc = {WORKLOAD: {"layout": "8192 tokens x 32 heads, row = token*32 + head",
                            "outliers": "1% of channels x50 in x, z, dy"}}.get(a.workload, {})
@@ -460,8 +468,12 @@ def run_ours(a):
             "invariance": inv,
             "roofline": {"bound": "hbm",
                          "kernel": "rmsnorm_bwd call (backward kernel + dw fold pass)",
-                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "peak_source": src,
+                         "timing": rl_timing,
+                         "achieved": round(rl_gbs, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(rl_gbs / peak, 4), "peak_source": src,
+                         "per_call": {"achieved": round(achieved, 1),
+                                      "frac": round(achieved / peak, 4),
+                                      "timing": "CUDA events around each call (bwd_us)"},
                          "traffic": traffic, "algorithmic_bytes": bwd_b},
             "cpu_baseline": cpu, "accuracy": acc, "e2e": e2e, "gpu_launches": launches,
             "clocks": clk,
