@@ -119,8 +119,8 @@ k_fold(const float* __restrict__ in, int64_t n, int H, float* __restrict__ out) 
 // perfect subtrees) by the pairwise tree in shared memory.  Absent nodes are
 // skipped, never added as zeros.  One launch where k_fold would need two, over
 // H/8 CTAs; W only sets how many lanes share the rows (32 warps of 8 rows a
-// lane when the H/8 CTAs fit one per SM, fewer and longer lanes for wider rows,
-// so the CTAs still fit in one wave), never the tree.
+// lane while the H/8 CTAs all fit on the GPU at once, fewer and longer lanes
+// for wider rows, so that they still do), never the tree.
 constexpr int kFold1Rows = 1024;
 template <int W>
 __global__ void __launch_bounds__(32 * W)
