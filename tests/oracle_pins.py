@@ -335,6 +335,36 @@ def pin_general_finite_differences(orc):
                 _close(dz, _fd(lambda a: L(x, a, w), z), rtol=1e-7, atol=1e-8, what=tag + " dz")
 
 
+def pin_autograd_gradients(orc):
+    """dx, dz, dw of every (activation, offset) equal torch.autograd's gradient
+    (fp64, CPU) of L = sum(y * dy) for the forward written here in torch ops
+    (not the oracle's): exact up to rounding, so a bound about a million times
+    tighter than the finite differences above."""
+    import torch
+    rng = np.random.default_rng(23)
+    R, H, eps = 3, 16, 1e-3
+    x = rng.normal(size=(R, H)); z = rng.normal(size=(R, H)) * 3.0
+    w = rng.normal(size=H); dy = rng.normal(size=(R, H))
+    for act in ("none", "silu", "sigmoid"):
+        for off in (0.0, 1.0, 0.5):
+            xt, zt, wt = (torch.tensor(a, dtype=torch.float64, requires_grad=True)
+                          for a in (x, z, w))
+            y = xt * torch.rsqrt((xt * xt).mean(dim=1, keepdim=True) + eps) * (wt + off)
+            if act == "silu":
+                y = y * (zt * torch.sigmoid(zt))
+            elif act == "sigmoid":
+                y = y * torch.sigmoid(zt)
+            loss = (y * torch.tensor(dy, dtype=torch.float64)).sum()
+            gx, gz, gw = torch.autograd.grad(loss, [xt, zt, wt], allow_unused=True)
+            dx, dz, dw = orc.rmsnorm_bwd(x, w, dy, eps, off, None if act == "none" else z, act)
+            tag = f"{act} offset {off}"
+            for got, want, n in ((dx, gx, "dx"), (dw, gw, "dw")) + \
+                    (((dz, gz, "dz"),) if act != "none" else ()):
+                want = want.detach().numpy()
+                _close(got, want, rtol=1e-11, atol=1e-13 * float(np.max(np.abs(want))),
+                       what=f"{tag} {n} vs autograd")
+
+
 def pin_signed_zero_weight(orc):
     """The offset is added only when it is nonzero, so with offset 0 a -0.0
     weight stays -0.0 and flips the sign of the zero it multiplies into (y and
@@ -650,6 +680,7 @@ ALL_PINS = [
     pin_worked_example_sigmoid_offset,
     pin_general_special_cases,
     pin_general_finite_differences,
+    pin_autograd_gradients,
     pin_signed_zero_weight,
     pin_row_mask,
     pin_round_to_format,
