@@ -89,3 +89,28 @@ def test_one_stream_per_call_in_turn(cuda_lib):
         for k in KEYS:
             if ref[k] is not None:
                 assert torch.equal(bits(out[k]), bits(ref[k])), k
+
+
+@pytest.mark.parametrize("case", [CASES[0], CASES[1], CASES[2]],
+                         ids=["stripe", "k_bwd", "lean-f16"])
+def test_graph_replay_gives_the_eager_bits(cuda_lib, case):
+    """The calls captured into a CUDA graph (as bench.py replays them) and the
+    graph replayed give the bits of the calls made eagerly."""
+    dev = torch.device("cuda:0")
+    wl = workloads.make(seed=77, **case).to(dev)
+    ref = run(cuda_lib, wl)
+    torch.cuda.synchronize()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(torch.cuda.current_stream(dev))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        out = run(cuda_lib, wl)
+    for _ in range(3):
+        for k in KEYS:
+            if out[k] is not None:
+                out[k].fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        for k in KEYS:
+            if ref[k] is not None:
+                assert torch.equal(bits(out[k]), bits(ref[k])), (case, k)
