@@ -766,11 +766,12 @@ const char* rn_describe(int32_t width, rn_dtype dt) {
   std::snprintf(t_describe, sizeof t_describe,
                 "backend=cuda-sm100a lib=librn kernels=k_fwd,%s,k_fold,k_fold1 dtype=%s width=%d "
                 "acc=fp32 team_threads=%d vectors_per_thread=%d elems_per_vector=%d "
+                "bwd_team_threads=%d bwd_vectors_per_thread=%d "
                 "thread_order=ascending-fma-from-neg0 lane_join=xor-butterfly(%d..1) "
                 "warp_join=%s dw_tree=leaf32-ascending-fold+level-pairwise "
                 "leaves_per_cta(262144_rows)=%d fast_math=off atomics=none",
                 stripe ? "k_bwd_stripe" : "k_bwd", dtype_name(dt), width, s.T, s.K, vec_elems(dt),
-                (s.T < 32 ? s.T : 32) / 2,
+                sb.T, sb.K, (s.T < 32 ? s.T : 32) / 2,
                 s.T > 32 ? "smem-pairwise" : "none", lpc);
   return t_describe;
 }

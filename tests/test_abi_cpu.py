@@ -347,8 +347,12 @@ def test_workspace_bytes_invalid(lib):
                                            (5120, DType.F16, 128), (2048, DType.F16, 128)])
 def test_describe(lib, width, dt, team):
     d = lib.rn_describe(width, dt).decode()
-    assert f"team_threads={team} " in d
+    assert f" team_threads={team} " in d
     assert "acc=fp32" in d and "atomics=none" in d and "fast_math=off" in d
+    # the backward runs the forward's team, except 16-bit rows of 128 (4 x 4, the
+    # forward's 8 x 2 order)
+    bwd = 4 if (width == 128 and dt in (DType.BF16, DType.F16)) else team
+    assert f" bwd_team_threads={bwd} " in d
 
 
 def test_describe_unsupported(lib):
